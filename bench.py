@@ -1,0 +1,348 @@
+"""Benchmark of the quantized MoE expert layer on B200.
+
+Default workload: the Mixtral-8x7B-shaped decode layer (E=8, top-2, d_model
+4096, d_ff 14336, SwiGLU, INT3 group-128 asymmetric codes, rank-32
+compensators on both blocks) with T=64 tokens per step. One step is one full
+forward pass (routing, permute, compensator down-projections, gate/up GEMM +
+SwiGLU, down GEMM, combine) through the C ABI.
+
+Prints ONE JSON line (rank 0). Multi-GPU: one process per GPU (torchrun); each
+rank runs an independent replica on its own token batch (the layer has no
+exchange step on one node in this build), so scaling is weak and the value is
+the total tokens/s of all ranks, timed on the device as the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this method
+has) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "mixtral8x7b_decode"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--config", default="mixtral_decode")
+    p.add_argument("--tokens", type=int, default=64)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=20.0)
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work
+# ---------------------------------------------------------------------------
+
+def block_bytes(cfg, spec, block):
+    M, Kin = (2 * cfg.N, cfg.K) if block == 0 else (cfg.K, cfg.N)
+    b = spec.bits[block]
+    r = spec.rank
+    if spec.fmt == 0:
+        wb = b * M * Kin / 8 + 4 * M * Kin / spec.group
+    elif spec.fmt == 1:
+        wb = b * M * Kin / 8 + 2 * (1 << b)
+    else:
+        wb = 2 * M * Kin
+    return wb, 2 * r * M, 2 * r * Kin  # codes+scales, B factor, A factor
+
+
+def layer_bytes(cfg, counts, T):
+    """Weights of touched experts (codes, scales/LUT, both factors) + X, logits, Y."""
+    tot = 0.0
+    for e, n in enumerate(counts):
+        if n > 0:
+            for b in (0, 1):
+                wb, bb, ab = block_bytes(cfg, cfg.experts[e], b)
+                tot += wb + bb + ab
+    return tot + 2 * T * cfg.K + 4 * T * cfg.E + 2 * T * cfg.K
+
+
+def gemm1_bytes(cfg, counts):
+    """Algorithmic bytes of one gate/up GEMM launch: codes + scales + B1 of the
+    touched experts, the routed activation rows (K + r columns, fp16) and the
+    SwiGLU output rows (N columns, fp16)."""
+    tot = 0.0
+    for e, n in enumerate(counts):
+        if n > 0:
+            wb, bb, _ = block_bytes(cfg, cfg.experts[e], 0)
+            r = cfg.experts[e].rank
+            tot += wb + bb + 2 * n * (cfg.K + r) + 2 * n * cfg.N
+    return tot
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region (NVML reads only)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        while not self.stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d.get("bf16_tflops"), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------
+
+def cpu_oracle_rate(cfg, blocks_cpu, X, logits, top_k, budget_s):
+    """Times the fp64 oracle on the first tokens of the batch, one token at a
+    time (each token dequantises its own experts), until ``budget_s`` seconds
+    have passed. Returns tokens/s, tokens done, seconds and threads."""
+    import numpy as np
+    import torch
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from moe_testlib import OracleExperts
+    import oracle as orc
+    Xn = X.float().cpu().numpy().astype(np.float64)
+    Ln = logits.cpu().numpy()
+    t0 = time.perf_counter()
+    done = 0
+    for t in range(Xn.shape[0]):
+        orc.moe_forward(Xn, Ln, top_k, OracleExperts(blocks_cpu), cfg.N, rows=[t])
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    threads = torch.get_num_threads()
+    return done / dt, done, dt, threads
+
+
+def build_layer(bq, cfg, blocks, max_tokens):
+    import ctypes
+    descs = [bq.ExpertDesc((ctypes.c_int * 2)(*sp.bits), sp.fmt, sp.group, sp.rank) for sp in cfg.experts[:cfg.E]]
+    L = bq.MoELayer(cfg.E, cfg.K, cfg.N, max_tokens, cfg.top_k, descs)
+    for (e, b), blk in blocks.items():
+        L.set_expert_weights(e, b, blk.codes, blk.scales, blk.zeros_or_lut,
+                             blk.A if blk.rank else None, blk.B if blk.rank else None)
+    return L
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    args = parse()
+    import torch
+    import torch.distributed as dist
+    import moe_synth as ms
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    T = args.tokens
+    cfg = ms.make_config(args.config)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        blocks = {}
+        for e in range(cfg.E):
+            for b in (0, 1):
+                blocks[(e, b)] = ms.make_block(cfg, e, b, device="cpu")
+        X, logits = ms.make_inputs(cfg, T, "cpu")
+        budget = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+        rates = []
+        for i in range(args.warmup + args.steps):
+            r, n, dt, thr = cpu_oracle_rate(cfg, blocks, X, logits, cfg.top_k, budget)
+            if i >= args.warmup:
+                rates.append((r, n, dt, thr))
+        val = statistics.median([r[0] for r in rates])
+        ms_step = 1000.0 * T / val
+        line = {"impl": "reference", "metric": "MoE-layer tokens/s", "value": val, "unit": "tokens/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": f"{WORKLOAD}_T{T}", "T": T},
+                "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": rates[0][3], "kind": "oracle",
+                                 "sample": f"first {rates[0][1]} token(s) of the T={T} batch per step, one token "
+                                           f"at a time (its experts dequantised in fp64)"},
+                "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    from bit_quantized_moe_top_b200 import build
+    build.build()
+    import bit_quantized_moe_top_b200 as bq
+
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+
+    blocks = {}
+    for e in range(cfg.E):
+        for b in (0, 1):
+            blocks[(e, b)] = ms.make_block(cfg, e, b, device=dev)
+    L = build_layer(bq, cfg, blocks, max_tokens=T)
+    X, logits = ms.make_inputs(cfg, T, dev, key_extra=rank)
+    Y = torch.empty_like(X)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step():
+        L.forward(X, logits, cfg.top_k, Y)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert L.sync_status() == 0
+    routing = L.routing(T, cfg.top_k)
+    counts = routing["counts"].cpu().tolist()
+    launches_per_step = L.last_launch_count()
+
+    # timed region: per-step events, L2 flushed (untimed) between steps
+    L.set_profiling(True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    kt = {}
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+            if i % 16 == 0 or i == args.steps - 1:
+                for name, t in L.kernel_times():
+                    kt.setdefault(name, []).append(t)
+        torch.cuda.synchronize()
+    L.set_profiling(False)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    ms_per_step = total_ms / args.steps
+    value = world * T / (ms_per_step / 1000.0)
+
+    # dominant kernel: gate/up GEMM (2/3 of the weight bytes)
+    k1 = statistics.mean(kt.get("decode_gemm_w1_swiglu", [float("nan")]))
+    hbm_peak, _, peak_src = measured_peaks()
+    b1 = gemm1_bytes(cfg, counts)
+    achieved = b1 / (k1 * 1e-3) / 1e9
+    layer_b = layer_bytes(cfg, counts, T)
+    kernel_means = {k: statistics.mean(v) for k, v in kt.items()}
+
+    # end to end: host buffers through moe_layer_forward_host (copies inside the timed region)
+    Xh = X.cpu().pin_memory()
+    Lh = logits.cpu().pin_memory()
+    Yh = torch.empty_like(Xh).pin_memory()
+    for _ in range(3):
+        L.forward_host(Xh, Lh, cfg.top_k, Yh)
+    e2e_steps = max(10, args.steps // 4)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        L.forward_host(Xh, Lh, cfg.top_k, Yh)
+    e2e_s = (time.perf_counter() - t0) / e2e_steps
+    e2e_val = world * T / e2e_s
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            cpu_blocks = {k: ms.BlockWeights(**{**v.__dict__, "codes": v.codes.cpu(),
+                                              "scales": None if v.scales is None else v.scales.cpu(),
+                                              "zeros_or_lut": None if v.zeros_or_lut is None else v.zeros_or_lut.cpu(),
+                                              "A": None if v.A is None else v.A.cpu(),
+                                              "B": None if v.B is None else v.B.cpu()})
+                          for k, v in blocks.items()}
+            r, n, dt, thr = cpu_oracle_rate(cfg, cpu_blocks, X.cpu(), logits.cpu(), cfg.top_k, args.cpu_seconds)
+            cpu = {"value": r, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                   "sample": f"first {n} token(s) of the T={T} batch, one token at a time (its two experts "
+                             f"dequantised in fp64), {dt:.1f} s"}
+        line = {
+            "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16 operands, f32 accumulate",
+            "data": "synthetic",
+            "config": {"workload": f"{WORKLOAD}_T{T}", "T": T, "E": cfg.E, "top_k": cfg.top_k, "d_model": cfg.K,
+                       "d_ff": cfg.N, "bits": 3, "group": 128, "rank": 32, "parallelism": f"replicas x{world}",
+                       "l2": "flushed between steps (256 MiB write, untimed); weights 599 MB > L2"},
+            "layer_hbm_gbs": layer_b / (ms_per_step * 1e-3) / 1e9,
+            "layer_bytes_per_step": layer_b,
+            "roofline": {"bound": "hbm", "kernel": "decode_gemm_w1_swiglu", "achieved": achieved, "peak": hbm_peak,
+                         "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": None,
+                         "peak_source": peak_src, "algorithmic_bytes_per_launch": b1, "launch_ms": k1},
+            "kernels_ms": kernel_means,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": T * cfg.K * 2 + T * cfg.E * 4,
+                    "d2h_bytes_per_step": T * cfg.K * 2},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    L.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,153 @@
+// Shared device definitions of the quantized MoE layer: internal weight and
+// activation layouts, the per-block descriptor, and small PTX helpers.
+//
+// Internal layouts (all built on the device at weight-load time):
+//
+//  * Rows of W1 (gate||up, 2N x K) are interleaved per 16-row fragment:
+//    internal row 16f+i is gate row 8f+i for i < 8 and up row 8f+i-8 for
+//    i >= 8, so one mma.sync accumulator fragment (rows g and g+8) holds the
+//    gate and the up value of the same SwiGLU column.
+//  * Codes are stored per (row fragment rf, 128-wide K chunk kc) in the order a
+//    warp's lanes consume them as mma.m16n8k16 A fragments: lane (g = lane/4,
+//    c = lane%4), step s (0..7, a k16 slice of the chunk), slot j (0..3 = the
+//    A registers a0a1, a2a3, a4a5, a6a7), half h (0/1) is the element
+//    (row 16rf + g + 8*(j&1), k = 128kc + 16s + 2c + 8*(j>>1) + h).
+//    A chunk holds 256*b bytes (b = bits; 16 for dense fp16).
+//  * Activations for the mma.sync path are stored per (8-row tile, 32-wide k
+//    block) as 32 lanes x uint4 = the B fragments of two k16 steps.
+#pragma once
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+namespace moeq {
+
+constexpr int kChunkK = 128;   // K per code chunk
+constexpr int kMaxRank = 64;
+constexpr int kMaxTopK = 8;
+constexpr int kMaxExperts = 256;
+
+enum : int { FMT_INT = 0, FMT_BITPLANE = 1, FMT_DENSE = 2 };
+
+// device status word bits
+enum : unsigned { ST_BOUNDS = 1u, ST_TIMEOUT = 2u, ST_ROUTE = 4u };
+
+// One expert linear block as the kernels see it.
+struct BlockDesc {
+  const uint8_t* codes;   // internal chunked codes (INT / DENSE) or plane 0 (BITPLANE)
+  const uint32_t* sz;     // INT: [MF][K/g][8] uint2 = half2(s, -z*s) for rows g and g+8
+  const uint32_t* lut;    // BITPLANE: 28 fp16 as 14 u32
+  const uint4* bfrag;     // compensator B [M, r] as dense A-fragments [MF][r/16][32] uint4 (fp16)
+  const uint4* afrag;     // compensator A [r, K] as dense A-fragments [r/16][K/16][32] uint4 (fp16)
+  long long plane_stride; // BITPLANE: bytes between planes
+  int fmt, bits, group, rank;
+  int M, K;
+  int loaded;
+  int pad_;
+};
+
+struct ExpertDesc {
+  BlockDesc blk[2];
+};
+
+// ---------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t lop3_sel(uint32_t a, uint32_t b, uint32_t m) {
+  // (a & m) | (b & ~m)
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xE4;\n" : "=r"(d) : "r"(a), "r"(b), "r"(m));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t m, uint32_t o) {
+  // (a & m) | o
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(d) : "r"(a), "r"(m), "r"(o));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(s));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hsub2u(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hfma2u(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
+  uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// layout index helpers (shared by the re-layout kernels and the GEMMs)
+// ---------------------------------------------------------------------------
+
+// canonical row of internal row ir of a block (W1 interleaves gate/up per fragment)
+__host__ __device__ __forceinline__ int canon_row(int ir, int block, int N) {
+  if (block != 0) return ir;
+  int f = ir >> 4, i = ir & 15;
+  return i < 8 ? 8 * f + i : N + 8 * f + (i - 8);
+}
+
+// (row-in-fragment, k-in-chunk) of element (lane, step, slot, half)
+__host__ __device__ __forceinline__ void frag_elem(int lane, int s, int j, int h, int& r, int& k) {
+  int g = lane >> 2, c = lane & 3;
+  r = g + 8 * (j & 1);
+  k = 16 * s + 2 * c + 8 * (j >> 1) + h;
+}
+
+// Activation B-fragment layout: element (row n, col k) of a [rows, Kpad]
+// activation matrix, Kpad % 32 == 0. Returns the fp16 index.
+__host__ __device__ __forceinline__ long long act_frag_index(long long n, int k, int Kpad) {
+  long long nt = n >> 3;
+  int g = (int)(n & 7);
+  int kk = k >> 5, kin = k & 31;
+  int step = kin >> 4, k16 = kin & 15;
+  int hi = k16 >> 3, c = (k16 & 7) >> 1, h = k16 & 1;
+  int lane = g * 4 + c;
+  int comp = step * 2 + hi;  // u32 within the uint4
+  return ((nt * (Kpad >> 5) + kk) * 32 + lane) * 8 + comp * 2 + h;
+}
+
+}  // namespace moeq

@@ -1,0 +1,105 @@
+// Internal launch interface between the C-ABI host code and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include "common.cuh"
+
+namespace moeq {
+
+enum : int { ACT_FRAG = 0, ACT_ROW = 1 };
+enum : int { MODE_SWIGLU = 0, MODE_OUT = 1 };
+
+struct RouteArgs {
+  const float* logits;        // [T, E]
+  const __nv_bfloat16* X;     // [T, K]
+  int T, E, k, K, renorm;
+  int* idx;                   // [T, k]
+  float* w;                   // [T, k]
+  int* block_counts;          // [nb, E]
+  int* block_base;            // [nb, E]
+  int* pblock_base;           // [nb, E]
+  int* counts;                // [E]
+  int* offsets;               // [E+1]
+  int* poffsets;              // [E+1] (8-row padded)
+  int* active;                // [E]
+  int* n_active;              // [1]
+  int* ticket;                // [1], zero between launches
+  int* perm_token;            // [T*k]
+  int* inv_pos;               // [T, k]
+  int* pinv;                  // [T, k] padded row
+  void* act;                  // activation buffer (fp16), layout act_layout
+  int Kpad;                   // activation row width (elements)
+  int act_layout;
+  unsigned* status;
+};
+
+struct GemmArgs {
+  const ExpertDesc* experts;
+  int block;                  // 0 = W1, 1 = W2
+  const int* active;
+  const int* n_active;
+  const int* counts;
+  const int* poffsets;
+  const uint4* act;           // input activations (fragment layout)
+  int Kpad_in;
+  int K;                      // quantised K of the block
+  int M;                      // rows of the block
+  int mode;
+  __half* zout;               // MODE_SWIGLU: output activations (fragment layout)
+  int Kpad_out;
+  float* out;                 // MODE_OUT: [KS][prows][M] fp32 partials
+  long long out_ks_stride;
+  int KS;
+  unsigned* status;
+};
+
+struct LowrankArgs {
+  const ExpertDesc* experts;
+  int block;
+  const int* active;
+  const int* n_active;
+  const int* counts;
+  const int* poffsets;
+  __half* act;                // activation buffer; reads [0,K), writes ext columns [K, K+r)
+  int Kpad;
+  int K;
+  int KS;
+  float* part;                // [KS][prows][64]
+  long long part_ks_stride;
+  int* sem;                   // [E], zero between launches
+  int act_layout;
+  unsigned* status;
+};
+
+struct CombineArgs {
+  const float* O;             // [KS][prows][K]
+  long long ks_stride;
+  int KS;
+  const float* w;             // [T, k]
+  const int* pinv;            // [T, k]
+  int T, k, K;
+  __nv_bfloat16* Y;           // [T, K]
+};
+
+cudaError_t launch_relayout_int(const uint8_t* canon, uint8_t* out, int M, int K, int bits, int block, int N,
+                                cudaStream_t st);
+cudaError_t launch_relayout_sz(const __half* s, const __half* z, uint32_t* out, int M, int K, int group, int block,
+                               int N, cudaStream_t st);
+cudaError_t launch_relayout_dense(const __nv_bfloat16* src, uint4* out, int M, int K, int block, int N, long long ld,
+                                  cudaStream_t st);
+cudaError_t launch_relayout_planes(const uint32_t* canon, uint32_t* out, int M, int K, int block, int N,
+                                   cudaStream_t st);
+cudaError_t launch_debug_unpack(const BlockDesc& d, uint8_t* out, int block, int N, cudaStream_t st);
+
+cudaError_t launch_route_topk(const RouteArgs& a, cudaStream_t st, int* launches);
+cudaError_t launch_route_permute(const RouteArgs& a, cudaStream_t st, int* launches);
+int route_num_blocks(int T);
+
+// grid sizing helpers for the decode GEMM
+int decode_rows_per_cta();
+size_t decode_smem_bytes(int nt, int maxbits);
+cudaError_t launch_decode_gemm(const GemmArgs& a, int nt_max, int maxbits, int grid_y, cudaStream_t st,
+                               int* launches);
+cudaError_t launch_lowrank(const LowrankArgs& a, int grid_y, cudaStream_t st, int* launches);
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st, int* launches);
+
+}  // namespace moeq

@@ -1,0 +1,631 @@
+// C ABI of the quantized MoE expert layer: ownership, validation, weight
+// loading (device re-layout) and the launch sequence of one forward pass.
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <vector>
+
+#include "../../include/moe_layer.h"
+#include "kernels.h"
+
+using namespace moeq;
+
+namespace {
+
+struct DevBuf {
+  void* p = nullptr;
+  size_t n = 0;
+};
+
+// allocation-failure injection for the error-path tests (host side only)
+int g_alloc_count = 0;
+int fail_alloc_at() {
+  const char* s = std::getenv("MOE_TEST_FAIL_ALLOC_AT");
+  return s ? std::atoi(s) : -1;
+}
+
+moe_status_t dalloc(DevBuf& b, size_t n) {
+  const int at = fail_alloc_at();
+  ++g_alloc_count;
+  if (at >= 0 && g_alloc_count == at) return MOE_ERR_OOM;
+  if (n == 0) n = 16;
+  if (cudaMalloc(&b.p, n) != cudaSuccess) {
+    cudaGetLastError();
+    b.p = nullptr;
+    return MOE_ERR_OOM;
+  }
+  b.n = n;
+  return MOE_OK;
+}
+void dfree(DevBuf& b) {
+  if (b.p) cudaFree(b.p);
+  b.p = nullptr;
+  b.n = 0;
+}
+
+struct BlockStore {
+  DevBuf codes, sz, lut, afrag, bfrag;
+};
+
+}  // namespace
+
+struct moe_layer {
+  int E = 0, K = 0, N = 0, max_tokens = 0, max_top_k = 0;
+  unsigned flags = 0;
+  int path = MOE_PATH_AUTO;
+  std::vector<moe_expert_desc_t> descs;
+  std::vector<ExpertDesc> hdesc;
+  std::vector<BlockStore> store;  // [E * 2]
+  DevBuf d_experts;
+  // workspace
+  int rmax_pad = 0, Kpad_x = 0, Kpad_z = 0;
+  long long rows_pad_max = 0;
+  int nb_max = 0, ks2_max = 1, kslr_max = 1;
+  DevBuf idx, w, counts, offsets, poffsets, active, n_active, ticket, perm, inv_pos, pinv;
+  DevBuf block_counts, block_base, pblock_base, sem, status;
+  DevBuf xact, zact, obuf, part;
+  DevBuf hx, hl, hy;  // device buffers for forward_host
+  int last_T = 0, last_k = 0, last_launches = 0;
+  cudaStream_t last_stream = nullptr;
+  // profiling: events around each launch of the last forward
+  bool profiling = false;
+  std::vector<cudaEvent_t> events;
+  std::vector<const char*> prof_names;
+  int prof_count = -1;
+};
+
+// records an event before a kernel (profiling only); returns the slot
+static void prof_mark(moe_layer_t* L, cudaStream_t st, const char* name) {
+  if (!L->profiling) return;
+  const size_t i = L->prof_names.size();
+  while (L->events.size() < i + 2) {
+    cudaEvent_t ev;
+    if (cudaEventCreate(&ev) != cudaSuccess) return;
+    L->events.push_back(ev);
+  }
+  cudaEventRecord(L->events[i], st);
+  L->prof_names.push_back(name);
+}
+static void prof_end(moe_layer_t* L, cudaStream_t st) {
+  if (!L->profiling) return;
+  const size_t i = L->prof_names.size();
+  if (L->events.size() > i) cudaEventRecord(L->events[i], st);
+  L->prof_count = (int)i;
+}
+
+static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+static bool valid_desc(const moe_expert_desc_t& d, int K, int N) {
+  if (d.rank < 0 || d.rank > kMaxRank) return false;
+  if (d.format == MOE_FMT_INT_ASYM) {
+    for (int b = 0; b < 2; ++b)
+      if (d.bits[b] < 2 || d.bits[b] > 4) return false;
+    if (d.group_size != 64 && d.group_size != 128) return false;
+    if (K % d.group_size || N % d.group_size) return false;
+    return true;
+  }
+  if (d.format == MOE_FMT_BITPLANE_LUT) {
+    for (int b = 0; b < 2; ++b)
+      if (d.bits[b] < 2 || d.bits[b] > 4) return false;
+    return true;
+  }
+  if (d.format == MOE_FMT_DENSE16) return d.bits[0] == 16 && d.bits[1] == 16;
+  return false;
+}
+
+static void free_block(BlockStore& s) {
+  dfree(s.codes);
+  dfree(s.sz);
+  dfree(s.lut);
+  dfree(s.afrag);
+  dfree(s.bfrag);
+}
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_OOM: return "device allocation failed";
+    case MOE_ERR_NOT_LOADED: return "expert weights not loaded";
+    case MOE_ERR_UNSUPPORTED: return "unsupported";
+    case MOE_ERR_BITS_UNAVAILABLE: return "bitwidth not available";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_CHECK: return "device-side check failed";
+    case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+void moe_layer_destroy(moe_layer_t* L) {
+  if (!L) return;
+  for (auto& s : L->store) free_block(s);
+  DevBuf* bufs[] = {&L->d_experts, &L->idx, &L->w, &L->counts, &L->offsets, &L->poffsets, &L->active,
+                    &L->n_active, &L->ticket, &L->perm, &L->inv_pos, &L->pinv, &L->block_counts,
+                    &L->block_base, &L->pblock_base, &L->sem, &L->status, &L->xact, &L->zact, &L->obuf,
+                    &L->part, &L->hx, &L->hl, &L->hy};
+  for (DevBuf* b : bufs) dfree(*b);
+  for (cudaEvent_t ev : L->events) cudaEventDestroy(ev);
+  delete L;
+}
+
+moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k, const moe_expert_desc_t* descs,
+                              unsigned flags, moe_layer_t** out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!descs || E < 1 || E > kMaxExperts || K < 128 || N < 128 || K % 128 || N % 128 || max_tokens < 1 ||
+      max_top_k < 1 || max_top_k > kMaxTopK || max_top_k > E || (flags & ~MOE_FLAG_NO_TOPK_RENORM))
+    return MOE_ERR_INVALID_ARG;
+  int rmax = 0;
+  for (int e = 0; e < E; ++e) {
+    if (!valid_desc(descs[e], K, N)) return MOE_ERR_INVALID_ARG;
+    const int rp = (descs[e].rank + 15) / 16 * 16;
+    rmax = rp > rmax ? rp : rmax;
+  }
+  g_alloc_count = 0;
+  moe_layer_t* L = new moe_layer_t();
+  L->E = E;
+  L->K = K;
+  L->N = N;
+  L->max_tokens = max_tokens;
+  L->max_top_k = max_top_k;
+  L->flags = flags;
+  L->descs.assign(descs, descs + E);
+  L->hdesc.assign(E, ExpertDesc{});
+  L->store.resize(2 * E);
+  for (int e = 0; e < E; ++e)
+    for (int b = 0; b < 2; ++b) {
+      BlockDesc& d = L->hdesc[e].blk[b];
+      std::memset(&d, 0, sizeof(d));
+      d.fmt = descs[e].format == MOE_FMT_INT_ASYM ? FMT_INT : descs[e].format == MOE_FMT_BITPLANE_LUT ? FMT_BITPLANE : FMT_DENSE;
+      d.bits = descs[e].bits[b];
+      d.group = descs[e].group_size;
+      d.rank = (descs[e].rank + 15) / 16 * 16;  // kernels take the rank in k16 steps
+      d.M = b == 0 ? 2 * N : K;
+      d.K = b == 0 ? K : N;
+      d.loaded = 0;
+    }
+  L->rmax_pad = (rmax + 31) / 32 * 32;
+  L->Kpad_x = K + L->rmax_pad;
+  L->Kpad_z = N + L->rmax_pad;
+  const long long rows = (long long)max_tokens * max_top_k;
+  L->rows_pad_max = (rows + 7LL * E + 7) / 8 * 8;
+  L->nb_max = route_num_blocks(max_tokens);
+  L->ks2_max = 16;
+  L->kslr_max = 32;
+  // split-K partial outputs (ks2 > 1) are used only when T*k <= 1024
+  const long long small_rows = std::min<long long>(L->rows_pad_max, (1024 + 7LL * E + 7) / 8 * 8);
+  const long long o_elems = std::max<long long>(L->rows_pad_max, (long long)L->ks2_max * small_rows);
+  moe_status_t st = MOE_OK;
+  auto A = [&](DevBuf& b, size_t n) {
+    if (st == MOE_OK) st = dalloc(b, n);
+  };
+  A(L->d_experts, sizeof(ExpertDesc) * E);
+  A(L->idx, sizeof(int) * rows);
+  A(L->w, sizeof(float) * rows);
+  A(L->counts, sizeof(int) * E);
+  A(L->offsets, sizeof(int) * (E + 1));
+  A(L->poffsets, sizeof(int) * (E + 1));
+  A(L->active, sizeof(int) * E);
+  A(L->n_active, sizeof(int));
+  A(L->ticket, sizeof(int));
+  A(L->perm, sizeof(int) * rows);
+  A(L->inv_pos, sizeof(int) * rows);
+  A(L->pinv, sizeof(int) * rows);
+  A(L->block_counts, sizeof(int) * (size_t)L->nb_max * E);
+  A(L->block_base, sizeof(int) * (size_t)L->nb_max * E);
+  A(L->pblock_base, sizeof(int) * (size_t)L->nb_max * E);
+  A(L->sem, sizeof(int) * E);
+  A(L->status, sizeof(unsigned));
+  A(L->xact, sizeof(__half) * (size_t)L->rows_pad_max * L->Kpad_x);
+  A(L->zact, sizeof(__half) * (size_t)L->rows_pad_max * L->Kpad_z);
+  A(L->obuf, sizeof(float) * (size_t)o_elems * K);
+  A(L->part, sizeof(float) * (size_t)L->kslr_max * L->rows_pad_max * kMaxRank);
+  A(L->hx, sizeof(__nv_bfloat16) * (size_t)max_tokens * K);
+  A(L->hl, sizeof(float) * (size_t)max_tokens * E);
+  A(L->hy, sizeof(__nv_bfloat16) * (size_t)max_tokens * K);
+  if (st != MOE_OK) {
+    moe_layer_destroy(L);
+    return st;
+  }
+  cudaError_t ce = cudaSuccess;
+  DevBuf* zero[] = {&L->ticket, &L->sem, &L->status, &L->xact, &L->zact, &L->n_active, &L->counts};
+  for (DevBuf* b : zero)
+    if (ce == cudaSuccess) ce = cudaMemset(b->p, 0, b->n);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpy(L->d_experts.p, L->hdesc.data(), sizeof(ExpertDesc) * E, cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess) ce = cudaDeviceSynchronize();
+  if (ce != cudaSuccess) {
+    moe_layer_destroy(L);
+    return MOE_ERR_CUDA;
+  }
+  *out = L;
+  return MOE_OK;
+}
+
+static moe_status_t upload_desc(moe_layer_t* L, int e) {
+  return cuda_status(cudaMemcpy(static_cast<ExpertDesc*>(L->d_experts.p) + e, &L->hdesc[e], sizeof(ExpertDesc),
+                                cudaMemcpyHostToDevice));
+}
+
+// device copy of a caller buffer (host or device); owned by `tmp`
+static moe_status_t stage_in(DevBuf& tmp, const void* src, size_t n, int ptr_kind, const void** dev) {
+  if (ptr_kind == 1) {
+    *dev = src;
+    return MOE_OK;
+  }
+  moe_status_t st = dalloc(tmp, n);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpy(tmp.p, src, n, cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+  *dev = tmp.p;
+  return MOE_OK;
+}
+
+moe_status_t moe_layer_set_expert_weights(moe_layer_t* L, int e, int block, const void* codes, const void* scales,
+                                          const void* zeros_or_lut, const void* Af, const void* Bf, int ptr_kind) {
+  if (!L || e < 0 || e >= L->E || block < 0 || block > 1 || !codes || (ptr_kind != 0 && ptr_kind != 1))
+    return MOE_ERR_INVALID_ARG;
+  BlockDesc& d = L->hdesc[e].blk[block];
+  const int M = d.M, Kin = d.K, r = d.rank;
+  if (d.fmt == FMT_INT && (!scales || !zeros_or_lut)) return MOE_ERR_INVALID_ARG;
+  if (d.fmt == FMT_BITPLANE && !zeros_or_lut) return MOE_ERR_INVALID_ARG;
+  if (r > 0 && (!Af || !Bf)) return MOE_ERR_INVALID_ARG;
+  BlockStore& S = L->store[2 * e + block];
+  free_block(S);
+  d.loaded = 0;
+  moe_status_t st = MOE_OK;
+  DevBuf t1, t2, t3, t4, t5;
+  const int MF = M / 16, KC = Kin / kChunkK;
+  cudaStream_t s0 = 0;
+  cudaError_t ce = cudaSuccess;
+  const void* dc = nullptr;
+  if (d.fmt == FMT_INT) {
+    const size_t nbytes = (size_t)M * Kin * d.bits / 8;
+    const size_t nsz = (size_t)M * (Kin / d.group) * sizeof(__half);
+    const void *ds = nullptr, *dz = nullptr;
+    st = stage_in(t1, codes, nbytes, ptr_kind, &dc);
+    if (st == MOE_OK) st = stage_in(t2, scales, nsz, ptr_kind, &ds);
+    if (st == MOE_OK) st = stage_in(t3, zeros_or_lut, nsz, ptr_kind, &dz);
+    if (st == MOE_OK) st = dalloc(S.codes, (size_t)MF * KC * 256 * d.bits);
+    if (st == MOE_OK) st = dalloc(S.sz, (size_t)MF * (Kin / d.group) * 16 * sizeof(uint32_t));
+    if (st == MOE_OK) {
+      ce = launch_relayout_int(static_cast<const uint8_t*>(dc), static_cast<uint8_t*>(S.codes.p), M, Kin, d.bits,
+                               block, L->N, s0);
+      if (ce == cudaSuccess)
+        ce = launch_relayout_sz(static_cast<const __half*>(ds), static_cast<const __half*>(dz),
+                                static_cast<uint32_t*>(S.sz.p), M, Kin, d.group, block, L->N, s0);
+    }
+  } else if (d.fmt == FMT_BITPLANE) {
+    const size_t nbytes = (size_t)4 * M * (Kin / 32) * sizeof(uint32_t);
+    const void* dl = nullptr;
+    st = stage_in(t1, codes, nbytes, ptr_kind, &dc);
+    if (st == MOE_OK) st = stage_in(t3, zeros_or_lut, 28 * sizeof(__half), ptr_kind, &dl);
+    if (st == MOE_OK) st = dalloc(S.codes, (size_t)4 * MF * KC * 256);
+    if (st == MOE_OK) st = dalloc(S.lut, 28 * sizeof(__half));
+    if (st == MOE_OK) {
+      ce = launch_relayout_planes(static_cast<const uint32_t*>(dc), static_cast<uint32_t*>(S.codes.p), M, Kin, block,
+                                  L->N, s0);
+      if (ce == cudaSuccess) ce = cudaMemcpy(S.lut.p, dl, 28 * sizeof(__half), cudaMemcpyDeviceToDevice);
+    }
+  } else {
+    const size_t nbytes = (size_t)M * Kin * sizeof(__nv_bfloat16);
+    st = stage_in(t1, codes, nbytes, ptr_kind, &dc);
+    if (st == MOE_OK) st = dalloc(S.codes, nbytes);
+    if (st == MOE_OK)
+      ce = launch_relayout_dense(static_cast<const __nv_bfloat16*>(dc), static_cast<uint4*>(S.codes.p), M, Kin, block,
+                                 L->N, Kin, s0);
+  }
+  if (st == MOE_OK && ce == cudaSuccess && r > 0) {
+    // factors padded with zeros to the k16 rank r (caller rank r0 <= r)
+    const int r0 = L->descs[e].rank;
+    const size_t es = sizeof(__nv_bfloat16);
+    const void *da = nullptr, *db = nullptr;
+    st = dalloc(t4, (size_t)r * Kin * es);
+    if (st == MOE_OK) st = dalloc(t5, (size_t)M * r * es);
+    if (st == MOE_OK) {
+      const cudaMemcpyKind kind = ptr_kind == 1 ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+      ce = cudaMemset(t4.p, 0, t4.n);
+      if (ce == cudaSuccess) ce = cudaMemset(t5.p, 0, t5.n);
+      if (ce == cudaSuccess) ce = cudaMemcpy(t4.p, Af, (size_t)r0 * Kin * es, kind);
+      if (ce == cudaSuccess) ce = cudaMemcpy2D(t5.p, r * es, Bf, r0 * es, r0 * es, M, kind);
+      da = t4.p;
+      db = t5.p;
+    }
+    if (st == MOE_OK) st = dalloc(S.afrag, (size_t)r * Kin * sizeof(__half));
+    if (st == MOE_OK) st = dalloc(S.bfrag, (size_t)M * r * sizeof(__half));
+    if (st == MOE_OK && ce == cudaSuccess) {
+      ce = launch_relayout_dense(static_cast<const __nv_bfloat16*>(da), static_cast<uint4*>(S.afrag.p), r, Kin, -1,
+                                 L->N, Kin, s0);
+      if (ce == cudaSuccess)
+        ce = launch_relayout_dense(static_cast<const __nv_bfloat16*>(db), static_cast<uint4*>(S.bfrag.p), M, r, block,
+                                   L->N, r, s0);
+    }
+  }
+  if (st == MOE_OK && ce == cudaSuccess) ce = cudaDeviceSynchronize();
+  dfree(t1);
+  dfree(t2);
+  dfree(t3);
+  dfree(t4);
+  dfree(t5);
+  if (st == MOE_OK && ce != cudaSuccess) st = MOE_ERR_CUDA;
+  if (st != MOE_OK) {
+    free_block(S);
+    upload_desc(L, e);
+    return st;
+  }
+  d.codes = static_cast<const uint8_t*>(S.codes.p);
+  d.sz = static_cast<const uint32_t*>(S.sz.p);
+  d.lut = static_cast<const uint32_t*>(S.lut.p);
+  d.afrag = static_cast<const uint4*>(S.afrag.p);
+  d.bfrag = static_cast<const uint4*>(S.bfrag.p);
+  d.plane_stride = (long long)MF * KC * 256;
+  d.loaded = 1;
+  return upload_desc(L, e);
+}
+
+moe_status_t moe_layer_set_bits(moe_layer_t* L, int e, int block, int bits) {
+  if (!L || e < 0 || e >= L->E || block < -1 || block > 1) return MOE_ERR_INVALID_ARG;
+  const int b0 = block < 0 ? 0 : block, b1 = block < 0 ? 1 : block;
+  const int fmt = L->hdesc[e].blk[b0].fmt;
+  if (fmt == FMT_DENSE) return MOE_ERR_UNSUPPORTED;
+  if (bits > 4) return MOE_ERR_BITS_UNAVAILABLE;
+  if (bits < 2) return MOE_ERR_INVALID_ARG;
+  for (int b = b0; b <= b1; ++b) {
+    BlockDesc& d = L->hdesc[e].blk[b];
+    if (d.bits == bits) continue;
+    d.bits = bits;
+    L->descs[e].bits[b] = bits;
+    if (fmt == FMT_INT) {
+      free_block(L->store[2 * e + b]);
+      d.loaded = 0;
+      d.codes = nullptr;
+      d.sz = nullptr;
+      d.afrag = nullptr;
+      d.bfrag = nullptr;
+    }
+  }
+  return upload_desc(L, e);
+}
+
+moe_status_t moe_layer_set_path(moe_layer_t* L, int path) {
+  if (!L || path < MOE_PATH_AUTO || path > MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
+  L->path = path;
+  return MOE_OK;
+}
+
+int moe_layer_last_launch_count(const moe_layer_t* L) { return L ? L->last_launches : 0; }
+
+moe_status_t moe_layer_set_profiling(moe_layer_t* L, int enable) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  L->profiling = enable != 0;
+  L->prof_count = -1;
+  return MOE_OK;
+}
+
+int moe_layer_kernel_times(moe_layer_t* L, const char** names, float* ms, int cap) {
+  if (!L || L->prof_count < 0) return -1;
+  if (cudaStreamSynchronize(L->last_stream) != cudaSuccess) return -1;
+  const int n = L->prof_count;
+  for (int i = 0; i < n && i < cap; ++i) {
+    if (names) names[i] = L->prof_names[i];
+    if (ms) {
+      float t = 0.f;
+      cudaEventElapsedTime(&t, L->events[i], L->events[i + 1]);
+      ms[i] = t;
+    }
+  }
+  return n;
+}
+
+moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logits, int T, int top_k, void* Y,
+                               void* stream) {
+  if (!L || !X || !logits || !Y || T < 1 || T > L->max_tokens || top_k < 1 || top_k > L->max_top_k)
+    return MOE_ERR_INVALID_ARG;
+  for (int e = 0; e < L->E; ++e)
+    if (!L->hdesc[e].blk[0].loaded || !L->hdesc[e].blk[1].loaded) return MOE_ERR_NOT_LOADED;
+  int path = L->path;
+  if (path == MOE_PATH_AUTO) path = MOE_PATH_DECODE;
+  if (path != MOE_PATH_DECODE) return MOE_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int E = L->E, K = L->K, N = L->N;
+  int maxbits[2] = {0, 0}, rmax = 0;
+  for (int e = 0; e < E; ++e) {
+    for (int b = 0; b < 2; ++b) {
+      const int bb = L->hdesc[e].blk[b].bits;
+      maxbits[b] = bb > maxbits[b] ? bb : maxbits[b];
+    }
+    rmax = L->hdesc[e].blk[0].rank > rmax ? L->hdesc[e].blk[0].rank : rmax;
+  }
+  const long long rows = (long long)T * top_k;
+  const int grid_y = (int)std::min<long long>(E, rows);
+  int launches = 0;
+  cudaError_t ce = cudaSuccess;
+
+  RouteArgs ra{};
+  ra.logits = logits;
+  ra.X = static_cast<const __nv_bfloat16*>(X);
+  ra.T = T;
+  ra.E = E;
+  ra.k = top_k;
+  ra.K = K;
+  ra.renorm = (L->flags & MOE_FLAG_NO_TOPK_RENORM) ? 0 : 1;
+  ra.idx = static_cast<int*>(L->idx.p);
+  ra.w = static_cast<float*>(L->w.p);
+  ra.block_counts = static_cast<int*>(L->block_counts.p);
+  ra.block_base = static_cast<int*>(L->block_base.p);
+  ra.pblock_base = static_cast<int*>(L->pblock_base.p);
+  ra.counts = static_cast<int*>(L->counts.p);
+  ra.offsets = static_cast<int*>(L->offsets.p);
+  ra.poffsets = static_cast<int*>(L->poffsets.p);
+  ra.active = static_cast<int*>(L->active.p);
+  ra.n_active = static_cast<int*>(L->n_active.p);
+  ra.ticket = static_cast<int*>(L->ticket.p);
+  ra.perm_token = static_cast<int*>(L->perm.p);
+  ra.inv_pos = static_cast<int*>(L->inv_pos.p);
+  ra.pinv = static_cast<int*>(L->pinv.p);
+  ra.act = L->xact.p;
+  ra.Kpad = L->Kpad_x;
+  ra.act_layout = ACT_FRAG;
+  ra.status = static_cast<unsigned*>(L->status.p);
+  L->prof_names.clear();
+  prof_mark(L, st, "route_topk");
+  ce = launch_route_topk(ra, st, &launches);
+  prof_mark(L, st, "route_permute");
+  if (ce == cudaSuccess) ce = launch_route_permute(ra, st, &launches);
+
+  const ExpertDesc* dexp = static_cast<const ExpertDesc*>(L->d_experts.p);
+  const long long prows = (rows + 7LL * E + 7) / 8 * 8;
+  auto lowrank = [&](int block, __half* act, int Kpad, int Kin) {
+    if (ce != cudaSuccess || rmax == 0) return;
+    LowrankArgs la{};
+    la.experts = dexp;
+    la.block = block;
+    la.active = ra.active;
+    la.n_active = ra.n_active;
+    la.counts = ra.counts;
+    la.poffsets = ra.poffsets;
+    la.act = act;
+    la.Kpad = Kpad;
+    la.K = Kin;
+    int ks = 296 / grid_y;
+    ks = std::max(1, std::min(ks, std::min(L->kslr_max, Kin / 16 / 8)));
+    la.KS = ks;
+    la.part = static_cast<float*>(L->part.p);
+    la.part_ks_stride = (long long)L->rows_pad_max * kMaxRank;
+    la.sem = static_cast<int*>(L->sem.p);
+    la.act_layout = ACT_FRAG;
+    la.status = ra.status;
+    prof_mark(L, st, block == 0 ? "lowrank_w1" : "lowrank_w2");
+    ce = launch_lowrank(la, grid_y, st, &launches);
+  };
+  // W1 side compensator U1 = X A1^T
+  lowrank(0, static_cast<__half*>(L->xact.p), L->Kpad_x, K);
+  const int nt_max = (int)std::min<long long>(8, (std::min<long long>(T, 64) + 7) / 8);
+  if (ce == cudaSuccess) {
+    GemmArgs ga{};
+    ga.experts = dexp;
+    ga.block = 0;
+    ga.active = ra.active;
+    ga.n_active = ra.n_active;
+    ga.counts = ra.counts;
+    ga.poffsets = ra.poffsets;
+    ga.act = static_cast<const uint4*>(L->xact.p);
+    ga.Kpad_in = L->Kpad_x;
+    ga.K = K;
+    ga.M = 2 * N;
+    ga.mode = MODE_SWIGLU;
+    ga.zout = static_cast<__half*>(L->zact.p);
+    ga.Kpad_out = L->Kpad_z;
+    ga.KS = 1;
+    ga.status = ra.status;
+    prof_mark(L, st, "decode_gemm_w1_swiglu");
+    ce = launch_decode_gemm(ga, nt_max, maxbits[0], grid_y, st, &launches);
+  }
+  lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N);
+  int ks2 = 1;
+  if (ce == cudaSuccess) {
+    const int row_tiles = (K + decode_rows_per_cta() - 1) / decode_rows_per_cta();
+    const int want = 2 * 148;
+    ks2 = std::max(1, want / std::max(1, row_tiles * grid_y));
+    ks2 = std::min(ks2, std::min(L->ks2_max, N / kChunkK));
+    if (rows > 1024) ks2 = 1;
+    GemmArgs ga{};
+    ga.experts = dexp;
+    ga.block = 1;
+    ga.active = ra.active;
+    ga.n_active = ra.n_active;
+    ga.counts = ra.counts;
+    ga.poffsets = ra.poffsets;
+    ga.act = static_cast<const uint4*>(L->zact.p);
+    ga.Kpad_in = L->Kpad_z;
+    ga.K = N;
+    ga.M = K;
+    ga.mode = MODE_OUT;
+    ga.out = static_cast<float*>(L->obuf.p);
+    ga.out_ks_stride = prows * K;
+    ga.KS = ks2;
+    ga.status = ra.status;
+    prof_mark(L, st, "decode_gemm_w2");
+    ce = launch_decode_gemm(ga, nt_max, maxbits[1], grid_y, st, &launches);
+  }
+  if (ce == cudaSuccess) {
+    CombineArgs ca{};
+    ca.O = static_cast<const float*>(L->obuf.p);
+    ca.ks_stride = prows * K;
+    ca.KS = ks2;
+    ca.w = ra.w;
+    ca.pinv = ra.pinv;
+    ca.T = T;
+    ca.k = top_k;
+    ca.K = K;
+    ca.Y = static_cast<__nv_bfloat16*>(Y);
+    prof_mark(L, st, "combine");
+    ce = launch_combine(ca, st, &launches);
+  }
+  prof_end(L, st);
+  L->last_T = T;
+  L->last_k = top_k;
+  L->last_launches = launches;
+  L->last_stream = st;
+  return cuda_status(ce);
+}
+
+moe_status_t moe_layer_forward_host(moe_layer_t* L, const void* Xh, const float* Lh, int T, int top_k, void* Yh,
+                                    void* stream) {
+  if (!L || !Xh || !Lh || !Yh || T < 1 || T > L->max_tokens) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t xb = (size_t)T * L->K * sizeof(__nv_bfloat16), lb = (size_t)T * L->E * sizeof(float);
+  cudaError_t ce = cudaMemcpyAsync(L->hx.p, Xh, xb, cudaMemcpyHostToDevice, st);
+  if (ce == cudaSuccess) ce = cudaMemcpyAsync(L->hl.p, Lh, lb, cudaMemcpyHostToDevice, st);
+  if (ce != cudaSuccess) return MOE_ERR_CUDA;
+  moe_status_t s = moe_layer_forward(L, L->hx.p, static_cast<const float*>(L->hl.p), T, top_k, L->hy.p, stream);
+  if (s != MOE_OK) return s;
+  ce = cudaMemcpyAsync(Yh, L->hy.p, xb, cudaMemcpyDeviceToHost, st);
+  if (ce == cudaSuccess) ce = cudaStreamSynchronize(st);
+  return cuda_status(ce);
+}
+
+moe_status_t moe_layer_get_routing(moe_layer_t* L, int* idx, float* w, int* counts, int* offsets, int* perm_token,
+                                   int* inv_pos) {
+  if (!L || L->last_T == 0) return MOE_ERR_INVALID_ARG;
+  const size_t tk = (size_t)L->last_T * L->last_k;
+  cudaError_t ce = cudaStreamSynchronize(L->last_stream);
+  auto cp = [&](void* dst, const DevBuf& src, size_t n) {
+    if (dst && ce == cudaSuccess) ce = cudaMemcpy(dst, src.p, n, cudaMemcpyDeviceToDevice);
+  };
+  cp(idx, L->idx, tk * sizeof(int));
+  cp(w, L->w, tk * sizeof(float));
+  cp(counts, L->counts, L->E * sizeof(int));
+  cp(offsets, L->offsets, (L->E + 1) * sizeof(int));
+  cp(perm_token, L->perm, tk * sizeof(int));
+  cp(inv_pos, L->inv_pos, tk * sizeof(int));
+  return cuda_status(ce);
+}
+
+moe_status_t moe_layer_debug_unpack(moe_layer_t* L, int e, int block, unsigned char* out) {
+  if (!L || e < 0 || e >= L->E || block < 0 || block > 1 || !out) return MOE_ERR_INVALID_ARG;
+  const BlockDesc& d = L->hdesc[e].blk[block];
+  if (!d.loaded) return MOE_ERR_NOT_LOADED;
+  if (d.fmt == FMT_DENSE) return MOE_ERR_UNSUPPORTED;
+  cudaError_t ce = launch_debug_unpack(d, out, block, L->N, 0);
+  if (ce == cudaSuccess) ce = cudaDeviceSynchronize();
+  return cuda_status(ce);
+}
+
+moe_status_t moe_layer_sync_status(moe_layer_t* L) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  cudaError_t ce = cudaStreamSynchronize(L->last_stream);
+  if (ce == cudaSuccess) ce = cudaGetLastError();
+  if (ce != cudaSuccess) return MOE_ERR_CUDA;
+  unsigned word = 0;
+  ce = cudaMemcpy(&word, L->status.p, sizeof(unsigned), cudaMemcpyDeviceToHost);
+  if (ce != cudaSuccess) return MOE_ERR_CUDA;
+  if (word) {
+    cudaMemset(L->status.p, 0, sizeof(unsigned));
+    return (word & ST_TIMEOUT) ? MOE_ERR_TIMEOUT : MOE_ERR_DEVICE_CHECK;
+  }
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,183 @@
+/*
+ * moe_layer.h - C ABI of the B200 quantized Mixture-of-Experts expert layer.
+ *
+ * The layer computes, for tokens X [T, K] and router logits [T, E]:
+ *
+ *   top-k routing      idx[t, 0..k-1] = the k largest logits of token t
+ *                      (descending, ties to the lower expert index);
+ *                      w[t, j] = softmax over the k selected logits
+ *                      (Bandwidth-Efficient Adaptive Mixture-of-Experts via
+ *                      Low-Rank Compensation, abstract: per-token Top-n of the
+ *                      k routed experts presumes this routing);
+ *   bucketing          routed (t, j) pairs grouped per expert, expert-major,
+ *                      token-ascending;
+ *   per expert e       h = W1^_e x + B1_e (A1_e x)      (W1 = [gate; up], 2N x K)
+ *                      z = silu(h[0:N]) * h[N:2N]
+ *                      o = W2^_e z + B2_e (A2_e z)      (W2 = down, K x N)
+ *                      where W^ is the dequantised weight and B A the rank-r_e
+ *                      low-rank compensator of the quantisation residual
+ *                      (MiLo: Efficient Quantized MoE Inference with Mixture of
+ *                      Low-Rank Compensators, abstract);
+ *   combine            y_t = sum_j w[t, j] * o_(t, j).
+ *
+ * Weight formats (per expert linear block, the "weight page" of PagedWeight:
+ * Efficient MoE LLM Serving with Dynamic Quality-Aware Weight Quantization,
+ * "What carries the argument"):
+ *
+ *   MOE_FMT_INT_ASYM     b in {2,3,4}; w^ = (q - z) * s, one fp16 scale s and one
+ *                        fp16 zero z per group of g consecutive elements along K.
+ *                        codes: uint8 [M, K*b/8], each row a little-endian
+ *                        bit-stream, code k at bits [b*k, b*k+b);
+ *                        scales, zeros: fp16 [M, K/g] row-major.
+ *   MOE_FMT_BITPLANE_LUT 4 stored bit-planes, bitwidth b in {2,3,4} chosen at run
+ *                        time (PagedWeight, Figure 3 caption: subsets of
+ *                        bit-planes give the effective bitwidths; one LUT of
+ *                        bitwidth-specific centroids per quantised tensor).
+ *                        codes: uint32 [4, M, K/32]; plane 0 = most significant
+ *                        bit; bit i of word w of a row is element 32*w + i; the
+ *                        b-bit code is the top b planes; w^ = LUT_b[code].
+ *                        zeros_or_lut: fp16 [28] = LUT_2 (4) | LUT_3 (8) | LUT_4 (16).
+ *   MOE_FMT_DENSE16      codes: bf16 [M, K] row-major (bits = 16).
+ *
+ * Compensator factors per block: A bf16 [r, K_in], B bf16 [M_out, r], r = the
+ * expert's rank (0 disables the term).
+ *
+ * Conventions.
+ *   - Every call returns a moe_status_t; nothing aborts or throws across the ABI.
+ *   - The layer owns its device copies of the weights and its workspace (sized
+ *     at create from max_tokens and max_top_k). The caller owns X, logits and Y.
+ *   - moe_layer_forward is asynchronous on the given CUDA stream; device-side
+ *     errors surface at moe_layer_sync_status or at the next call.
+ *   - One layer is used from one stream at a time.
+ *   - Arithmetic: fp16 tensor-core operands (X, dequantised weights, the
+ *     SwiGLU output and the compensator terms are rounded to fp16), fp32
+ *     accumulation, bf16 output. |X| and |z| must stay below 65504.
+ */
+#ifndef MOE_LAYER_H
+#define MOE_LAYER_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,      /* bad pointer, shape, index or flag */
+  MOE_ERR_OOM = 2,              /* a device allocation failed */
+  MOE_ERR_NOT_LOADED = 3,       /* forward before every expert's weights were set */
+  MOE_ERR_UNSUPPORTED = 4,      /* valid request this build does not implement */
+  MOE_ERR_BITS_UNAVAILABLE = 5, /* set_bits asks for planes that are not stored */
+  MOE_ERR_CUDA = 6,             /* a CUDA runtime call failed */
+  MOE_ERR_DEVICE_CHECK = 7,     /* a kernel's own check failed (status word) */
+  MOE_ERR_TIMEOUT = 8           /* a bounded device-side wait gave up */
+} moe_status_t;
+
+typedef enum {
+  MOE_FMT_INT_ASYM = 0,
+  MOE_FMT_BITPLANE_LUT = 1,
+  MOE_FMT_DENSE16 = 2
+} moe_format_t;
+
+/* Per-expert descriptor. bits[0] is W1's (gate||up) bitwidth, bits[1] W2's.
+ * INT_ASYM: bits in {2,3,4}, group_size in {64,128} dividing d_model and d_ff.
+ * BITPLANE_LUT: bits in {2,3,4} (the planes read), group_size ignored.
+ * DENSE16: bits = 16. rank: 0..64 (0 disables the compensator; a rank that is
+ * not a multiple of 16 is zero-padded to one internally). */
+typedef struct {
+  int bits[2];
+  moe_format_t format;
+  int group_size;
+  int rank;
+} moe_expert_desc_t;
+
+typedef struct moe_layer moe_layer_t; /* opaque */
+
+/* flags for moe_layer_create */
+#define MOE_FLAG_NO_TOPK_RENORM 1u /* w[t, j] = full-softmax probability of the selected expert */
+
+/* paths for moe_layer_set_path */
+#define MOE_PATH_AUTO 0    /* by T: decode kernels for small batches, prefill kernels above */
+#define MOE_PATH_DECODE 1  /* register-dequant mma.sync grouped GEMM */
+#define MOE_PATH_PREFILL 2 /* TMA + shared-memory dequant + tcgen05/TMEM grouped GEMM */
+
+/* Create a layer on the current CUDA device.
+ * d_model and d_ff: multiples of 128. num_experts <= 256, max_top_k <= 8 and
+ * <= num_experts, max_tokens >= 1. descs: [num_experts], copied.
+ * Weights start unset (forward returns MOE_ERR_NOT_LOADED until every expert's
+ * two blocks are set). On failure *out is NULL. */
+moe_status_t moe_layer_create(int num_experts, int d_model, int d_ff, int max_tokens, int max_top_k,
+                              const moe_expert_desc_t* descs, unsigned flags, moe_layer_t** out);
+
+/* Load one block (0 = W1 gate||up [2*d_ff, d_model], 1 = W2 down [d_model, d_ff])
+ * of one expert from the canonical layouts above. ptr_kind 0 = host pointers,
+ * 1 = device pointers. The data are copied and re-laid out on the device (the
+ * caller keeps ownership). scales is used by INT_ASYM only; zeros_or_lut holds
+ * the zeros (INT_ASYM) or the 28-entry LUT (BITPLANE_LUT). A and B may be NULL
+ * only if the expert's rank is 0. Synchronous. */
+moe_status_t moe_layer_set_expert_weights(moe_layer_t* layer, int expert, int block, const void* codes,
+                                          const void* scales, const void* zeros_or_lut, const void* A,
+                                          const void* B, int ptr_kind);
+
+/* Commit a new bitwidth for (expert, block); block = -1 applies to both.
+ * BITPLANE_LUT: 2 <= bits <= 4 (bits > 4: MOE_ERR_BITS_UNAVAILABLE); only the
+ * descriptor changes, no weight bytes move (PagedWeight, Figure 4: a lower
+ * committed bitwidth reads fewer planes). INT_ASYM: the codes cannot be
+ * truncated; the block's descriptor changes and its weights must be set again
+ * before the next forward (MOE_ERR_NOT_LOADED until then). DENSE16:
+ * MOE_ERR_UNSUPPORTED. Must not be called while a forward is in flight. */
+moe_status_t moe_layer_set_bits(moe_layer_t* layer, int expert, int block, int bits);
+
+/* Choose the kernel path (MOE_PATH_*). */
+moe_status_t moe_layer_set_path(moe_layer_t* layer, int path);
+
+/* Forward pass. X: bf16 [T, d_model] device; router_logits: fp32 [T, E] device;
+ * Y: bf16 [T, d_model] device, caller-allocated. 1 <= T <= max_tokens,
+ * 1 <= top_k <= max_top_k. cuda_stream: a cudaStream_t (NULL = legacy stream).
+ * Asynchronous. */
+moe_status_t moe_layer_forward(moe_layer_t* layer, const void* X, const float* router_logits, int T,
+                               int top_k, void* Y, void* cuda_stream);
+
+/* The same forward with HOST buffers: copies X and the logits to the device
+ * into layer-owned device buffers (pass pinned host memory for asynchronous
+ * copies), runs moe_layer_forward and copies Y
+ * back; returns after the stream has synchronised. */
+moe_status_t moe_layer_forward_host(moe_layer_t* layer, const void* X_host, const float* logits_host, int T,
+                                    int top_k, void* Y_host, void* cuda_stream);
+
+/* Routing of the last forward, copied into caller DEVICE buffers (any may be
+ * NULL): idx int32 [T, k], w fp32 [T, k], counts int32 [E], offsets int32
+ * [E+1], perm_token int32 [T*k], inv_pos int32 [T, k]. Synchronous. */
+moe_status_t moe_layer_get_routing(moe_layer_t* layer, int* idx, float* w, int* counts, int* offsets,
+                                   int* perm_token, int* inv_pos);
+
+/* Test hook: the codes of (expert, block) unpacked by the same device routine
+ * the GEMM kernels use, as uint8 [M, K] in canonical row order into a caller
+ * DEVICE buffer (INT_ASYM: q; BITPLANE_LUT: the code at the committed bits).
+ * Synchronous. */
+moe_status_t moe_layer_debug_unpack(moe_layer_t* layer, int expert, int block, unsigned char* codes_out);
+
+/* Synchronise the layer's last stream; return the device status word (bounds
+ * and wait checks) or the pending CUDA error, and clear the status word. */
+moe_status_t moe_layer_sync_status(moe_layer_t* layer);
+
+/* Number of kernels the last moe_layer_forward launched. */
+int moe_layer_last_launch_count(const moe_layer_t* layer);
+
+/* Profiling. When enabled (enable != 0), every forward records a CUDA event on
+ * its stream before and after each kernel it launches. */
+moe_status_t moe_layer_set_profiling(moe_layer_t* layer, int enable);
+
+/* Durations in ms of the kernels of the last profiled forward, in launch order:
+ * names[i] (static strings) and ms[i] for i < min(count, cap). Synchronises the
+ * stream. Returns the count, or -1 if nothing was profiled. */
+int moe_layer_kernel_times(moe_layer_t* layer, const char** names, float* ms, int cap);
+
+const char* moe_status_string(moe_status_t status);
+
+/* Free everything the layer owns. NULL is a no-op. */
+void moe_layer_destroy(moe_layer_t* layer);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_LAYER_H */
