@@ -32,6 +32,121 @@ __host__ __device__ inline int stage_bytes_of(int nt, int maxbits) {
 }
 __host__ __device__ inline int stages_of(int maxbits) { return maxbits >= 16 ? 2 : 4; }
 
+// Lane words of one row fragment's chunk, from shared memory.
+template <int FMT, int BITS>
+__device__ __forceinline__ void load_words(const uint8_t* ws, int lane, uint32_t (&w)[8]) {
+  if constexpr (FMT == FMT_INT && BITS == 4) {
+    const uint4 v0 = reinterpret_cast<const uint4*>(ws)[lane];
+    const uint4 v1 = reinterpret_cast<const uint4*>(ws)[32 + lane];
+    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+  } else if constexpr (FMT == FMT_INT) {
+    const uint4 v0 = reinterpret_cast<const uint4*>(ws)[lane];
+    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+    if constexpr (BITS == 3) {
+      const uint2 h = reinterpret_cast<const uint2*>(ws + 512)[lane];
+      w[4] = h.x; w[5] = h.y;
+    }
+  } else if constexpr (FMT == FMT_BITPLANE) {
+#pragma unroll
+    for (int p = 0; p < BITS; ++p) {
+      const uint2 v = reinterpret_cast<const uint2*>(ws + p * 256)[lane];
+      w[2 * p] = v.x; w[2 * p + 1] = v.y;
+    }
+  }
+}
+
+// One 128-wide K chunk for the warp's kRF row fragments and NP token tiles
+// (NP is the exact number of live tiles: no predicated MMAs).
+template <int NP, int NT, int FMT, int BITS, int GROUP>
+__device__ __forceinline__ void chunk_compute(const uint8_t* base, int warp, int lane, int wbytes_rf,
+                                              const LutRegs& lut, float (&acc)[kRF][NT][4]) {
+  const int g = lane >> 2;
+  const uint4* as = reinterpret_cast<const uint4*>(base);
+  uint32_t w[kRF][8];
+  const uint32_t* ssz[kRF];
+#pragma unroll
+  for (int r = 0; r < kRF; ++r) {
+    const uint8_t* ws = base + NT * 2048 + (warp * kRF + r) * wbytes_rf;
+    ssz[r] = reinterpret_cast<const uint32_t*>(base + NT * 2048 + kWarps * kRF * wbytes_rf +
+                                               (warp * kRF + r) * kSzBytesPerRf);
+    load_words<FMT, BITS>(ws, lane, w[r]);
+  }
+  uint32_t sA[kRF], nA[kRF], sB[kRF], nB[kRF];
+  uint4 bq[NP];
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    if ((s & 1) == 0) {
+#pragma unroll
+      for (int t = 0; t < NP; ++t) bq[t] = as[t * 128 + (s >> 1) * 32 + lane];
+    }
+#pragma unroll
+    for (int r = 0; r < kRF; ++r) {
+      uint32_t av[4];
+      if constexpr (FMT == FMT_INT) {
+        if ((16 * s) % GROUP == 0) {
+          const int gs = (16 * s) / GROUP;
+          const uint2 z2 = *reinterpret_cast<const uint2*>(ssz[r] + (gs * 8 + g) * 2);
+          sA[r] = prmt(z2.x, z2.x, 0x1010u); nA[r] = prmt(z2.x, z2.x, 0x3232u);
+          sB[r] = prmt(z2.y, z2.y, 0x1010u); nB[r] = prmt(z2.y, z2.y, 0x3232u);
+        }
+        uint32_t q[4];
+        int_codes<BITS>(w[r], s, q);
+        av[0] = hfma2u(q[0], sA[r], nA[r]);
+        av[1] = hfma2u(q[1], sB[r], nB[r]);
+        av[2] = hfma2u(q[2], sA[r], nA[r]);
+        av[3] = hfma2u(q[3], sB[r], nB[r]);
+      } else if constexpr (FMT == FMT_BITPLANE) {
+        lut_decode<BITS>(plane_codes<BITS>(w[r], s), lut, av);
+      } else {
+        const uint8_t* ws = base + NT * 2048 + (warp * kRF + r) * wbytes_rf;
+        const uint4 v = reinterpret_cast<const uint4*>(ws)[s * 32 + lane];
+        av[0] = v.x; av[1] = v.y; av[2] = v.z; av[3] = v.w;
+      }
+#pragma unroll
+      for (int t = 0; t < NP; ++t)
+        mma_16816(acc[r][t], av, (s & 1) ? bq[t].z : bq[t].x, (s & 1) ? bq[t].w : bq[t].y);
+    }
+  }
+}
+
+// rank-r compensator columns: B factor fragments against the U columns
+template <int NP, int NT>
+__device__ __forceinline__ void ext_compute(const GemmArgs& a, const BlockDesc& d, int rfw, long long tile0,
+                                            long long kblk, int lane, float (&acc)[kRF][NT][4]) {
+  const int RS = d.rank / 16;
+  for (int rs = 0; rs < RS; ++rs) {
+    const long long kk = (a.K >> 5) + (rs >> 1);
+    uint32_t b0[NP], b1[NP];
+#pragma unroll
+    for (int t = 0; t < NP; ++t) {
+      const uint4 v = a.act[((tile0 + t) * kblk + kk) * 32 + lane];
+      b0[t] = (rs & 1) ? v.z : v.x;
+      b1[t] = (rs & 1) ? v.w : v.y;
+    }
+#pragma unroll
+    for (int r = 0; r < kRF; ++r) {
+      const uint4 bv = d.bfrag[((long long)(rfw + r) * RS + rs) * 32 + lane];
+      const uint32_t av[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+      for (int t = 0; t < NP; ++t) mma_16816(acc[r][t], av, b0[t], b1[t]);
+    }
+  }
+}
+
+#define MOEQ_DISPATCH_NP(NPV, CALL)                 \
+  switch (NPV) {                                    \
+    case 1: { constexpr int NP_ = 1; CALL; } break; \
+    case 2: if constexpr (NT >= 2) { constexpr int NP_ = 2; CALL; } break; \
+    case 3: if constexpr (NT >= 3) { constexpr int NP_ = 3; CALL; } break; \
+    case 4: if constexpr (NT >= 4) { constexpr int NP_ = 4; CALL; } break; \
+    case 5: if constexpr (NT >= 5) { constexpr int NP_ = 5; CALL; } break; \
+    case 6: if constexpr (NT >= 6) { constexpr int NP_ = 6; CALL; } break; \
+    case 7: if constexpr (NT >= 7) { constexpr int NP_ = 7; CALL; } break; \
+    case 8: if constexpr (NT >= 8) { constexpr int NP_ = 8; CALL; } break; \
+    default: break;                                 \
+  }
+
 template <int NT, int FMT, int BITS, int GROUP>
 __device__ __forceinline__ void run_tile(const GemmArgs& a, const BlockDesc& d, uint8_t* smem, int nstages,
                                          int stage_b, int wbytes_rf, int n_e, int prow0, int rt, int ks) {
@@ -42,6 +157,7 @@ __device__ __forceinline__ void run_tile(const GemmArgs& a, const BlockDesc& d, 
   const int kc0 = (int)((long long)KC * ks / a.KS), kc1 = (int)((long long)KC * (ks + 1) / a.KS);
   const int nchunks = kc1 - kc0;
   const int rfw = rt * (kWarps * kRF) + warp * kRF;
+  const bool wvalid = rfw + kRF <= MF;  // M % 128 == 0: a warp's fragments are all valid or all past M
   const int ntiles = (n_e + 7) >> 3;
   const long long kblk = a.Kpad_in >> 5;
   constexpr int CB = (FMT == FMT_DENSE) ? 4096 : 256 * BITS;
@@ -69,10 +185,10 @@ __device__ __forceinline__ void run_tile(const GemmArgs& a, const BlockDesc& d, 
         const int t = i >> 7, p = i & 127;
         cp_async16(as + t * 128 + p, a.act + ((tile0 + t) * kblk + kc * 4) * 32 + p);
       }
+      if (wvalid) {
 #pragma unroll
-      for (int r = 0; r < kRF; ++r) {
-        const int rf = rfw + r;
-        if (rf < MF) {
+        for (int r = 0; r < kRF; ++r) {
+          const int rf = rfw + r;
           uint8_t* ws = base + NT * 2048 + (warp * kRF + r) * wbytes_rf;
           if constexpr (FMT == FMT_BITPLANE) {
             for (int pc = lane; pc < 16 * BITS; pc += 32)
@@ -104,127 +220,39 @@ __device__ __forceinline__ void run_tile(const GemmArgs& a, const BlockDesc& d, 
         if (nc < nchunks) load_stage(kc0 + nc, nc % nstages);
         cp_async_commit();
       }
-      const int st = ci % nstages;
-      const uint8_t* base = smem + st * stage_b;
-      const uint4* as = reinterpret_cast<const uint4*>(base);
-      uint32_t w[kRF][8];
-      const uint32_t* ssz[kRF];
-#pragma unroll
-      for (int r = 0; r < kRF; ++r) {
-        const uint8_t* ws = base + NT * 2048 + (warp * kRF + r) * wbytes_rf;
-        ssz[r] = reinterpret_cast<const uint32_t*>(base + NT * 2048 + kWarps * kRF * wbytes_rf +
-                                                   (warp * kRF + r) * kSzBytesPerRf);
-        if constexpr (FMT == FMT_INT && BITS == 4) {
-          const uint4 v0 = reinterpret_cast<const uint4*>(ws)[lane];
-          const uint4 v1 = reinterpret_cast<const uint4*>(ws)[32 + lane];
-          w[r][0] = v0.x; w[r][1] = v0.y; w[r][2] = v0.z; w[r][3] = v0.w;
-          w[r][4] = v1.x; w[r][5] = v1.y; w[r][6] = v1.z; w[r][7] = v1.w;
-        } else if constexpr (FMT == FMT_INT) {
-          const uint4 v0 = reinterpret_cast<const uint4*>(ws)[lane];
-          w[r][0] = v0.x; w[r][1] = v0.y; w[r][2] = v0.z; w[r][3] = v0.w;
-          if constexpr (BITS == 3) {
-            const uint2 h = reinterpret_cast<const uint2*>(ws + 512)[lane];
-            w[r][4] = h.x; w[r][5] = h.y;
-          }
-        } else if constexpr (FMT == FMT_BITPLANE) {
-#pragma unroll
-          for (int p = 0; p < BITS; ++p) {
-            const uint2 v = reinterpret_cast<const uint2*>(ws + p * 256)[lane];
-            w[r][2 * p] = v.x; w[r][2 * p + 1] = v.y;
-          }
-        }
-      }
-      uint32_t sA[kRF], nA[kRF], sB[kRF], nB[kRF];
-      uint4 bq[NT];
-#pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        if ((s & 1) == 0) {
-#pragma unroll
-          for (int t = 0; t < NT; ++t)
-            if (t < np) bq[t] = as[t * 128 + (s >> 1) * 32 + lane];
-        }
-#pragma unroll
-        for (int r = 0; r < kRF; ++r) {
-          if (rfw + r >= MF) continue;
-          uint32_t av[4];
-          if constexpr (FMT == FMT_INT) {
-            if ((16 * s) % GROUP == 0) {
-              const int gs = (16 * s) / GROUP;
-              const uint32_t za = ssz[r][(gs * 8 + g) * 2 + 0];
-              const uint32_t zb = ssz[r][(gs * 8 + g) * 2 + 1];
-              sA[r] = prmt(za, za, 0x1010u); nA[r] = prmt(za, za, 0x3232u);
-              sB[r] = prmt(zb, zb, 0x1010u); nB[r] = prmt(zb, zb, 0x3232u);
-            }
-            uint32_t q[4];
-            int_codes<BITS>(w[r], s, q);
-            av[0] = hfma2u(q[0], sA[r], nA[r]);
-            av[1] = hfma2u(q[1], sB[r], nB[r]);
-            av[2] = hfma2u(q[2], sA[r], nA[r]);
-            av[3] = hfma2u(q[3], sB[r], nB[r]);
-          } else if constexpr (FMT == FMT_BITPLANE) {
-            lut_decode<BITS>(plane_codes<BITS>(w[r], s), lut, av);
-          } else {
-            const uint8_t* ws = base + NT * 2048 + (warp * kRF + r) * wbytes_rf;
-            const uint4 v = reinterpret_cast<const uint4*>(ws)[s * 32 + lane];
-            av[0] = v.x; av[1] = v.y; av[2] = v.z; av[3] = v.w;
-          }
-#pragma unroll
-          for (int t = 0; t < NT; ++t)
-            if (t < np) mma_16816(acc[r][t], av, (s & 1) ? bq[t].z : bq[t].x, (s & 1) ? bq[t].w : bq[t].y);
-        }
+      if (wvalid) {
+        const uint8_t* base = smem + (ci % nstages) * stage_b;
+        MOEQ_DISPATCH_NP(np, (chunk_compute<NP_, NT, FMT, BITS, GROUP>(base, warp, lane, wbytes_rf, lut, acc)))
       }
     }
     cp_async_wait<0>();
     __syncthreads();
 
-    // rank-r compensator columns (one K split adds them)
-    if (ks == 0 && d.rank > 0) {
-      const int RS = d.rank / 16;
-      for (int rs = 0; rs < RS; ++rs) {
-        const long long kk = (a.K >> 5) + (rs >> 1);
-        uint32_t b0[NT], b1[NT];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          b0[t] = b1[t] = 0;
-          if (t < np) {
-            const uint4 v = a.act[((tile0 + t) * kblk + kk) * 32 + lane];
-            b0[t] = (rs & 1) ? v.z : v.x;
-            b1[t] = (rs & 1) ? v.w : v.y;
-          }
-        }
-#pragma unroll
-        for (int r = 0; r < kRF; ++r) {
-          const int rf = rfw + r;
-          if (rf >= MF) continue;
-          const uint4 bv = d.bfrag[((long long)rf * RS + rs) * 32 + lane];
-          const uint32_t av[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-          for (int t = 0; t < NT; ++t)
-            if (t < np) mma_16816(acc[r][t], av, b0[t], b1[t]);
-        }
-      }
+    if (ks == 0 && d.rank > 0 && wvalid) {
+      MOEQ_DISPATCH_NP(np, (ext_compute<NP_, NT>(a, d, rfw, tile0, kblk, lane, acc)))
     }
 
     // epilogue
+    if (wvalid) {
 #pragma unroll
-    for (int r = 0; r < kRF; ++r) {
-      const int rf = rfw + r;
-      if (rf >= MF) continue;
+      for (int r = 0; r < kRF; ++r) {
+        const int rf = rfw + r;
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        if (t >= np) continue;
+        for (int t = 0; t < NT; ++t) {
+          if (t >= np) continue;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int n = (pb + t) * 8 + 2 * c + h;
-          if (n >= n_e) continue;
-          if (a.mode == MODE_SWIGLU) {
-            const float gate = acc[r][t][h], up = acc[r][t][2 + h];
-            const float z = gate / (1.f + expf(-gate)) * up;
-            a.zout[act_frag_index(prow0 + n, 8 * rf + g, a.Kpad_out)] = __float2half_rn(z);
-          } else {
-            float* o = a.out + ks * a.out_ks_stride + (long long)(prow0 + n) * a.M + 16 * rf + g;
-            o[0] = acc[r][t][h];
-            o[8] = acc[r][t][2 + h];
+          for (int h = 0; h < 2; ++h) {
+            const int n = (pb + t) * 8 + 2 * c + h;
+            if (n >= n_e) continue;
+            if (a.mode == MODE_SWIGLU) {
+              const float gate = acc[r][t][h], up = acc[r][t][2 + h];
+              const float z = gate / (1.f + expf(-gate)) * up;
+              a.zout[act_frag_index(prow0 + n, 8 * rf + g, a.Kpad_out)] = __float2half_rn(z);
+            } else {
+              float* o = a.out + ks * a.out_ks_stride + (long long)(prow0 + n) * a.M + 16 * rf + g;
+              o[0] = acc[r][t][h];
+              o[8] = acc[r][t][2 + h];
+            }
           }
         }
       }

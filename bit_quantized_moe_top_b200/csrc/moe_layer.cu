@@ -1,6 +1,7 @@
 // C ABI of the quantized MoE expert layer: ownership, validation, weight
 // loading (device re-layout) and the launch sequence of one forward pass.
 #include <algorithm>
+#include <cmath>
 #include <cstdlib>
 #include <cstring>
 #include <vector>
@@ -501,7 +502,11 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
   };
   // W1 side compensator U1 = X A1^T
   lowrank(0, static_cast<__half*>(L->xact.p), L->Kpad_x, K);
-  const int nt_max = (int)std::min<long long>(8, (std::min<long long>(T, 64) + 7) / 8);
+  // token tiles per pass: cover the expected per-expert batch (mean + 3 sd);
+  // larger batches take more passes
+  const double avg = (double)rows / E;
+  int nt_max = (int)std::ceil((avg + 3.0 * std::sqrt(avg) + 1.0) / 8.0);
+  nt_max = std::max(1, std::min(nt_max, std::min(4, (T + 7) / 8)));
   if (ce == cudaSuccess) {
     GemmArgs ga{};
     ga.experts = dexp;

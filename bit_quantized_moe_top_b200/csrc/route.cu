@@ -11,14 +11,14 @@
 
 namespace moeq {
 
-constexpr int kRouteTokensPerCta = 64;
+constexpr int kRouteTokensPerCta = 16;
 constexpr int kRouteThreads = 256;
 
 __device__ __forceinline__ bool better(float a, int ia, float b, int ib) {
   return a > b || (a == b && ia < ib);
 }
 
-// grid: ceil(T/64) CTAs of 256 threads (8 warps, 8 tokens each).
+// grid: ceil(T/16) CTAs of 256 threads (8 warps, 2 tokens each).
 // The last CTA to finish (atomic ticket) scans the block histograms.
 __global__ void __launch_bounds__(kRouteThreads) route_topk_kernel(RouteArgs a) {
   __shared__ int hist[kMaxExperts];
@@ -143,69 +143,79 @@ __global__ void __launch_bounds__(kRouteThreads) route_topk_kernel(RouteArgs a) 
   }
 }
 
-// grid: same CTAs as route_topk. Ranks within the CTA from per-expert token
-// bitmasks; writes perm/inv_pos and gathers X rows (bf16 -> fp16) into the
-// activation buffer in the layout of the chosen GEMM path.
+// grid: (token blocks of route_topk, K slices). Ranks within the block come
+// from per-expert token bitmasks; slice 0 writes perm/inv_pos; every CTA
+// gathers its K slice of the block's routed rows (bf16 -> fp16) into the
+// activation buffer, in the layout of the chosen GEMM path.
 __global__ void __launch_bounds__(kRouteThreads) route_permute_kernel(RouteArgs a) {
-  __shared__ unsigned long long mask[kMaxExperts];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int e = threadIdx.x; e < a.E; e += blockDim.x) mask[e] = 0ull;
+  __shared__ unsigned mask[kMaxExperts];
+  __shared__ int prow_s[kRouteTokensPerCta * kMaxTopK];
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) mask[e] = 0u;
   __syncthreads();
   const int t0 = blockIdx.x * kRouteTokensPerCta;
   const int nt = min(kRouteTokensPerCta, a.T - t0);
   for (int i = threadIdx.x; i < nt * a.k; i += blockDim.x) {
     const int tt = i / a.k;
     const int e = a.idx[(long long)(t0 + tt) * a.k + (i % a.k)];
-    atomicOr(&mask[e], 1ull << tt);
+    atomicOr(&mask[e], 1u << tt);
   }
   __syncthreads();
   for (int i = threadIdx.x; i < nt * a.k; i += blockDim.x) {
     const int tt = i / a.k, j = i % a.k;
     const int t = t0 + tt;
     const int e = a.idx[(long long)t * a.k + j];
-    const int rank = __popcll(mask[e] & ((1ull << tt) - 1ull));
+    const int rank = __popc(mask[e] & ((1u << tt) - 1u));
     const long long bi = (long long)blockIdx.x * a.E + e;
-    const int pos = a.block_base[bi] + rank;
     const int ppos = a.pblock_base[bi] + rank;
-    a.perm_token[pos] = t;
-    a.inv_pos[(long long)t * a.k + j] = pos;
-    a.pinv[(long long)t * a.k + j] = ppos;
+    prow_s[i] = ppos;
+    if (blockIdx.y == 0) {
+      const int pos = a.block_base[bi] + rank;
+      a.perm_token[pos] = t;
+      a.inv_pos[(long long)t * a.k + j] = pos;
+      a.pinv[(long long)t * a.k + j] = ppos;
+    }
   }
-  // gather: one warp per routed (token, slot)
+  __syncthreads();
+  // gather of this CTA's K slice
   const int Kq = a.K;
-  for (int i = warp; i < nt * a.k; i += 8) {
-    const int tt = i / a.k, j = i % a.k;
-    const int t = t0 + tt;
-    const int e = a.idx[(long long)t * a.k + j];
-    const int rank = __popcll(mask[e] & ((1ull << tt) - 1ull));
-    const long long prow = a.pblock_base[(long long)blockIdx.x * a.E + e] + rank;
-    const __nv_bfloat16* x = a.X + (long long)t * Kq;
-    if (a.act_layout == ACT_FRAG) {
-      // lane (g', c') of k-block kk: one uint4 of row prow
-      const int c = lane & 3;
-      const long long nt8 = prow >> 3;
-      const int g = (int)(prow & 7);
-      for (int kk = lane >> 2; kk < Kq / 32; kk += 8) {
-        uint32_t v[4];
+  const int ks0 = (int)((long long)Kq * blockIdx.y / gridDim.y), ks1 = (int)((long long)Kq * (blockIdx.y + 1) / gridDim.y);
+  if (a.act_layout == ACT_FRAG) {
+    // one item = one uint4 of B fragments: (routed row, 32-wide k block, c)
+    const int kb0 = ks0 / 32, nkb = ks1 / 32 - kb0;
+    const int items = nt * a.k * nkb * 4;
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+      const int c = it & 3;
+      const int rest = it >> 2;
+      const int kb = kb0 + rest % nkb;
+      const int i = rest / nkb;
+      const int t = t0 + i / a.k;
+      const long long prow = prow_s[i];
+      const __nv_bfloat16* x = a.X + (long long)t * Kq;
+      uint32_t v[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int k = 32 * kk + 2 * c + 8 * q;
-          const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(x + k);
-          v[q] = pack_half2(__bfloat162float(b2.x), __bfloat162float(b2.y));
-        }
-        uint4* dst = reinterpret_cast<uint4*>(a.act) + (nt8 * (a.Kpad >> 5) + kk) * 32 + g * 4 + c;
-        *dst = make_uint4(v[0], v[1], v[2], v[3]);
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(x + 32 * kb + 2 * c + 8 * q);
+        v[q] = pack_half2(__bfloat162float(b2.x), __bfloat162float(b2.y));
       }
-    } else {
-      __half* dst = reinterpret_cast<__half*>(a.act) + prow * a.Kpad;
-      for (int k = lane * 8; k < Kq; k += 256) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(x + k);
-        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&raw);
-        uint32_t v[4];
+      uint4* dst = reinterpret_cast<uint4*>(a.act) + ((prow >> 3) * (a.Kpad >> 5) + kb) * 32 + (prow & 7) * 4 + c;
+      *dst = make_uint4(v[0], v[1], v[2], v[3]);
+    }
+  } else {
+    // one item = 8 consecutive elements of a routed row
+    const int k80 = ks0 / 8, nk8 = ks1 / 8 - k80;
+    const int items = nt * a.k * nk8;
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+      const int k8 = k80 + it % nk8;
+      const int i = it / nk8;
+      const int t = t0 + i / a.k;
+      const long long prow = prow_s[i];
+      const uint4 raw = *reinterpret_cast<const uint4*>(a.X + (long long)t * Kq + 8 * k8);
+      const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      uint32_t v[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) v[q] = pack_half2(__bfloat162float(b[q].x), __bfloat162float(b[q].y));
-        *reinterpret_cast<uint4*>(dst + k) = make_uint4(v[0], v[1], v[2], v[3]);
-      }
+      for (int q = 0; q < 4; ++q) v[q] = pack_half2(__bfloat162float(b[q].x), __bfloat162float(b[q].y));
+      *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(a.act) + prow * a.Kpad + 8 * k8) =
+          make_uint4(v[0], v[1], v[2], v[3]);
     }
   }
 }
@@ -219,7 +229,9 @@ cudaError_t launch_route_topk(const RouteArgs& a, cudaStream_t st, int* launches
 
 cudaError_t launch_route_permute(const RouteArgs& a, cudaStream_t st, int* launches) {
   const int nb = (a.T + kRouteTokensPerCta - 1) / kRouteTokensPerCta;
-  route_permute_kernel<<<nb, kRouteThreads, 0, st>>>(a);
+  int gs = 296 / nb;
+  gs = gs < 1 ? 1 : gs > a.K / 256 ? a.K / 256 : gs;
+  route_permute_kernel<<<dim3(nb, gs), kRouteThreads, 0, st>>>(a);
   if (launches) ++*launches;
   return cudaGetLastError();
 }
