@@ -17,7 +17,8 @@ LIB_PATH = os.path.join(HERE, "libmoeq.so")
 
 MOE_OK = 0
 STATUS_NAMES = ["MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_OOM", "MOE_ERR_NOT_LOADED", "MOE_ERR_UNSUPPORTED",
-                "MOE_ERR_BITS_UNAVAILABLE", "MOE_ERR_CUDA", "MOE_ERR_DEVICE_CHECK", "MOE_ERR_TIMEOUT"]
+                "MOE_ERR_BITS_UNAVAILABLE", "MOE_ERR_CUDA", "MOE_ERR_DEVICE_CHECK", "MOE_ERR_TIMEOUT",
+                "MOE_ERR_TOO_LARGE"]
 FMT_INT_ASYM, FMT_BITPLANE_LUT, FMT_DENSE16 = 0, 1, 2
 FLAG_NO_TOPK_RENORM = 1
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
@@ -26,7 +27,7 @@ PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 EXPORTS = ["moe_layer_create", "moe_layer_set_expert_weights", "moe_layer_set_bits", "moe_layer_set_path",
            "moe_layer_forward", "moe_layer_forward_host", "moe_layer_get_routing", "moe_layer_debug_unpack",
            "moe_layer_sync_status", "moe_layer_last_launch_count", "moe_layer_set_profiling",
-           "moe_layer_kernel_times", "moe_status_string", "moe_layer_destroy"]
+           "moe_layer_kernel_times", "moe_route_topk_noalloc", "moe_status_string", "moe_layer_destroy"]
 
 
 class MoEError(RuntimeError):
@@ -63,6 +64,7 @@ def _lib() -> ctypes.CDLL:
         lib.moe_layer_last_launch_count.argtypes = [P]
         lib.moe_layer_set_profiling.argtypes = [P, I]
         lib.moe_layer_kernel_times.argtypes = [P, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float), I]
+        lib.moe_route_topk_noalloc.argtypes = [P, I, I, I, U, P, P, P, P, P]
         lib.moe_status_string.argtypes = [I]
         lib.moe_status_string.restype = ctypes.c_char_p
         lib.moe_layer_destroy.argtypes = [P]
@@ -158,6 +160,18 @@ def moe_layer_kernel_times(layer: int, cap: int = 64):
     if n < 0:
         return []
     return [(names[i].decode(), float(ms[i])) for i in range(min(n, cap))]
+
+
+def moe_route_topk_noalloc(logits, top_k: int, idx, w, counts, offsets, flags: int = 0,
+                           stream: Optional[int] = None) -> None:
+    """Top-k routing with no device allocation (scratch lives in the library
+    image): for callers that may not allocate device memory themselves."""
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(logits.device).cuda_stream
+    T, E = logits.shape
+    _check(_lib().moe_route_topk_noalloc(_ptr(logits), T, E, top_k, flags, _ptr(idx), _ptr(w), _ptr(counts),
+                                         _ptr(offsets), stream), "moe_route_topk_noalloc")
 
 
 def moe_status_string(status: int) -> str:

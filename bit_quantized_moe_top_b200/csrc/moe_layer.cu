@@ -135,6 +135,7 @@ const char* moe_status_string(moe_status_t s) {
     case MOE_ERR_CUDA: return "CUDA error";
     case MOE_ERR_DEVICE_CHECK: return "device-side check failed";
     case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_TOO_LARGE: return "request exceeds a fixed capacity";
   }
   return "unknown status";
 }

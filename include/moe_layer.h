@@ -69,7 +69,8 @@ typedef enum {
   MOE_ERR_BITS_UNAVAILABLE = 5, /* set_bits asks for planes that are not stored */
   MOE_ERR_CUDA = 6,             /* a CUDA runtime call failed */
   MOE_ERR_DEVICE_CHECK = 7,     /* a kernel's own check failed (status word) */
-  MOE_ERR_TIMEOUT = 8           /* a bounded device-side wait gave up */
+  MOE_ERR_TIMEOUT = 8,          /* a bounded device-side wait gave up */
+  MOE_ERR_TOO_LARGE = 9         /* request exceeds a fixed capacity (moe_route_topk_noalloc) */
 } moe_status_t;
 
 typedef enum {
@@ -171,6 +172,27 @@ moe_status_t moe_layer_set_profiling(moe_layer_t* layer, int enable);
  * names[i] (static strings) and ms[i] for i < min(count, cap). Synchronises the
  * stream. Returns the count, or -1 if nothing was profiled. */
 int moe_layer_kernel_times(moe_layer_t* layer, const char** names, float* ms, int cap);
+
+/* Routing without any device allocation. The pages have no counterpart of
+ * this call; it exists for callers that cannot allocate device memory: a
+ * plugin or extension whose host framework owns all device memory, or a
+ * serving loop that must not pay the implicit device-wide synchronisation of
+ * cudaMalloc/cudaFree. It runs the layer's top-k routing kernel (the same
+ * selection and weights as moe_layer_forward) with its scratch in a fixed
+ * 196 KiB array that is part of the library image on every GPU that loads the
+ * library, kept until the process exits.
+ *   logits: fp32 [T, E] device. Outputs (device, caller-allocated): idx int32
+ *   [T, top_k], w fp32 [T, top_k], counts int32 [E], offsets int32 [E+1].
+ *   flags: 0 or MOE_FLAG_NO_TOPK_RENORM. Asynchronous on cuda_stream.
+ *   Capacity: ceil(T / 16) * E <= 16384 (e.g. T <= 4096 at E = 64, T <= 1024 at
+ *   E = 256); larger requests return MOE_ERR_TOO_LARGE before any launch.
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture. Every call
+ * shares the one array and clears the words that must start at zero, so calls
+ * whose kernels overlap on the GPU (concurrent streams or threads) race and
+ * must be serialised by the caller. Calls no allocating routine. */
+moe_status_t moe_route_topk_noalloc(const float* router_logits, int T, int E, int top_k, unsigned flags, int* idx,
+                                    float* w, int* counts, int* offsets, void* cuda_stream);
 
 const char* moe_status_string(moe_status_t status);
 
