@@ -27,7 +27,8 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = "mixtral8x7b_decode"
+WORKLOADS = {"mixtral_decode": "mixtral8x7b_decode", "mixtral_prefill": "mixtral8x7b_prefill",
+             "dsv2lite_decode": "deepseek_v2_lite_decode", "dsv3_bitplane": "deepseek_v3_bitplane", "tiny": "tiny"}
 
 
 def parse():
@@ -84,6 +85,21 @@ def gemm1_bytes(cfg, counts):
     return tot
 
 
+def gemm1_flops(cfg, counts):
+    """Algorithmic flops of one gate/up GEMM launch: 2 * rows * 2N * (K + r)."""
+    return sum(2.0 * n * 2 * cfg.N * (cfg.K + cfg.experts[e].rank) for e, n in enumerate(counts))
+
+
+def layer_flops(cfg, counts):
+    """2 * rows * 3NK for the three projections plus the compensator terms
+    2 * rows * r * (2K + 3N)."""
+    tot = 0.0
+    for e, n in enumerate(counts):
+        r = cfg.experts[e].rank
+        tot += 2.0 * n * 3 * cfg.N * cfg.K + 2.0 * n * r * (2 * cfg.K + 3 * cfg.N)
+    return tot
+
+
 # ---------------------------------------------------------------------------
 # clocks sampled during the timed region (NVML reads only)
 # ---------------------------------------------------------------------------
@@ -137,12 +153,13 @@ class ClockSampler:
 
 
 def measured_peaks():
+    """(HBM GB/s, dense bf16 TFLOP/s burst, sustained, source)."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             d = json.load(f)
-        return d["hbm_gbs"], d.get("bf16_tflops"), "measured"
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
     except Exception:
-        return 6650.0, 1590.0, "fallback"
+        return 6650.0, 1590.0, 1400.0, "fallback"
 
 
 # ---------------------------------------------------------------------------
@@ -215,7 +232,7 @@ def main():
         line = {"impl": "reference", "metric": "MoE-layer tokens/s", "value": val, "unit": "tokens/s",
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "config": {"workload": f"{WORKLOAD}_T{T}", "T": T},
+                "data": "synthetic", "config": {"workload": f"{WORKLOADS[args.config]}_T{T}", "T": T},
                 "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": rates[0][3], "kind": "oracle",
                                  "sample": f"first {rates[0][1]} token(s) of the T={T} batch per step, one token "
                                            f"at a time (its experts dequantised in fp64)"},
@@ -281,13 +298,28 @@ def main():
     ms_per_step = total_ms / args.steps
     value = world * T / (ms_per_step / 1000.0)
 
-    # dominant kernel: gate/up GEMM (2/3 of the weight bytes)
-    k1 = statistics.mean(kt.get("decode_gemm_w1_swiglu", [float("nan")]))
-    hbm_peak, _, peak_src = measured_peaks()
-    b1 = gemm1_bytes(cfg, counts)
-    achieved = b1 / (k1 * 1e-3) / 1e9
-    layer_b = layer_bytes(cfg, counts, T)
+    # dominant kernel: the gate/up GEMM (2/3 of the weight bytes and flops)
+    hbm_peak, tc_peak, tc_sustained, peak_src = measured_peaks()
     kernel_means = {k: statistics.mean(v) for k, v in kt.items()}
+    prefill = "prefill_gemm_w1_swiglu" in kernel_means
+    kname = "prefill_gemm_w1_swiglu" if prefill else "decode_gemm_w1_swiglu"
+    k1 = kernel_means.get(kname, float("nan"))
+    layer_b = layer_bytes(cfg, counts, T)
+    layer_f = layer_flops(cfg, counts)
+    if prefill:
+        f1 = gemm1_flops(cfg, counts)
+        achieved = f1 / (k1 * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": tc_sustained,
+                    "unit": "TFLOP/s", "frac": achieved / tc_sustained, "traffic": None,
+                    "peak_source": f"{peak_src} bf16 sustained (fp16 has the same dense rate)",
+                    "frac_of_burst_peak": achieved / tc_peak, "algorithmic_flops_per_launch": f1,
+                    "launch_ms": k1}
+    else:
+        b1 = gemm1_bytes(cfg, counts)
+        achieved = b1 / (k1 * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": achieved / hbm_peak, "traffic": None, "peak_source": peak_src,
+                    "algorithmic_bytes_per_launch": b1, "launch_ms": k1}
 
     # end to end: host buffers through moe_layer_forward_host (copies inside the timed region)
     Xh = X.cpu().pin_memory()
@@ -322,14 +354,18 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16 operands, f32 accumulate",
             "data": "synthetic",
-            "config": {"workload": f"{WORKLOAD}_T{T}", "T": T, "E": cfg.E, "top_k": cfg.top_k, "d_model": cfg.K,
-                       "d_ff": cfg.N, "bits": 3, "group": 128, "rank": 32, "parallelism": f"replicas x{world}",
-                       "l2": "flushed between steps (256 MiB write, untimed); weights 599 MB > L2"},
+            "config": {"workload": f"{WORKLOADS[args.config]}_T{T}", "T": T, "E": cfg.E, "top_k": cfg.top_k,
+                       "d_model": cfg.K, "d_ff": cfg.N,
+                       "bits": sorted(set(b for sp in cfg.experts for b in sp.bits)),
+                       "format": "bit-plane+LUT" if cfg.experts[0].fmt == 1 else "int asym",
+                       "group": cfg.experts[0].group, "ranks": sorted(set(sp.rank for sp in cfg.experts)),
+                       "parallelism": f"replicas x{world}",
+                       "l2": "flushed between steps (256 MiB write, untimed)"},
             "layer_hbm_gbs": layer_b / (ms_per_step * 1e-3) / 1e9,
+            "layer_tflops": layer_f / (ms_per_step * 1e-3) / 1e12,
             "layer_bytes_per_step": layer_b,
-            "roofline": {"bound": "hbm", "kernel": "decode_gemm_w1_swiglu", "achieved": achieved, "peak": hbm_peak,
-                         "unit": "GB/s", "frac": achieved / hbm_peak, "traffic": None,
-                         "peak_source": peak_src, "algorithmic_bytes_per_launch": b1, "launch_ms": k1},
+            "layer_flops_per_step": layer_f,
+            "roofline": roofline,
             "kernels_ms": kernel_means,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": T * cfg.K * 2 + T * cfg.E * 4,

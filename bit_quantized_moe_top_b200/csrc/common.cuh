@@ -13,8 +13,10 @@
 //    A registers a0a1, a2a3, a4a5, a6a7), half h (0/1) is the element
 //    (row 16rf + g + 8*(j&1), k = 128kc + 16s + 2c + 8*(j>>1) + h).
 //    A chunk holds 256*b bytes (b = bits; 16 for dense fp16).
-//  * Activations for the mma.sync path are stored per (8-row tile, 32-wide k
-//    block) as 32 lanes x uint4 = the B fragments of two k16 steps.
+//  * Chunks are stored chunk-major: [kc][rf] (bit-planes: [plane][kc][rf]), so
+//    the 16 row fragments a CTA streams for one chunk are one contiguous range.
+//  * Activations for the mma.sync path are stored per (128-wide k chunk, 8-row
+//    tile) as 4 k32 blocks x 32 lanes x uint4 = B fragments of 8 k16 steps.
 #pragma once
 #include <cstdint>
 #include <cuda_fp16.h>
@@ -34,12 +36,12 @@ enum : unsigned { ST_BOUNDS = 1u, ST_TIMEOUT = 2u, ST_ROUTE = 4u };
 
 // One expert linear block as the kernels see it.
 struct BlockDesc {
-  const uint8_t* codes;   // internal chunked codes (INT / DENSE) or plane 0 (BITPLANE)
-  const uint32_t* sz;     // INT: [MF][K/g][8] uint2 = half2(s, -z*s) for rows g and g+8
+  const uint8_t* codes;   // chunked codes [kc][rf][256*b bytes] (INT / DENSE) or plane 0 (BITPLANE)
+  const uint32_t* sz;     // INT: [K/g][MF][8] uint2 = half2(s, -z*s) for rows g and g+8
   const uint32_t* lut;    // BITPLANE: 28 fp16 as 14 u32
   const uint4* bfrag;     // compensator B [M, r] as dense A-fragments [MF][r/16][32] uint4 (fp16)
   const uint4* afrag;     // compensator A [r, K] as dense A-fragments [r/16][K/16][32] uint4 (fp16)
-  long long plane_stride; // BITPLANE: bytes between planes
+  long long plane_stride; // BITPLANE: bytes between planes ([kc][rf][256] each)
   int fmt, bits, group, rank;
   int M, K;
   int loaded;
@@ -137,17 +139,78 @@ __host__ __device__ __forceinline__ void frag_elem(int lane, int s, int j, int h
   k = 16 * s + 2 * c + 8 * (j >> 1) + h;
 }
 
-// Activation B-fragment layout: element (row n, col k) of a [rows, Kpad]
-// activation matrix, Kpad % 32 == 0. Returns the fp16 index.
-__host__ __device__ __forceinline__ long long act_frag_index(long long n, int k, int Kpad) {
-  long long nt = n >> 3;
-  int g = (int)(n & 7);
-  int kk = k >> 5, kin = k & 31;
-  int step = kin >> 4, k16 = kin & 15;
-  int hi = k16 >> 3, c = (k16 & 7) >> 1, h = k16 & 1;
-  int lane = g * 4 + c;
-  int comp = step * 2 + hi;  // u32 within the uint4
-  return ((nt * (Kpad >> 5) + kk) * 32 + lane) * 8 + comp * 2 + h;
+// Activation B-fragment layout, chunk-major: for each 128-wide k chunk kc,
+// the 8-row tiles nt of the whole buffer (capacity nt8cap tiles) follow each
+// other, each holding 4 k32 blocks x 32 lanes x uint4 (2 KiB). An expert's
+// consecutive row tiles of one chunk are therefore one contiguous range.
+// Returns the fp16 index of element (row n, col k).
+__host__ __device__ __forceinline__ long long act_frag_index(long long n, int k, long long nt8cap) {
+  const long long nt = n >> 3;
+  const int g = (int)(n & 7);
+  const int kc = k >> 7, kin = k & 127;
+  const int kk = kin >> 5, k32 = kin & 31;
+  const int step = k32 >> 4, k16 = k32 & 15;
+  const int hi = k16 >> 3, c = (k16 & 7) >> 1, h = k16 & 1;
+  const int lane = g * 4 + c;
+  const int comp = step * 2 + hi;
+  return ((((long long)kc * nt8cap + nt) * 4 + kk) * 32 + lane) * 8 + comp * 2 + h;
+}
+// uint4 index of the B fragments of k16 steps (2*kk2, 2*kk2+1) of row tile nt
+// (kk2 = k / 32 over the whole row)
+__host__ __device__ __forceinline__ long long act_frag_u4(long long nt, int kk2, long long nt8cap, int lane) {
+  return ((((long long)(kk2 >> 2) * nt8cap + nt) * 4 + (kk2 & 3)) * 32 + lane);
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier / bulk-copy helpers (TMA engine, no multicast)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+  return t;
+}
+// Bounded wait: gives up after ~limit_ns, sets ST_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* status,
+                                          unsigned long long limit_ns = 2000000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      atomicOr(status, ST_TIMEOUT);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
 }
 
 }  // namespace moeq

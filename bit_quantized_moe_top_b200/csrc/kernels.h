@@ -1,5 +1,6 @@
 // Internal launch interface between the C-ABI host code and the kernels.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include "common.cuh"
 
@@ -27,7 +28,8 @@ struct RouteArgs {
   int* inv_pos;               // [T, k]
   int* pinv;                  // [T, k] padded row
   void* act;                  // activation buffer (fp16), layout act_layout
-  int Kpad;                   // activation row width (elements)
+  int Kpad;                   // ACT_ROW: row width (elements)
+  long long nt8cap;           // ACT_FRAG: row-tile capacity of the buffer
   int act_layout;
   unsigned* status;
 };
@@ -40,12 +42,11 @@ struct GemmArgs {
   const int* counts;
   const int* poffsets;
   const uint4* act;           // input activations (fragment layout)
-  int Kpad_in;
+  long long nt8cap;           // row-tile capacity of the activation buffers
   int K;                      // quantised K of the block
   int M;                      // rows of the block
   int mode;
   __half* zout;               // MODE_SWIGLU: output activations (fragment layout)
-  int Kpad_out;
   float* out;                 // MODE_OUT: [KS][prows][M] fp32 partials
   long long out_ks_stride;
   int KS;
@@ -60,13 +61,31 @@ struct LowrankArgs {
   const int* counts;
   const int* poffsets;
   __half* act;                // activation buffer; reads [0,K), writes ext columns [K, K+r)
-  int Kpad;
+  int Kpad;                   // ACT_ROW: row width
+  long long nt8cap;           // ACT_FRAG: row-tile capacity
   int K;
   int KS;
   float* part;                // [KS][prows][64]
   long long part_ks_stride;
   int* sem;                   // [E], zero between launches
   int act_layout;
+  unsigned* status;
+};
+
+struct PrefillArgs {
+  CUtensorMap tmap_act;       // activations [rows, Kpad] fp16 row-major; box 64 x 128, 128-byte swizzle
+  const ExpertDesc* experts;
+  int block;
+  const int* active;
+  const int* n_active;
+  const int* counts;
+  const int* poffsets;
+  int K;                      // quantised K of the block
+  int M;                      // rows of the block
+  int mode;
+  __half* zout;               // MODE_SWIGLU: output rows (fp16), leading dimension ldz
+  long long ldz;
+  float* out;                 // MODE_OUT: [prows][M] fp32
   unsigned* status;
 };
 
@@ -85,7 +104,7 @@ cudaError_t launch_relayout_int(const uint8_t* canon, uint8_t* out, int M, int K
 cudaError_t launch_relayout_sz(const __half* s, const __half* z, uint32_t* out, int M, int K, int group, int block,
                                int N, cudaStream_t st);
 cudaError_t launch_relayout_dense(const __nv_bfloat16* src, uint4* out, int M, int K, int block, int N, long long ld,
-                                  cudaStream_t st);
+                                  int chunked, cudaStream_t st);
 cudaError_t launch_relayout_planes(const uint32_t* canon, uint32_t* out, int M, int K, int block, int N,
                                    cudaStream_t st);
 cudaError_t launch_debug_unpack(const BlockDesc& d, uint8_t* out, int block, int N, cudaStream_t st);
@@ -100,6 +119,8 @@ size_t decode_smem_bytes(int nt, int maxbits);
 cudaError_t launch_decode_gemm(const GemmArgs& a, int nt_max, int maxbits, int grid_y, cudaStream_t st,
                                int* launches);
 cudaError_t launch_lowrank(const LowrankArgs& a, int grid_y, cudaStream_t st, int* launches);
+cudaError_t launch_prefill_gemm(const PrefillArgs& a, int grid_y, int grid_z, cudaStream_t st, int* launches);
+int prefill_smem_bytes();
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st, int* launches);
 
 }  // namespace moeq

@@ -36,7 +36,6 @@ __global__ void __launch_bounds__(256) lowrank_kernel(LowrankArgs a) {
   const int s0 = (int)((long long)S16 * ks / a.KS), s1 = (int)((long long)S16 * (ks + 1) / a.KS);
   const int prow0 = a.poffsets[e];
   const int ntiles = (n_e + 7) >> 3;
-  const long long kblk = a.Kpad >> 5;
   const uint4* act4 = reinterpret_cast<const uint4*>(a.act);
   for (int pb = 0; pb < ntiles; pb += kLrNT) {
     const int np = min(kLrNT, ntiles - pb);
@@ -55,7 +54,7 @@ __global__ void __launch_bounds__(256) lowrank_kernel(LowrankArgs a) {
         if (t < np) {
           const long long n0 = prow0 + 8LL * (pb + t);
           if (a.act_layout == ACT_FRAG) {
-            const uint4 v = act4[((n0 >> 3) * kblk + (S >> 1)) * 32 + lane];
+            const uint4 v = act4[act_frag_u4(n0 >> 3, S >> 1, a.nt8cap, lane)];
             b0[t] = (S & 1) ? v.z : v.x;
             b1[t] = (S & 1) ? v.w : v.y;
           } else {
@@ -111,7 +110,7 @@ __global__ void __launch_bounds__(256) lowrank_kernel(LowrankArgs a) {
     float s = 0.f;
     for (int k2 = 0; k2 < a.KS; ++k2) s += __ldcg(a.part + k2 * a.part_ks_stride + (long long)(prow0 + n) * kMaxRank + j);
     const __half hv = __float2half_rn(s);
-    if (a.act_layout == ACT_FRAG) a.act[act_frag_index(prow0 + n, a.K + j, a.Kpad)] = hv;
+    if (a.act_layout == ACT_FRAG) a.act[act_frag_index(prow0 + n, a.K + j, a.nt8cap)] = hv;
     else a.act[(long long)(prow0 + n) * a.Kpad + a.K + j] = hv;
   }
   if (threadIdx.x == 0) a.sem[e] = 0;

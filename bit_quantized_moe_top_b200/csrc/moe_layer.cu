@@ -6,6 +6,8 @@
 #include <cstring>
 #include <vector>
 
+#include <cudaTypedefs.h>
+
 #include "../../include/moe_layer.h"
 #include "kernels.h"
 
@@ -60,12 +62,14 @@ struct moe_layer {
   DevBuf d_experts;
   // workspace
   int rmax_pad = 0, Kpad_x = 0, Kpad_z = 0;
-  long long rows_pad_max = 0;
+  long long rows_pad_max = 0, nt8cap = 0;
   int nb_max = 0, ks2_max = 1, kslr_max = 1;
   DevBuf idx, w, counts, offsets, poffsets, active, n_active, ticket, perm, inv_pos, pinv;
   DevBuf block_counts, block_base, pblock_base, sem, status;
   DevBuf xact, zact, obuf, part;
   DevBuf hx, hl, hy;  // device buffers for forward_host
+  CUtensorMap tmap_x, tmap_z;  // row-layout activation buffers for the prefill GEMMs
+  bool have_tmaps = false;
   int last_T = 0, last_k = 0, last_launches = 0;
   cudaStream_t last_stream = nullptr;
   // profiling: events around each launch of the last forward
@@ -95,6 +99,27 @@ static void prof_end(moe_layer_t* L, cudaStream_t st) {
 }
 
 static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// 2-D tensor map over a row-major fp16 [rows, cols] buffer: box 64 columns x
+// 128 rows, 128-byte swizzle, zero fill outside the buffer.
+static bool encode_act_map(CUtensorMap* map, void* base, int cols, long long rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p)
+      return false;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 static bool valid_desc(const moe_expert_desc_t& d, int K, int N) {
   if (d.rank < 0 || d.rank > kMaxRank) return false;
@@ -193,6 +218,7 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   L->Kpad_z = N + L->rmax_pad;
   const long long rows = (long long)max_tokens * max_top_k;
   L->rows_pad_max = (rows + 7LL * E + 7) / 8 * 8;
+  L->nt8cap = L->rows_pad_max / 8;
   L->nb_max = route_num_blocks(max_tokens);
   L->ks2_max = 16;
   L->kslr_max = 32;
@@ -220,8 +246,9 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   A(L->pblock_base, sizeof(int) * (size_t)L->nb_max * E);
   A(L->sem, sizeof(int) * E);
   A(L->status, sizeof(unsigned));
-  A(L->xact, sizeof(__half) * (size_t)L->rows_pad_max * L->Kpad_x);
-  A(L->zact, sizeof(__half) * (size_t)L->rows_pad_max * L->Kpad_z);
+  const size_t kx = (size_t)(L->Kpad_x + 127) / 128 * 128, kz = (size_t)(L->Kpad_z + 127) / 128 * 128;
+  A(L->xact, sizeof(__half) * (size_t)L->rows_pad_max * kx);
+  A(L->zact, sizeof(__half) * (size_t)L->rows_pad_max * kz);
   A(L->obuf, sizeof(float) * (size_t)o_elems * K);
   A(L->part, sizeof(float) * (size_t)L->kslr_max * L->rows_pad_max * kMaxRank);
   A(L->hx, sizeof(__nv_bfloat16) * (size_t)max_tokens * K);
@@ -242,6 +269,8 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
     moe_layer_destroy(L);
     return MOE_ERR_CUDA;
   }
+  L->have_tmaps = encode_act_map(&L->tmap_x, L->xact.p, L->Kpad_x, L->rows_pad_max) &&
+                  encode_act_map(&L->tmap_z, L->zact.p, L->Kpad_z, L->rows_pad_max);
   *out = L;
   return MOE_OK;
 }
@@ -316,7 +345,7 @@ moe_status_t moe_layer_set_expert_weights(moe_layer_t* L, int e, int block, cons
     if (st == MOE_OK) st = dalloc(S.codes, nbytes);
     if (st == MOE_OK)
       ce = launch_relayout_dense(static_cast<const __nv_bfloat16*>(dc), static_cast<uint4*>(S.codes.p), M, Kin, block,
-                                 L->N, Kin, s0);
+                                 L->N, Kin, 1, s0);
   }
   if (st == MOE_OK && ce == cudaSuccess && r > 0) {
     // factors padded with zeros to the k16 rank r (caller rank r0 <= r)
@@ -338,10 +367,10 @@ moe_status_t moe_layer_set_expert_weights(moe_layer_t* L, int e, int block, cons
     if (st == MOE_OK) st = dalloc(S.bfrag, (size_t)M * r * sizeof(__half));
     if (st == MOE_OK && ce == cudaSuccess) {
       ce = launch_relayout_dense(static_cast<const __nv_bfloat16*>(da), static_cast<uint4*>(S.afrag.p), r, Kin, -1,
-                                 L->N, Kin, s0);
+                                 L->N, Kin, 0, s0);
       if (ce == cudaSuccess)
         ce = launch_relayout_dense(static_cast<const __nv_bfloat16*>(db), static_cast<uint4*>(S.bfrag.p), M, r, block,
-                                   L->N, r, s0);
+                                   L->N, r, 0, s0);
     }
   }
   if (st == MOE_OK && ce == cudaSuccess) ce = cudaDeviceSynchronize();
@@ -426,9 +455,13 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     return MOE_ERR_INVALID_ARG;
   for (int e = 0; e < L->E; ++e)
     if (!L->hdesc[e].blk[0].loaded || !L->hdesc[e].blk[1].loaded) return MOE_ERR_NOT_LOADED;
+  bool any_dense = false;
+  for (int e = 0; e < L->E; ++e) any_dense |= L->hdesc[e].blk[0].fmt == FMT_DENSE;
   int path = L->path;
-  if (path == MOE_PATH_AUTO) path = MOE_PATH_DECODE;
-  if (path != MOE_PATH_DECODE) return MOE_ERR_UNSUPPORTED;
+  if (path == MOE_PATH_AUTO)
+    path = ((long long)T * top_k >= 64LL * L->E && !any_dense && L->have_tmaps) ? MOE_PATH_PREFILL : MOE_PATH_DECODE;
+  if (path == MOE_PATH_PREFILL && (any_dense || !L->have_tmaps)) return MOE_ERR_UNSUPPORTED;
+  const bool prefill = path == MOE_PATH_PREFILL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int E = L->E, K = L->K, N = L->N;
   int maxbits[2] = {0, 0}, rmax = 0;
@@ -468,7 +501,8 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
   ra.pinv = static_cast<int*>(L->pinv.p);
   ra.act = L->xact.p;
   ra.Kpad = L->Kpad_x;
-  ra.act_layout = ACT_FRAG;
+  ra.nt8cap = L->nt8cap;
+  ra.act_layout = prefill ? ACT_ROW : ACT_FRAG;
   ra.status = static_cast<unsigned*>(L->status.p);
   L->prof_names.clear();
   prof_mark(L, st, "route_topk");
@@ -489,6 +523,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     la.poffsets = ra.poffsets;
     la.act = act;
     la.Kpad = Kpad;
+    la.nt8cap = L->nt8cap;
     la.K = Kin;
     int ks = 296 / grid_y;
     ks = std::max(1, std::min(ks, std::min(L->kslr_max, Kin / 16 / 8)));
@@ -496,64 +531,92 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     la.part = static_cast<float*>(L->part.p);
     la.part_ks_stride = (long long)L->rows_pad_max * kMaxRank;
     la.sem = static_cast<int*>(L->sem.p);
-    la.act_layout = ACT_FRAG;
+    la.act_layout = prefill ? ACT_ROW : ACT_FRAG;
     la.status = ra.status;
     prof_mark(L, st, block == 0 ? "lowrank_w1" : "lowrank_w2");
     ce = launch_lowrank(la, grid_y, st, &launches);
   };
   // W1 side compensator U1 = X A1^T
   lowrank(0, static_cast<__half*>(L->xact.p), L->Kpad_x, K);
-  // token tiles per pass: cover the expected per-expert batch (mean + 3 sd);
-  // larger batches take more passes
-  const double avg = (double)rows / E;
-  int nt_max = (int)std::ceil((avg + 3.0 * std::sqrt(avg) + 1.0) / 8.0);
-  nt_max = std::max(1, std::min(nt_max, std::min(4, (T + 7) / 8)));
-  if (ce == cudaSuccess) {
-    GemmArgs ga{};
-    ga.experts = dexp;
-    ga.block = 0;
-    ga.active = ra.active;
-    ga.n_active = ra.n_active;
-    ga.counts = ra.counts;
-    ga.poffsets = ra.poffsets;
-    ga.act = static_cast<const uint4*>(L->xact.p);
-    ga.Kpad_in = L->Kpad_x;
-    ga.K = K;
-    ga.M = 2 * N;
-    ga.mode = MODE_SWIGLU;
-    ga.zout = static_cast<__half*>(L->zact.p);
-    ga.Kpad_out = L->Kpad_z;
-    ga.KS = 1;
-    ga.status = ra.status;
-    prof_mark(L, st, "decode_gemm_w1_swiglu");
-    ce = launch_decode_gemm(ga, nt_max, maxbits[0], grid_y, st, &launches);
-  }
-  lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N);
   int ks2 = 1;
-  if (ce == cudaSuccess) {
-    const int row_tiles = (K + decode_rows_per_cta() - 1) / decode_rows_per_cta();
-    const int want = 2 * 148;
-    ks2 = std::max(1, want / std::max(1, row_tiles * grid_y));
-    ks2 = std::min(ks2, std::min(L->ks2_max, N / kChunkK));
-    if (rows > 1024) ks2 = 1;
-    GemmArgs ga{};
-    ga.experts = dexp;
-    ga.block = 1;
-    ga.active = ra.active;
-    ga.n_active = ra.n_active;
-    ga.counts = ra.counts;
-    ga.poffsets = ra.poffsets;
-    ga.act = static_cast<const uint4*>(L->zact.p);
-    ga.Kpad_in = L->Kpad_z;
-    ga.K = N;
-    ga.M = K;
-    ga.mode = MODE_OUT;
-    ga.out = static_cast<float*>(L->obuf.p);
-    ga.out_ks_stride = prows * K;
-    ga.KS = ks2;
-    ga.status = ra.status;
-    prof_mark(L, st, "decode_gemm_w2");
-    ce = launch_decode_gemm(ga, nt_max, maxbits[1], grid_y, st, &launches);
+  if (prefill) {
+    // tcgen05 path: one launch per block, CTAs over (row tile, 256-token pair, expert)
+    const int pairs = (T + 255) / 256;
+    auto prefill_gemm = [&](int block, const CUtensorMap& map, int Kin, int M, int mode) {
+      if (ce != cudaSuccess) return;
+      PrefillArgs pa;
+      std::memset(&pa, 0, sizeof(pa));
+      pa.tmap_act = map;
+      pa.experts = dexp;
+      pa.block = block;
+      pa.active = ra.active;
+      pa.n_active = ra.n_active;
+      pa.counts = ra.counts;
+      pa.poffsets = ra.poffsets;
+      pa.K = Kin;
+      pa.M = M;
+      pa.mode = mode;
+      pa.zout = static_cast<__half*>(L->zact.p);
+      pa.ldz = L->Kpad_z;
+      pa.out = static_cast<float*>(L->obuf.p);
+      pa.status = ra.status;
+      prof_mark(L, st, block == 0 ? "prefill_gemm_w1_swiglu" : "prefill_gemm_w2");
+      ce = launch_prefill_gemm(pa, pairs, grid_y, st, &launches);
+    };
+    prefill_gemm(0, L->tmap_x, K, 2 * N, MODE_SWIGLU);
+    lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N);
+    prefill_gemm(1, L->tmap_z, N, K, MODE_OUT);
+  } else {
+    // token tiles per pass: cover the expected per-expert batch (mean + 3 sd);
+    // larger batches take more passes
+    const double avg = (double)rows / E;
+    int nt_max = (int)std::ceil((avg + 3.0 * std::sqrt(avg) + 1.0) / 8.0);
+    nt_max = std::max(1, std::min(nt_max, std::min(4, (T + 7) / 8)));
+    if (ce == cudaSuccess) {
+      GemmArgs ga{};
+      ga.experts = dexp;
+      ga.block = 0;
+      ga.active = ra.active;
+      ga.n_active = ra.n_active;
+      ga.counts = ra.counts;
+      ga.poffsets = ra.poffsets;
+      ga.act = static_cast<const uint4*>(L->xact.p);
+      ga.nt8cap = L->nt8cap;
+      ga.K = K;
+      ga.M = 2 * N;
+      ga.mode = MODE_SWIGLU;
+      ga.zout = static_cast<__half*>(L->zact.p);
+      ga.KS = 1;
+      ga.status = ra.status;
+      prof_mark(L, st, "decode_gemm_w1_swiglu");
+      ce = launch_decode_gemm(ga, nt_max, maxbits[0], grid_y, st, &launches);
+    }
+    lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N);
+    if (ce == cudaSuccess) {
+      const int row_tiles = (K + decode_rows_per_cta() - 1) / decode_rows_per_cta();
+      const int want = 2 * 148;
+      ks2 = std::max(1, want / std::max(1, row_tiles * grid_y));
+      ks2 = std::min(ks2, std::min(L->ks2_max, N / kChunkK));
+      if (rows > 1024) ks2 = 1;
+      GemmArgs ga{};
+      ga.experts = dexp;
+      ga.block = 1;
+      ga.active = ra.active;
+      ga.n_active = ra.n_active;
+      ga.counts = ra.counts;
+      ga.poffsets = ra.poffsets;
+      ga.act = static_cast<const uint4*>(L->zact.p);
+      ga.nt8cap = L->nt8cap;
+      ga.K = N;
+      ga.M = K;
+      ga.mode = MODE_OUT;
+      ga.out = static_cast<float*>(L->obuf.p);
+      ga.out_ks_stride = prows * K;
+      ga.KS = ks2;
+      ga.status = ra.status;
+      prof_mark(L, st, "decode_gemm_w2");
+      ce = launch_decode_gemm(ga, nt_max, maxbits[1], grid_y, st, &launches);
+    }
   }
   if (ce == cudaSuccess) {
     CombineArgs ca{};

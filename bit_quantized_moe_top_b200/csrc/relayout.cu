@@ -46,7 +46,7 @@ __global__ void relayout_int_kernel(const uint8_t* __restrict__ canon, uint8_t* 
           }
         }
       }
-  uint32_t* chunk = reinterpret_cast<uint32_t*>(out + ch * 256LL * bits);
+  uint32_t* chunk = reinterpret_cast<uint32_t*>(out + ((long long)kc * MF + rf) * 256LL * bits);
   if (bits == 4) {
     for (int s = 0; s < 8; ++s) chunk[(s >> 2) * 128 + lane * 4 + (s & 3)] = w[s];
   } else {
@@ -71,14 +71,14 @@ __global__ void relayout_sz_kernel(const __half* __restrict__ s, const __half* _
     const int crow = canon_row(16 * rf + g + 8 * hrow, block, N);
     const float sv = __half2float(s[(long long)crow * G + gi]);
     const float zv = __half2float(z[(long long)crow * G + gi]);
-    out[tid * 2 + hrow] = pack_half2(sv, -zv * sv);
+    out[(((long long)gi * MF + rf) * 8 + g) * 2 + hrow] = pack_half2(sv, -zv * sv);
   }
 }
 
 // dense bf16 [rows, K] (row map by block/N, or identity when block < 0) ->
 // fp16 A fragments [MF][K/16][32] uint4
 __global__ void relayout_dense_kernel(const __nv_bfloat16* __restrict__ src, uint4* __restrict__ out, int M, int K,
-                                      int block, int N, long long src_ld) {
+                                      int block, int N, long long src_ld, int chunked) {
   const int S = K / 16, MF = M / 16;
   const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (tid >= (long long)MF * S * 32) return;
@@ -97,7 +97,9 @@ __global__ void relayout_dense_kernel(const __nv_bfloat16* __restrict__ src, uin
     }
     v[j] = pack_half2(e[0], e[1]);
   }
-  out[tid] = make_uint4(v[0], v[1], v[2], v[3]);
+  // chunked: [kc][rf][8 steps][32] (the GEMM weight layout); else [rf][K/16][32]
+  const long long o = chunked ? ((((long long)(st >> 3) * MF + rf) * 8 + (st & 7)) * 32 + lane) : tid;
+  out[o] = make_uint4(v[0], v[1], v[2], v[3]);
 }
 
 // bit-planes [4][M][K/32] u32 -> per plane [MF][KC][32] uint2
@@ -124,8 +126,9 @@ __global__ void relayout_planes_kernel(const uint32_t* __restrict__ canon, uint3
         const uint32_t bit = (word >> (kk & 31)) & 1u;
         w[s >> 2] |= bit << (4 * (2 * j + h) + (s & 3));
       }
-  out[tid * 2 + 0] = w[0];
-  out[tid * 2 + 1] = w[1];
+  const long long o = (((long long)p * KC + kc) * MF + rf) * 32 + lane;
+  out[o * 2 + 0] = w[0];
+  out[o * 2 + 1] = w[1];
 }
 
 // ---------------------------------------------------------------------------
@@ -143,7 +146,7 @@ __global__ void debug_unpack_kernel(BlockDesc d, uint8_t* __restrict__ out, int 
   const int kc = (int)(ch % KC), rf = (int)(ch / KC);
   uint32_t w[8];
   if (d.fmt == FMT_INT) {
-    const uint32_t* chunk = reinterpret_cast<const uint32_t*>(d.codes + ch * 256LL * d.bits);
+    const uint32_t* chunk = reinterpret_cast<const uint32_t*>(d.codes + ((long long)kc * MF + rf) * 256LL * d.bits);
     if (d.bits == 4) {
       for (int s = 0; s < 8; ++s) w[s] = chunk[(s >> 2) * 128 + lane * 4 + (s & 3)];
     } else {
@@ -156,8 +159,9 @@ __global__ void debug_unpack_kernel(BlockDesc d, uint8_t* __restrict__ out, int 
   } else {
     for (int p = 0; p < d.bits; ++p) {
       const uint32_t* pl = reinterpret_cast<const uint32_t*>(d.codes + p * d.plane_stride);
-      w[2 * p] = pl[tid * 2];
-      w[2 * p + 1] = pl[tid * 2 + 1];
+      const long long o = ((long long)kc * MF + rf) * 32 + lane;
+      w[2 * p] = pl[o * 2];
+      w[2 * p + 1] = pl[o * 2 + 1];
     }
   }
   for (int s = 0; s < 8; ++s) {
@@ -199,9 +203,9 @@ cudaError_t launch_relayout_sz(const __half* s, const __half* z, uint32_t* out, 
   return cudaGetLastError();
 }
 cudaError_t launch_relayout_dense(const __nv_bfloat16* src, uint4* out, int M, int K, int block, int N,
-                                  long long ld, cudaStream_t st) {
+                                  long long ld, int chunked, cudaStream_t st) {
   const long long n = (long long)(M / 16) * (K / 16) * 32;
-  relayout_dense_kernel<<<grid_for(n, 256), 256, 0, st>>>(src, out, M, K, block, N, ld);
+  relayout_dense_kernel<<<grid_for(n, 256), 256, 0, st>>>(src, out, M, K, block, N, ld, chunked);
   return cudaGetLastError();
 }
 cudaError_t launch_relayout_planes(const uint32_t* canon, uint32_t* out, int M, int K, int block, int N,

@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_permute_kernel(RouteArgs 
         const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(x + 32 * kb + 2 * c + 8 * q);
         v[q] = pack_half2(__bfloat162float(b2.x), __bfloat162float(b2.y));
       }
-      uint4* dst = reinterpret_cast<uint4*>(a.act) + ((prow >> 3) * (a.Kpad >> 5) + kb) * 32 + (prow & 7) * 4 + c;
+      uint4* dst = reinterpret_cast<uint4*>(a.act) + act_frag_u4(prow >> 3, kb, a.nt8cap, (int)(prow & 7) * 4 + c);
       *dst = make_uint4(v[0], v[1], v[2], v[3]);
     }
   } else {
