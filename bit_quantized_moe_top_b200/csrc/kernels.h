@@ -64,10 +64,12 @@ struct LowrankArgs {
   int Kpad;                   // ACT_ROW: row width
   long long nt8cap;           // ACT_FRAG: row-tile capacity
   int K;
-  int KS;
+  int KS;                     // K splits
+  int tiles;                  // token tiles of 64 rows per expert covered by the grid
   float* part;                // [KS][prows][64]
   long long part_ks_stride;
-  int* sem;                   // [E], zero between launches
+  int* sem;                   // [E][sem_stride], zero between launches
+  long long sem_stride;
   int act_layout;
   unsigned* status;
 };

@@ -1,12 +1,10 @@
 // Low-rank compensator down-projection and the weighted combine.
 //
 // lowrank_kernel: U = V A^T for every expert's routed rows (V = the block's
-// input activations, A = the compensator's [r, K] factor), split over K across
-// CTAs; each CTA writes an fp32 partial and the last CTA of an expert (atomic
-// ticket) sums the partials in a fixed order and stores U as fp16 into the
-// activation columns [K, K + r) that the expert GEMM reads as extra K
-// (MiLo abstract: per-expert low-rank compensators of the quantisation
-// residual).
+// input activations, A = the compensator's [r, K] factor), stored as fp16
+// into the activation columns [K, K + r) that the expert GEMM reads as extra
+// K (MiLo abstract: per-expert low-rank compensators of the quantisation
+// residual). Small batches split K across CTAs (fixed-order sum of partials).
 //
 // combine_kernel: y_t = sum_j w[t, j] * o_(t, j), slots in a fixed order, the
 // K-split partials of o summed first; bf16 out.
@@ -14,106 +12,115 @@
 
 namespace moeq {
 
-constexpr int kLrWarps = 8;
-constexpr int kLrNT = 4;  // n8 token tiles per pass
+constexpr int kLrWarps = 4;    // each warp: 16 routed rows (tokens) x all r columns
+constexpr int kLrRows = 16 * kLrWarps;
 
-__global__ void __launch_bounds__(256) lowrank_kernel(LowrankArgs a) {
-  __shared__ float red[4 * kLrNT * 32 * 4];
+// grid: (KS x token tiles of 64 rows, expert slots). Tokens are the MMA's M:
+// a warp's A fragments are 16 routed rows of the activations, its B
+// fragments come straight from the factor's dense fragments (two n8 tiles per
+// uint4). With KS == 1 the result is written directly; otherwise each CTA
+// writes an fp32 partial and the last CTA of a (expert, token tile) sums the
+// partials in a fixed order.
+__global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
   __shared__ int is_last;
   const int slot = blockIdx.y;
   if (slot >= *a.n_active) return;
   const int e = a.active[slot];
   const int n_e = a.counts[e];
+  const int ks = blockIdx.x % a.KS, tile = blockIdx.x / a.KS;
+  if (tile * kLrRows >= n_e) return;
   const BlockDesc& dd = a.experts[e].blk[a.block];
   const int r = dd.rank;
-  if (r <= 0 || n_e <= 0) return;
+  if (r <= 0) return;
   const uint4* afrag = dd.afrag;
   const int RF = r / 16;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, c = lane & 3;
-  const int ks = blockIdx.x;
   const int S16 = a.K / 16;
   const int s0 = (int)((long long)S16 * ks / a.KS), s1 = (int)((long long)S16 * (ks + 1) / a.KS);
   const int prow0 = a.poffsets[e];
-  const int ntiles = (n_e + 7) >> 3;
+  const int rbase = tile * kLrRows + warp * 16;  // first row (within the expert) of this warp
   const uint4* act4 = reinterpret_cast<const uint4*>(a.act);
-  for (int pb = 0; pb < ntiles; pb += kLrNT) {
-    const int np = min(kLrNT, ntiles - pb);
-    float acc[4][kLrNT][4];
+  const uint32_t* act32 = reinterpret_cast<const uint32_t*>(a.act);
+  float acc[8][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+  for (int t = 0; t < 8; ++t)
 #pragma unroll
-      for (int t = 0; t < kLrNT; ++t)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[i][t][q] = 0.f;
-    for (int S = s0 + warp; S < s1; S += kLrWarps) {
-      uint32_t b0[kLrNT], b1[kLrNT];
-#pragma unroll
-      for (int t = 0; t < kLrNT; ++t) {
-        b0[t] = b1[t] = 0;
-        if (t < np) {
-          const long long n0 = prow0 + 8LL * (pb + t);
-          if (a.act_layout == ACT_FRAG) {
-            const uint4 v = act4[act_frag_u4(n0 >> 3, S >> 1, a.nt8cap, lane)];
-            b0[t] = (S & 1) ? v.z : v.x;
-            b1[t] = (S & 1) ? v.w : v.y;
-          } else {
-            const uint32_t* row = reinterpret_cast<const uint32_t*>(a.act + (n0 + g) * a.Kpad + 16 * S);
-            b0[t] = row[c];
-            b1[t] = row[c + 4];
-          }
-        }
+    for (int q = 0; q < 4; ++q) acc[t][q] = 0.f;
+  if (rbase < n_e) {
+    const long long ra = prow0 + rbase + g, rb = ra + 8;  // rows of a0a1/a4a5 and a2a3/a6a7
+#pragma unroll 4
+    for (int S = s0; S < s1; ++S) {
+      uint32_t av[4];
+      if (a.act_layout == ACT_FRAG) {
+        // rows rbase.. are 8-aligned inside the expert's padded range: two row tiles
+        const uint4 v0 = act4[act_frag_u4((prow0 + rbase) >> 3, S >> 1, a.nt8cap, lane)];
+        const uint4 v1 = act4[act_frag_u4(((prow0 + rbase) >> 3) + 1, S >> 1, a.nt8cap, lane)];
+        av[0] = (S & 1) ? v0.z : v0.x;
+        av[1] = (S & 1) ? v1.z : v1.x;
+        av[2] = (S & 1) ? v0.w : v0.y;
+        av[3] = (S & 1) ? v1.w : v1.y;
+      } else {
+        const long long ldw = a.Kpad >> 1;  // row pitch in u32
+        av[0] = act32[ra * ldw + 8 * S + c];
+        av[1] = act32[rb * ldw + 8 * S + c];
+        av[2] = act32[ra * ldw + 8 * S + c + 4];
+        av[3] = act32[rb * ldw + 8 * S + c + 4];
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        if (i >= RF) break;
-        const uint4 v = afrag[((long long)i * S16 + S) * 32 + lane];
-        const uint32_t av[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int t = 0; t < kLrNT; ++t)
-          if (t < np) mma_16816(acc[i][t], av, b0[t], b1[t]);
+        if (i < RF) {
+          const uint4 v = afrag[((long long)i * S16 + S) * 32 + lane];
+          mma_16816(acc[2 * i], av, v.x, v.z);
+          mma_16816(acc[2 * i + 1], av, v.y, v.w);
+        }
       }
     }
-    // fixed-order reduction over warps
-    for (int i = threadIdx.x; i < 4 * kLrNT * 32 * 4; i += blockDim.x) red[i] = 0.f;
-    __syncthreads();
-    for (int w = 0; w < kLrWarps; ++w) {
-      if (warp == w) {
+  }
+  // acc[t][q]: row rbase + g + 8*(q>>1), column j = 8t + 2c + (q&1)
+  auto store_u = [&](int n, int j, float v) {
+    const __half hv = __float2half_rn(v);
+    if (a.act_layout == ACT_FRAG) a.act[act_frag_index(prow0 + n, a.K + j, a.nt8cap)] = hv;
+    else a.act[(long long)(prow0 + n) * a.Kpad + a.K + j] = hv;
+  };
+  if (a.KS == 1) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+    for (int t = 0; t < 8; ++t) {
+      if (t >= 2 * RF) break;
 #pragma unroll
-          for (int t = 0; t < kLrNT; ++t)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) red[((i * kLrNT + t) * 32 + lane) * 4 + q] += acc[i][t][q];
+      for (int q = 0; q < 4; ++q) {
+        const int n = rbase + g + 8 * (q >> 1);
+        if (n < n_e) store_u(n, 8 * t + 2 * c + (q & 1), acc[t][q]);
       }
-      __syncthreads();
     }
-    // CTA partial -> part[ks][prow][j]
-    for (int idx = threadIdx.x; idx < RF * kLrNT * 32 * 4; idx += blockDim.x) {
-      const int q = idx & 3, ln = (idx >> 2) & 31, t = (idx >> 7) % kLrNT, i = (idx >> 7) / kLrNT;
-      if (t >= np) continue;
-      const int n = 8 * (pb + t) + 2 * (ln & 3) + (q & 1);
-      if (n >= n_e) continue;
-      const int j = 16 * i + (ln >> 2) + 8 * (q >> 1);
-      a.part[ks * a.part_ks_stride + (long long)(prow0 + n) * kMaxRank + j] = red[idx];
+    return;
+  }
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    if (t >= 2 * RF) break;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int n = rbase + g + 8 * (q >> 1);
+      if (n < n_e)
+        a.part[ks * a.part_ks_stride + (long long)(prow0 + n) * kMaxRank + 8 * t + 2 * c + (q & 1)] = acc[t][q];
     }
-    __syncthreads();
   }
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) is_last = (atomicAdd(a.sem + e, 1) == a.KS - 1);
+  int* sem = a.sem + (long long)e * a.sem_stride + tile;
+  if (threadIdx.x == 0) is_last = (atomicAdd(sem, 1) == a.KS - 1);
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  for (int idx = threadIdx.x; idx < n_e * r; idx += blockDim.x) {
-    const int n = idx / r, j = idx % r;
-    float s = 0.f;
-    for (int k2 = 0; k2 < a.KS; ++k2) s += __ldcg(a.part + k2 * a.part_ks_stride + (long long)(prow0 + n) * kMaxRank + j);
-    const __half hv = __float2half_rn(s);
-    if (a.act_layout == ACT_FRAG) a.act[act_frag_index(prow0 + n, a.K + j, a.nt8cap)] = hv;
-    else a.act[(long long)(prow0 + n) * a.Kpad + a.K + j] = hv;
+  const int nrows = min(kLrRows, n_e - tile * kLrRows);
+  for (int idx = threadIdx.x; idx < nrows * r; idx += blockDim.x) {
+    const int n = tile * kLrRows + idx / r, j = idx % r;
+    float sum = 0.f;
+    for (int k2 = 0; k2 < a.KS; ++k2)
+      sum += __ldcg(a.part + k2 * a.part_ks_stride + (long long)(prow0 + n) * kMaxRank + j);
+    store_u(n, j, sum);
   }
-  if (threadIdx.x == 0) a.sem[e] = 0;
+  if (threadIdx.x == 0) *sem = 0;
 }
 
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
@@ -144,7 +151,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
 }
 
 cudaError_t launch_lowrank(const LowrankArgs& a, int grid_y, cudaStream_t st, int* launches) {
-  dim3 grid(a.KS, grid_y);
+  dim3 grid(a.KS * a.tiles, grid_y);
   lowrank_kernel<<<grid, kLrWarps * 32, 0, st>>>(a);
   if (launches) ++*launches;
   return cudaGetLastError();

@@ -64,6 +64,7 @@ struct moe_layer {
   int rmax_pad = 0, Kpad_x = 0, Kpad_z = 0;
   long long rows_pad_max = 0, nt8cap = 0;
   int nb_max = 0, ks2_max = 1, kslr_max = 1;
+  long long sem_stride = 0;
   DevBuf idx, w, counts, offsets, poffsets, active, n_active, ticket, perm, inv_pos, pinv;
   DevBuf block_counts, block_base, pblock_base, sem, status;
   DevBuf xact, zact, obuf, part;
@@ -217,7 +218,9 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   L->Kpad_x = K + L->rmax_pad;
   L->Kpad_z = N + L->rmax_pad;
   const long long rows = (long long)max_tokens * max_top_k;
-  L->rows_pad_max = (rows + 7LL * E + 7) / 8 * 8;
+  // padded rows of all experts, plus 16 rows of slack: 16-row fragments that
+  // start inside the last expert may read (and never store) past its end
+  L->rows_pad_max = (rows + 7LL * E + 7) / 8 * 8 + 16;
   L->nt8cap = L->rows_pad_max / 8;
   L->nb_max = route_num_blocks(max_tokens);
   L->ks2_max = 16;
@@ -244,7 +247,8 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   A(L->block_counts, sizeof(int) * (size_t)L->nb_max * E);
   A(L->block_base, sizeof(int) * (size_t)L->nb_max * E);
   A(L->pblock_base, sizeof(int) * (size_t)L->nb_max * E);
-  A(L->sem, sizeof(int) * E);
+  L->sem_stride = (max_tokens + 63) / 64 + 1;
+  A(L->sem, sizeof(int) * E * L->sem_stride);
   A(L->status, sizeof(unsigned));
   const size_t kx = (size_t)(L->Kpad_x + 127) / 128 * 128, kz = (size_t)(L->Kpad_z + 127) / 128 * 128;
   A(L->xact, sizeof(__half) * (size_t)L->rows_pad_max * kx);
@@ -525,9 +529,13 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     la.Kpad = Kpad;
     la.nt8cap = L->nt8cap;
     la.K = Kin;
-    int ks = 296 / grid_y;
-    ks = std::max(1, std::min(ks, std::min(L->kslr_max, Kin / 16 / 8)));
+    // token tiles of 64 rows per expert; split K only while the grid is small
+    la.tiles = (int)std::min<long long>((T + 63) / 64, (rows + 63) / 64);
+    const long long ctas = (rows + 63) / 64 + grid_y / 2;
+    int ks = (int)std::max<long long>(1, 296 / std::max<long long>(1, ctas));
+    ks = std::max(1, std::min(ks, std::min(L->kslr_max, Kin / 256)));
     la.KS = ks;
+    la.sem_stride = L->sem_stride;
     la.part = static_cast<float*>(L->part.p);
     la.part_ks_stride = (long long)L->rows_pad_max * kMaxRank;
     la.sem = static_cast<int*>(L->sem.p);
