@@ -189,6 +189,24 @@ def cpu_oracle_rate(cfg, blocks_cpu, X, logits, top_k, budget_s):
     return done / dt, done, dt, threads
 
 
+def max_over_ranks(total_ms, world, device):
+    """The job's time: the slowest rank's device-timed total (all ranks take
+    part in the same collective; a barrier follows)."""
+    if world <= 1:
+        return total_ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(total_ms)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.barrier()
+    return float(t.item())
+
+
+def weak_scaling_value(world, tokens_per_rank, ms_per_step):
+    """Tokens/s of the whole job: every rank runs its own batch of T tokens."""
+    return world * tokens_per_rank / (ms_per_step / 1000.0)
+
+
 def build_layer(bq, cfg, blocks, max_tokens):
     import ctypes
     descs = [bq.ExpertDesc((ctypes.c_int * 2)(*sp.bits), sp.fmt, sp.group, sp.rank) for sp in cfg.experts[:cfg.E]]
@@ -289,14 +307,9 @@ def main():
         torch.cuda.synchronize()
     L.set_profiling(False)
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-        dist.barrier()
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * T / (ms_per_step / 1000.0)
+    value = weak_scaling_value(world, T, ms_per_step)
 
     # dominant kernel: the gate/up GEMM (2/3 of the weight bytes and flops)
     hbm_peak, tc_peak, tc_sustained, peak_src = measured_peaks()

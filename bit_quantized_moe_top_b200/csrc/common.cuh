@@ -3,20 +3,19 @@
 //
 // Internal layouts (all built on the device at weight-load time):
 //
-//  * Rows of W1 (gate||up, 2N x K) are interleaved per 16-row fragment:
-//    internal row 16f+i is gate row 8f+i for i < 8 and up row 8f+i-8 for
-//    i >= 8, so one mma.sync accumulator fragment (rows g and g+8) holds the
-//    gate and the up value of the same SwiGLU column.
-//  * Codes are stored per (row fragment rf, 128-wide K chunk kc) in the order a
-//    warp's lanes consume them as mma.m16n8k16 A fragments: lane (g = lane/4,
-//    c = lane%4), step s (0..7, a k16 slice of the chunk), slot j (0..3 = the
-//    A registers a0a1, a2a3, a4a5, a6a7), half h (0/1) is the element
-//    (row 16rf + g + 8*(j&1), k = 128kc + 16s + 2c + 8*(j>>1) + h).
-//    A chunk holds 256*b bytes (b = bits; 16 for dense fp16).
-//  * Chunks are stored chunk-major: [kc][rf] (bit-planes: [plane][kc][rf]), so
-//    the 16 row fragments a CTA streams for one chunk are one contiguous range.
-//  * Activations for the mma.sync path are stored per (128-wide k chunk, 8-row
-//    tile) as 4 k32 blocks x 32 lanes x uint4 = B fragments of 8 k16 steps.
+//  * Rows of W1 (gate||up, 2N x K) are interleaved per 16-row group: internal
+//    row 16f+i is gate row 8f+i for i < 8 and up row 8f+i-8 for i >= 8, so the
+//    gate and up values of one SwiGLU column sit 8 rows (8 TMEM lanes) apart.
+//  * Codes are stored per 64-wide K chunk kc and 128-row block rb, chunk-major
+//    ([kc][rb]), so the rows a CTA streams for one chunk are one contiguous
+//    range. Inside a block, row i's 64 codes are "words" in the order one
+//    thread consumes them: step s (0..7) holds pairs j (0..3) of codes
+//    (k = 8s + 2j, 8s + 2j + 1). Words are stored word-quad-major
+//    ([quad][row][16 B]) so that a thread per row reads them conflict-free.
+//    A block holds 128 * 8 * b bytes (b = bits; 16 for dense fp16).
+//  * Activations are row-major fp16 [rows, Kpad]: routed rows bucketed per
+//    expert, each expert's range padded to a multiple of 8 rows; the rank
+//    columns U = A x sit after column K.
 #pragma once
 #include <cstdint>
 #include <cuda_fp16.h>
@@ -36,12 +35,12 @@ enum : unsigned { ST_BOUNDS = 1u, ST_TIMEOUT = 2u, ST_ROUTE = 4u };
 
 // One expert linear block as the kernels see it.
 struct BlockDesc {
-  const uint8_t* codes;   // chunked codes [kc][rf][256*b bytes] (INT / DENSE) or plane 0 (BITPLANE)
-  const uint32_t* sz;     // INT: [K/g][MF][8] uint2 = half2(s, -z*s) for rows g and g+8
+  const uint8_t* codes;   // code blocks [K/64][M/128][block] (INT / DENSE) or plane 0 (BITPLANE)
+  const uint32_t* sz;     // INT: [K/g][M] half2(s, -z*s), internal row order
   const uint32_t* lut;    // BITPLANE: 28 fp16 as 14 u32
-  const uint4* bfrag;     // compensator B [M, r] as dense A-fragments [MF][r/16][32] uint4 (fp16)
-  const uint4* afrag;     // compensator A [r, K] as dense A-fragments [r/16][K/16][32] uint4 (fp16)
-  long long plane_stride; // BITPLANE: bytes between planes ([kc][rf][256] each)
+  const uint32_t* brow;   // compensator B as fp16 pairs [r/2][M] (column-pair-major)
+  const uint4* afrag;     // compensator A [r, K] as mma A-fragments [r/16][K/16][32] uint4 (fp16)
+  long long plane_stride; // BITPLANE: bytes between planes ([K/64][M/128][1 KiB] each)
   int fmt, bits, group, rank;
   int M, K;
   int loaded;
@@ -132,34 +131,10 @@ __host__ __device__ __forceinline__ int canon_row(int ir, int block, int N) {
   return i < 8 ? 8 * f + i : N + 8 * f + (i - 8);
 }
 
-// (row-in-fragment, k-in-chunk) of element (lane, step, slot, half)
-__host__ __device__ __forceinline__ void frag_elem(int lane, int s, int j, int h, int& r, int& k) {
-  int g = lane >> 2, c = lane & 3;
-  r = g + 8 * (j & 1);
-  k = 16 * s + 2 * c + 8 * (j >> 1) + h;
-}
-
-// Activation B-fragment layout, chunk-major: for each 128-wide k chunk kc,
-// the 8-row tiles nt of the whole buffer (capacity nt8cap tiles) follow each
-// other, each holding 4 k32 blocks x 32 lanes x uint4 (2 KiB). An expert's
-// consecutive row tiles of one chunk are therefore one contiguous range.
-// Returns the fp16 index of element (row n, col k).
-__host__ __device__ __forceinline__ long long act_frag_index(long long n, int k, long long nt8cap) {
-  const long long nt = n >> 3;
-  const int g = (int)(n & 7);
-  const int kc = k >> 7, kin = k & 127;
-  const int kk = kin >> 5, k32 = kin & 31;
-  const int step = k32 >> 4, k16 = k32 & 15;
-  const int hi = k16 >> 3, c = (k16 & 7) >> 1, h = k16 & 1;
-  const int lane = g * 4 + c;
-  const int comp = step * 2 + hi;
-  return ((((long long)kc * nt8cap + nt) * 4 + kk) * 32 + lane) * 8 + comp * 2 + h;
-}
-// uint4 index of the B fragments of k16 steps (2*kk2, 2*kk2+1) of row tile nt
-// (kk2 = k / 32 over the whole row)
-__host__ __device__ __forceinline__ long long act_frag_u4(long long nt, int kk2, long long nt8cap, int lane) {
-  return ((((long long)(kk2 >> 2) * nt8cap + nt) * 4 + (kk2 & 3)) * 32 + lane);
-}
+// words per row of one 64-wide chunk (INT: 2*b; dense fp16: 32)
+__host__ __device__ __forceinline__ int words_per_row(int fmt, int bits) { return fmt == FMT_DENSE ? 32 : 2 * bits; }
+// bytes of one [128-row x 64-k] code block
+__host__ __device__ __forceinline__ int block_bytes(int fmt, int bits) { return 128 * 4 * words_per_row(fmt, bits); }
 
 // ---------------------------------------------------------------------------
 // mbarrier / bulk-copy helpers (TMA engine, no multicast)

@@ -1,5 +1,6 @@
-// Register-level unpack + dequantisation of one k16 step of a lane's codes
-// into the four fp16x2 A-fragment registers of mma.m16n8k16.
+// Register-level unpack + dequantisation of packed codes into fp16 pairs.
+// One thread owns one weight row; a 64-wide K chunk of that row is 8 "steps"
+// of 4 pairs, pair j of step s being the codes at k = 8s+2j and 8s+2j+1.
 //
 // Integer codes become fp16 through the exponent-bias trick: a b-bit field
 // OR-ed into the mantissa of a power of two P whose mantissa ulp is 1 reads as
@@ -51,7 +52,7 @@ __device__ __forceinline__ void int3_codes(uint32_t lo, uint32_t hi, int s, uint
   q[3] = hsub2u(lop3_and_or(lop3_sel(b, t, 0x00C000C0u), 0x01C001C0u, 0x4C004C00u), 0x4C004C00u);
 }
 
-// codes of step s for a lane, from the lane's chunk words (already in registers)
+// codes of step s (4 fp16x2 pairs) from the row's chunk words (in registers)
 //   INT2: w[0..3]   INT3: w[0..3] lo + w[4..5] hi   INT4: w[0..7]
 template <int BITS>
 __device__ __forceinline__ void int_codes(const uint32_t* w, int s, uint32_t (&q)[4]) {
@@ -134,6 +135,57 @@ __device__ __forceinline__ void lut_decode(uint32_t codes, const LutRegs& L, uin
     }
     a[2 * half + 0] = prmt(lo, hi, 0x5140u);
     a[2 * half + 1] = prmt(lo, hi, 0x7362u);
+  }
+}
+
+// ---- whole 64-wide chunk of one row ----
+
+// words of row `row` of a [128-row] code block (global or shared memory)
+__device__ __forceinline__ void load_row_words_int(const uint8_t* blk, int row, int bits, uint32_t (&w)[8]) {
+  const uint4 v0 = reinterpret_cast<const uint4*>(blk)[row];
+  w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+  w[4] = w[5] = w[6] = w[7] = 0u;
+  if (bits == 4) {
+    const uint4 v1 = reinterpret_cast<const uint4*>(blk + 2048)[row];
+    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+  } else if (bits == 3) {
+    const uint2 h = reinterpret_cast<const uint2*>(blk + 2048)[row];
+    w[4] = h.x; w[5] = h.y;
+  }
+}
+
+// bit-plane words of row `row`: plane p at blk + p * plane_bytes
+template <int BITS>
+__device__ __forceinline__ void load_row_planes(const uint8_t* blk, int plane_bytes, int row, uint32_t (&w)[8]) {
+#pragma unroll
+  for (int p = 0; p < BITS; ++p) {
+    const uint2 v = reinterpret_cast<const uint2*>(blk + p * plane_bytes)[row];
+    w[2 * p] = v.x; w[2 * p + 1] = v.y;
+  }
+}
+
+// 32 fp16 pairs (k = 0..63) of one row chunk: out[4s+j] = pair (8s+2j, 8s+2j+1)
+// INT: w^ = (q - z) * s with sz = half2(s, -z*s); bit-plane: LUT_b[code].
+template <int FMT, int BITS>
+__device__ __forceinline__ void decode_row64(const uint32_t (&w)[8], uint32_t sz, const LutRegs& lut,
+                                             uint32_t (&out)[32]) {
+  if constexpr (FMT == FMT_INT) {
+    const uint32_t s2 = prmt(sz, sz, 0x1010u), n2 = prmt(sz, sz, 0x3232u);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      uint32_t q[4];
+      int_codes<BITS>(w, s, q);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[4 * s + j] = hfma2u(q[j], s2, n2);
+    }
+  } else {
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      uint32_t av[4];
+      lut_decode<BITS>(plane_codes<BITS>(w, s), lut, av);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[4 * s + j] = av[j];
+    }
   }
 }
 

@@ -6,7 +6,6 @@
 
 namespace moeq {
 
-enum : int { ACT_FRAG = 0, ACT_ROW = 1 };
 enum : int { MODE_SWIGLU = 0, MODE_OUT = 1 };
 
 struct RouteArgs {
@@ -27,26 +26,24 @@ struct RouteArgs {
   int* perm_token;            // [T*k]
   int* inv_pos;               // [T, k]
   int* pinv;                  // [T, k] padded row
-  void* act;                  // activation buffer (fp16), layout act_layout
-  int Kpad;                   // ACT_ROW: row width (elements)
-  long long nt8cap;           // ACT_FRAG: row-tile capacity of the buffer
-  int act_layout;
+  void* act;                  // activation buffer, fp16 row-major [rows, Kpad]
+  int Kpad;
   unsigned* status;
 };
 
-struct GemmArgs {
+struct DecodeArgs {
+  CUtensorMap tmap_act;       // activations [rows, Kpad] fp16 row-major; box 64 x 16, 128-byte swizzle
   const ExpertDesc* experts;
   int block;                  // 0 = W1, 1 = W2
   const int* active;
   const int* n_active;
   const int* counts;
   const int* poffsets;
-  const uint4* act;           // input activations (fragment layout)
-  long long nt8cap;           // row-tile capacity of the activation buffers
   int K;                      // quantised K of the block
   int M;                      // rows of the block
   int mode;
-  __half* zout;               // MODE_SWIGLU: output activations (fragment layout)
+  __half* zout;               // MODE_SWIGLU: output rows (fp16), leading dimension ldz
+  long long ldz;
   float* out;                 // MODE_OUT: [KS][prows][M] fp32 partials
   long long out_ks_stride;
   int KS;
@@ -60,9 +57,8 @@ struct LowrankArgs {
   const int* n_active;
   const int* counts;
   const int* poffsets;
-  __half* act;                // activation buffer; reads [0,K), writes ext columns [K, K+r)
-  int Kpad;                   // ACT_ROW: row width
-  long long nt8cap;           // ACT_FRAG: row-tile capacity
+  __half* act;                // activation buffer, fp16 row-major; reads [0,K), writes columns [K, K+r)
+  int Kpad;
   int K;
   int KS;                     // K splits
   int tiles;                  // token tiles of 64 rows per expert covered by the grid
@@ -70,7 +66,6 @@ struct LowrankArgs {
   long long part_ks_stride;
   int* sem;                   // [E][sem_stride], zero between launches
   long long sem_stride;
-  int act_layout;
   unsigned* status;
 };
 
@@ -105,8 +100,11 @@ cudaError_t launch_relayout_int(const uint8_t* canon, uint8_t* out, int M, int K
                                 cudaStream_t st);
 cudaError_t launch_relayout_sz(const __half* s, const __half* z, uint32_t* out, int M, int K, int group, int block,
                                int N, cudaStream_t st);
-cudaError_t launch_relayout_dense(const __nv_bfloat16* src, uint4* out, int M, int K, int block, int N, long long ld,
-                                  int chunked, cudaStream_t st);
+cudaError_t launch_relayout_dense(const __nv_bfloat16* src, uint8_t* out, int M, int K, int block, int N,
+                                  cudaStream_t st);
+cudaError_t launch_relayout_afrag(const __nv_bfloat16* src, uint4* out, int r, int K, cudaStream_t st);
+cudaError_t launch_relayout_brow(const __nv_bfloat16* src, uint32_t* out, int M, int r, int block, int N,
+                                 cudaStream_t st);
 cudaError_t launch_relayout_planes(const uint32_t* canon, uint32_t* out, int M, int K, int block, int N,
                                    cudaStream_t st);
 cudaError_t launch_debug_unpack(const BlockDesc& d, uint8_t* out, int block, int N, cudaStream_t st);
@@ -115,10 +113,8 @@ cudaError_t launch_route_topk(const RouteArgs& a, cudaStream_t st, int* launches
 cudaError_t launch_route_permute(const RouteArgs& a, cudaStream_t st, int* launches);
 int route_num_blocks(int T);
 
-// grid sizing helpers for the decode GEMM
 int decode_rows_per_cta();
-size_t decode_smem_bytes(int nt, int maxbits);
-cudaError_t launch_decode_gemm(const GemmArgs& a, int nt_max, int maxbits, int grid_y, cudaStream_t st,
+cudaError_t launch_decode_gemm(const DecodeArgs& a, int ntok, int maxbits, int grid_y, cudaStream_t st,
                                int* launches);
 cudaError_t launch_lowrank(const LowrankArgs& a, int grid_y, cudaStream_t st, int* launches);
 cudaError_t launch_prefill_gemm(const PrefillArgs& a, int grid_y, int grid_z, cudaStream_t st, int* launches);

@@ -40,7 +40,6 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
   const int s0 = (int)((long long)S16 * ks / a.KS), s1 = (int)((long long)S16 * (ks + 1) / a.KS);
   const int prow0 = a.poffsets[e];
   const int rbase = tile * kLrRows + warp * 16;  // first row (within the expert) of this warp
-  const uint4* act4 = reinterpret_cast<const uint4*>(a.act);
   const uint32_t* act32 = reinterpret_cast<const uint32_t*>(a.act);
   float acc[8][4];
 #pragma unroll
@@ -52,21 +51,11 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
 #pragma unroll 4
     for (int S = s0; S < s1; ++S) {
       uint32_t av[4];
-      if (a.act_layout == ACT_FRAG) {
-        // rows rbase.. are 8-aligned inside the expert's padded range: two row tiles
-        const uint4 v0 = act4[act_frag_u4((prow0 + rbase) >> 3, S >> 1, a.nt8cap, lane)];
-        const uint4 v1 = act4[act_frag_u4(((prow0 + rbase) >> 3) + 1, S >> 1, a.nt8cap, lane)];
-        av[0] = (S & 1) ? v0.z : v0.x;
-        av[1] = (S & 1) ? v1.z : v1.x;
-        av[2] = (S & 1) ? v0.w : v0.y;
-        av[3] = (S & 1) ? v1.w : v1.y;
-      } else {
-        const long long ldw = a.Kpad >> 1;  // row pitch in u32
-        av[0] = act32[ra * ldw + 8 * S + c];
-        av[1] = act32[rb * ldw + 8 * S + c];
-        av[2] = act32[ra * ldw + 8 * S + c + 4];
-        av[3] = act32[rb * ldw + 8 * S + c + 4];
-      }
+      const long long ldw = a.Kpad >> 1;  // row pitch in u32
+      av[0] = act32[ra * ldw + 8 * S + c];
+      av[1] = act32[rb * ldw + 8 * S + c];
+      av[2] = act32[ra * ldw + 8 * S + c + 4];
+      av[3] = act32[rb * ldw + 8 * S + c + 4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         if (i < RF) {
@@ -79,9 +68,7 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
   }
   // acc[t][q]: row rbase + g + 8*(q>>1), column j = 8t + 2c + (q&1)
   auto store_u = [&](int n, int j, float v) {
-    const __half hv = __float2half_rn(v);
-    if (a.act_layout == ACT_FRAG) a.act[act_frag_index(prow0 + n, a.K + j, a.nt8cap)] = hv;
-    else a.act[(long long)(prow0 + n) * a.Kpad + a.K + j] = hv;
+    a.act[(long long)(prow0 + n) * a.Kpad + a.K + j] = __float2half_rn(v);
   };
   if (a.KS == 1) {
 #pragma unroll

@@ -47,7 +47,7 @@ void dfree(DevBuf& b) {
 }
 
 struct BlockStore {
-  DevBuf codes, sz, lut, afrag, bfrag;
+  DevBuf codes, sz, lut, afrag, brow;
 };
 
 }  // namespace
@@ -69,7 +69,8 @@ struct moe_layer {
   DevBuf block_counts, block_base, pblock_base, sem, status;
   DevBuf xact, zact, obuf, part;
   DevBuf hx, hl, hy;  // device buffers for forward_host
-  CUtensorMap tmap_x, tmap_z;  // row-layout activation buffers for the prefill GEMMs
+  CUtensorMap tmap_x, tmap_z;    // activation buffers, 128-row boxes (prefill GEMMs)
+  CUtensorMap tmap_xd, tmap_zd;  // activation buffers, 16-row boxes (decode GEMMs)
   bool have_tmaps = false;
   int last_T = 0, last_k = 0, last_launches = 0;
   cudaStream_t last_stream = nullptr;
@@ -102,8 +103,8 @@ static void prof_end(moe_layer_t* L, cudaStream_t st) {
 static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
 // 2-D tensor map over a row-major fp16 [rows, cols] buffer: box 64 columns x
-// 128 rows, 128-byte swizzle, zero fill outside the buffer.
-static bool encode_act_map(CUtensorMap* map, void* base, int cols, long long rows) {
+// box_rows rows, 128-byte swizzle, zero fill outside the buffer.
+static bool encode_act_map(CUtensorMap* map, void* base, int cols, long long rows, int box_rows) {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     cudaDriverEntryPointQueryResult q;
@@ -115,7 +116,7 @@ static bool encode_act_map(CUtensorMap* map, void* base, int cols, long long row
   }
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -145,7 +146,7 @@ static void free_block(BlockStore& s) {
   dfree(s.sz);
   dfree(s.lut);
   dfree(s.afrag);
-  dfree(s.bfrag);
+  dfree(s.brow);
 }
 
 extern "C" {
@@ -250,9 +251,8 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   L->sem_stride = (max_tokens + 63) / 64 + 1;
   A(L->sem, sizeof(int) * E * L->sem_stride);
   A(L->status, sizeof(unsigned));
-  const size_t kx = (size_t)(L->Kpad_x + 127) / 128 * 128, kz = (size_t)(L->Kpad_z + 127) / 128 * 128;
-  A(L->xact, sizeof(__half) * (size_t)L->rows_pad_max * kx);
-  A(L->zact, sizeof(__half) * (size_t)L->rows_pad_max * kz);
+  A(L->xact, sizeof(__half) * (size_t)L->rows_pad_max * L->Kpad_x);
+  A(L->zact, sizeof(__half) * (size_t)L->rows_pad_max * L->Kpad_z);
   A(L->obuf, sizeof(float) * (size_t)o_elems * K);
   A(L->part, sizeof(float) * (size_t)L->kslr_max * L->rows_pad_max * kMaxRank);
   A(L->hx, sizeof(__nv_bfloat16) * (size_t)max_tokens * K);
@@ -273,8 +273,14 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
     moe_layer_destroy(L);
     return MOE_ERR_CUDA;
   }
-  L->have_tmaps = encode_act_map(&L->tmap_x, L->xact.p, L->Kpad_x, L->rows_pad_max) &&
-                  encode_act_map(&L->tmap_z, L->zact.p, L->Kpad_z, L->rows_pad_max);
+  L->have_tmaps = encode_act_map(&L->tmap_x, L->xact.p, L->Kpad_x, L->rows_pad_max, 128) &&
+                  encode_act_map(&L->tmap_z, L->zact.p, L->Kpad_z, L->rows_pad_max, 128) &&
+                  encode_act_map(&L->tmap_xd, L->xact.p, L->Kpad_x, L->rows_pad_max, 16) &&
+                  encode_act_map(&L->tmap_zd, L->zact.p, L->Kpad_z, L->rows_pad_max, 16);
+  if (!L->have_tmaps) {
+    moe_layer_destroy(L);
+    return MOE_ERR_CUDA;
+  }
   *out = L;
   return MOE_OK;
 }
@@ -311,7 +317,7 @@ moe_status_t moe_layer_set_expert_weights(moe_layer_t* L, int e, int block, cons
   d.loaded = 0;
   moe_status_t st = MOE_OK;
   DevBuf t1, t2, t3, t4, t5;
-  const int MF = M / 16, KC = Kin / kChunkK;
+  const int RB = M / 128, KC = Kin / 64;
   cudaStream_t s0 = 0;
   cudaError_t ce = cudaSuccess;
   const void* dc = nullptr;
@@ -322,8 +328,8 @@ moe_status_t moe_layer_set_expert_weights(moe_layer_t* L, int e, int block, cons
     st = stage_in(t1, codes, nbytes, ptr_kind, &dc);
     if (st == MOE_OK) st = stage_in(t2, scales, nsz, ptr_kind, &ds);
     if (st == MOE_OK) st = stage_in(t3, zeros_or_lut, nsz, ptr_kind, &dz);
-    if (st == MOE_OK) st = dalloc(S.codes, (size_t)MF * KC * 256 * d.bits);
-    if (st == MOE_OK) st = dalloc(S.sz, (size_t)MF * (Kin / d.group) * 16 * sizeof(uint32_t));
+    if (st == MOE_OK) st = dalloc(S.codes, (size_t)KC * RB * block_bytes(FMT_INT, d.bits));
+    if (st == MOE_OK) st = dalloc(S.sz, (size_t)(Kin / d.group) * M * sizeof(uint32_t));
     if (st == MOE_OK) {
       ce = launch_relayout_int(static_cast<const uint8_t*>(dc), static_cast<uint8_t*>(S.codes.p), M, Kin, d.bits,
                                block, L->N, s0);
@@ -336,7 +342,7 @@ moe_status_t moe_layer_set_expert_weights(moe_layer_t* L, int e, int block, cons
     const void* dl = nullptr;
     st = stage_in(t1, codes, nbytes, ptr_kind, &dc);
     if (st == MOE_OK) st = stage_in(t3, zeros_or_lut, 28 * sizeof(__half), ptr_kind, &dl);
-    if (st == MOE_OK) st = dalloc(S.codes, (size_t)4 * MF * KC * 256);
+    if (st == MOE_OK) st = dalloc(S.codes, (size_t)4 * KC * RB * 1024);
     if (st == MOE_OK) st = dalloc(S.lut, 28 * sizeof(__half));
     if (st == MOE_OK) {
       ce = launch_relayout_planes(static_cast<const uint32_t*>(dc), static_cast<uint32_t*>(S.codes.p), M, Kin, block,
@@ -348,8 +354,8 @@ moe_status_t moe_layer_set_expert_weights(moe_layer_t* L, int e, int block, cons
     st = stage_in(t1, codes, nbytes, ptr_kind, &dc);
     if (st == MOE_OK) st = dalloc(S.codes, nbytes);
     if (st == MOE_OK)
-      ce = launch_relayout_dense(static_cast<const __nv_bfloat16*>(dc), static_cast<uint4*>(S.codes.p), M, Kin, block,
-                                 L->N, Kin, 1, s0);
+      ce = launch_relayout_dense(static_cast<const __nv_bfloat16*>(dc), static_cast<uint8_t*>(S.codes.p), M, Kin,
+                                 block, L->N, s0);
   }
   if (st == MOE_OK && ce == cudaSuccess && r > 0) {
     // factors padded with zeros to the k16 rank r (caller rank r0 <= r)
@@ -368,13 +374,12 @@ moe_status_t moe_layer_set_expert_weights(moe_layer_t* L, int e, int block, cons
       db = t5.p;
     }
     if (st == MOE_OK) st = dalloc(S.afrag, (size_t)r * Kin * sizeof(__half));
-    if (st == MOE_OK) st = dalloc(S.bfrag, (size_t)M * r * sizeof(__half));
+    if (st == MOE_OK) st = dalloc(S.brow, (size_t)M * r * sizeof(__half));
     if (st == MOE_OK && ce == cudaSuccess) {
-      ce = launch_relayout_dense(static_cast<const __nv_bfloat16*>(da), static_cast<uint4*>(S.afrag.p), r, Kin, -1,
-                                 L->N, Kin, 0, s0);
+      ce = launch_relayout_afrag(static_cast<const __nv_bfloat16*>(da), static_cast<uint4*>(S.afrag.p), r, Kin, s0);
       if (ce == cudaSuccess)
-        ce = launch_relayout_dense(static_cast<const __nv_bfloat16*>(db), static_cast<uint4*>(S.bfrag.p), M, r, block,
-                                   L->N, r, 0, s0);
+        ce = launch_relayout_brow(static_cast<const __nv_bfloat16*>(db), static_cast<uint32_t*>(S.brow.p), M, r, block,
+                                  L->N, s0);
     }
   }
   if (st == MOE_OK && ce == cudaSuccess) ce = cudaDeviceSynchronize();
@@ -393,8 +398,8 @@ moe_status_t moe_layer_set_expert_weights(moe_layer_t* L, int e, int block, cons
   d.sz = static_cast<const uint32_t*>(S.sz.p);
   d.lut = static_cast<const uint32_t*>(S.lut.p);
   d.afrag = static_cast<const uint4*>(S.afrag.p);
-  d.bfrag = static_cast<const uint4*>(S.bfrag.p);
-  d.plane_stride = (long long)MF * KC * 256;
+  d.brow = static_cast<const uint32_t*>(S.brow.p);
+  d.plane_stride = (long long)KC * RB * 1024;
   d.loaded = 1;
   return upload_desc(L, e);
 }
@@ -417,7 +422,7 @@ moe_status_t moe_layer_set_bits(moe_layer_t* L, int e, int block, int bits) {
       d.codes = nullptr;
       d.sz = nullptr;
       d.afrag = nullptr;
-      d.bfrag = nullptr;
+      d.brow = nullptr;
     }
   }
   return upload_desc(L, e);
@@ -505,8 +510,6 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
   ra.pinv = static_cast<int*>(L->pinv.p);
   ra.act = L->xact.p;
   ra.Kpad = L->Kpad_x;
-  ra.nt8cap = L->nt8cap;
-  ra.act_layout = prefill ? ACT_ROW : ACT_FRAG;
   ra.status = static_cast<unsigned*>(L->status.p);
   L->prof_names.clear();
   prof_mark(L, st, "route_topk");
@@ -527,7 +530,6 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     la.poffsets = ra.poffsets;
     la.act = act;
     la.Kpad = Kpad;
-    la.nt8cap = L->nt8cap;
     la.K = Kin;
     // token tiles of 64 rows per expert; split K only while the grid is small
     la.tiles = (int)std::min<long long>((T + 63) / 64, (rows + 63) / 64);
@@ -539,7 +541,6 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     la.part = static_cast<float*>(L->part.p);
     la.part_ks_stride = (long long)L->rows_pad_max * kMaxRank;
     la.sem = static_cast<int*>(L->sem.p);
-    la.act_layout = prefill ? ACT_ROW : ACT_FRAG;
     la.status = ra.status;
     prof_mark(L, st, block == 0 ? "lowrank_w1" : "lowrank_w2");
     ce = launch_lowrank(la, grid_y, st, &launches);
@@ -575,56 +576,42 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N);
     prefill_gemm(1, L->tmap_z, N, K, MODE_OUT);
   } else {
-    // token tiles per pass: cover the expected per-expert batch (mean + 3 sd);
+    // tokens per pass: cover the expected per-expert batch (mean + 3 sd);
     // larger batches take more passes
     const double avg = (double)rows / E;
-    int nt_max = (int)std::ceil((avg + 3.0 * std::sqrt(avg) + 1.0) / 8.0);
-    nt_max = std::max(1, std::min(nt_max, std::min(4, (T + 7) / 8)));
-    if (ce == cudaSuccess) {
-      GemmArgs ga{};
-      ga.experts = dexp;
-      ga.block = 0;
-      ga.active = ra.active;
-      ga.n_active = ra.n_active;
-      ga.counts = ra.counts;
-      ga.poffsets = ra.poffsets;
-      ga.act = static_cast<const uint4*>(L->xact.p);
-      ga.nt8cap = L->nt8cap;
-      ga.K = K;
-      ga.M = 2 * N;
-      ga.mode = MODE_SWIGLU;
-      ga.zout = static_cast<__half*>(L->zact.p);
-      ga.KS = 1;
-      ga.status = ra.status;
-      prof_mark(L, st, "decode_gemm_w1_swiglu");
-      ce = launch_decode_gemm(ga, nt_max, maxbits[0], grid_y, st, &launches);
-    }
+    const int want = (int)std::ceil(avg + 3.0 * std::sqrt(avg) + 1.0);
+    const int ntok = std::min(64, std::min(T, want) <= 16 ? 16 : std::min(T, want) <= 32 ? 32 : 64);
+    auto decode_gemm = [&](int block, const CUtensorMap& map, int Kin, int M, int mode, int KS) {
+      if (ce != cudaSuccess) return;
+      DecodeArgs da;
+      std::memset(&da, 0, sizeof(da));
+      da.tmap_act = map;
+      da.experts = dexp;
+      da.block = block;
+      da.active = ra.active;
+      da.n_active = ra.n_active;
+      da.counts = ra.counts;
+      da.poffsets = ra.poffsets;
+      da.K = Kin;
+      da.M = M;
+      da.mode = mode;
+      da.zout = static_cast<__half*>(L->zact.p);
+      da.ldz = L->Kpad_z;
+      da.out = static_cast<float*>(L->obuf.p);
+      da.out_ks_stride = prows * K;
+      da.KS = KS;
+      da.status = ra.status;
+      prof_mark(L, st, block == 0 ? "decode_gemm_w1_swiglu" : "decode_gemm_w2");
+      ce = launch_decode_gemm(da, ntok, maxbits[block], grid_y, st, &launches);
+    };
+    decode_gemm(0, L->tmap_xd, K, 2 * N, MODE_SWIGLU, 1);
     lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N);
-    if (ce == cudaSuccess) {
-      const int row_tiles = (K + decode_rows_per_cta() - 1) / decode_rows_per_cta();
-      const int want = 2 * 148;
-      ks2 = std::max(1, want / std::max(1, row_tiles * grid_y));
-      ks2 = std::min(ks2, std::min(L->ks2_max, N / kChunkK));
-      if (rows > 1024) ks2 = 1;
-      GemmArgs ga{};
-      ga.experts = dexp;
-      ga.block = 1;
-      ga.active = ra.active;
-      ga.n_active = ra.n_active;
-      ga.counts = ra.counts;
-      ga.poffsets = ra.poffsets;
-      ga.act = static_cast<const uint4*>(L->zact.p);
-      ga.nt8cap = L->nt8cap;
-      ga.K = N;
-      ga.M = K;
-      ga.mode = MODE_OUT;
-      ga.out = static_cast<float*>(L->obuf.p);
-      ga.out_ks_stride = prows * K;
-      ga.KS = ks2;
-      ga.status = ra.status;
-      prof_mark(L, st, "decode_gemm_w2");
-      ce = launch_decode_gemm(ga, nt_max, maxbits[1], grid_y, st, &launches);
-    }
+    // split the down projection's K while its grid is small (fixed-order sum in the combine)
+    const int row_tiles = K / decode_rows_per_cta();
+    ks2 = std::max(1, 600 / std::max(1, row_tiles * grid_y));
+    ks2 = std::min(ks2, std::min(L->ks2_max, N / 256));
+    if (rows > 1024) ks2 = 1;
+    decode_gemm(1, L->tmap_zd, N, K, MODE_OUT, ks2);
   }
   if (ce == cudaSuccess) {
     CombineArgs ca{};

@@ -23,6 +23,7 @@
 
 #include "kernels.h"
 #include "decode_frag.cuh"
+#include "tc.cuh"
 
 namespace moeq {
 
@@ -34,11 +35,11 @@ constexpr int kBN = 256;           // weight rows per CTA
 constexpr int kFr = kBN / 16;      // row fragments per CTA
 constexpr int kBK = 64;            // K per stage (one 128-byte swizzle atom of fp16)
 constexpr int kTileM = 128;        // tokens per accumulator
-constexpr int kSA = 3, kSB = 2, kSC = 2;
+constexpr int kSA = 3, kSB = 2, kSC = 3;
 constexpr int kATile = kTileM * kBK * 2;       // 16 KiB
 constexpr int kASlot = 2 * kATile;             // 32 KiB
 constexpr int kBSlot = kBN * kBK * 2;          // 32 KiB
-constexpr int kCSlot = kFr * 1024 + 2 * 1024;  // codes (<= 4 bits) + scales, 18 KiB
+constexpr int kCSlot = 2 * 4096 + 1024;        // two 128-row code blocks (<= 4 bits) + scales, 9 KiB
 constexpr int kSmemA = 0;
 constexpr int kSmemB = kSmemA + kSA * kASlot;
 constexpr int kSmemC = kSmemB + kSB * kBSlot;
@@ -47,58 +48,7 @@ constexpr int kNumBars = 2 * kSA + 2 * kSB + 2 * kSC + 1;
 constexpr int kSmemTotal = kSmemBar + kNumBars * 8 + 16;
 constexpr int kSmemAlloc = kSmemTotal + 1024;  // slack to align the base to 1024 B
 
-// tcgen05 instruction descriptor, kind::f16: D fp32, A/B fp16, both K-major,
-// N = 256, M = 128.
-constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
-
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address
-  d |= (uint64_t)1 << 16;                    // leading byte offset (unused for swizzled K-major)
-  d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset: 8 rows x 128 B
-  d |= (uint64_t)1 << 46;                    // descriptor version
-  d |= (uint64_t)2 << 61;                    // 128-byte swizzle
-  return d;
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::
-          "r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, int acc) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc));
-}
-
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-}
-
-// byte offset of element (row, k) (k < 64) in a K-major, 128-byte-swizzled tile
-__device__ __forceinline__ uint32_t sw128_off(int row, int k) {
-  const int chunk = (k >> 3) ^ (row & 7);
-  return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + chunk * 16 + (k & 7) * 2);
-}
+constexpr uint32_t kIdesc = idesc_f16(kTileM, kBN);
 
 struct Ctx {
   int e, n_e, prow0, rt, pair, ntile_live, nk;  // nk: 64-wide stages incl. the compensator stage
@@ -110,38 +60,34 @@ __device__ void producer(const PrefillArgs& a, const BlockDesc& d, const Ctx& c,
                          volatile int* abort_flag) {
   const uint32_t a_full = bars, a_empty = bars + 8 * kSA;
   const uint32_t c_full = bars + 8 * (2 * kSA + 2 * kSB), c_empty = c_full + 8 * kSC;
-  const int MF = a.M / 16;
-  const int rf0 = c.rt * kFr;
-  const int nfr = min(kFr, MF - rf0);
-  constexpr int CB = 256 * BITS;
-  constexpr int GPC = (FMT == FMT_INT) ? (kChunkK / GROUP) : 0;
+  const int RB = a.M / 128;
+  const int rb0 = c.rt * 2;
+  const int nrb = min(2, RB - rb0);
+  constexpr int kBlk = 128 * 8 * BITS;  // bytes of one 128-row code block (per plane: 1 KiB)
   const int row0 = c.prow0 + c.pair * 2 * kTileM;
   int issued_a = 0, issued_c = 0;
   for (int i = 0; i < c.nk && !*abort_flag; ++i) {
-    // code chunk for stages 2i' and 2i'+1 (main K only)
-    if ((i & 1) == 0 && (i >> 1) < c.KC) {
-      const int ch = i >> 1, slot = ch % kSC;
-      if (ch >= kSC && !mbar_wait(c_empty + 8 * slot, ((ch / kSC) & 1) ^ 1, a.status)) {
+    // code blocks + scales of stage i (main K only)
+    if (i < c.KC) {
+      const int slot = i % kSC;
+      if (i >= kSC && !mbar_wait(c_empty + 8 * slot, ((i / kSC) & 1) ^ 1, a.status)) {
         *abort_flag = 1;
         break;
       }
       uint8_t* cs = sm + kSmemC + slot * kCSlot;
-      const uint32_t wb = (FMT == FMT_BITPLANE ? BITS * 256 : CB) * nfr;
-      mbar_expect_tx(c_full + 8 * slot, wb + GPC * nfr * 64);
+      const long long bidx = (long long)i * RB + rb0;
+      const uint32_t wb = (FMT == FMT_BITPLANE ? BITS * 1024 : kBlk) * nrb;
+      mbar_expect_tx(c_full + 8 * slot, wb + (FMT == FMT_INT ? 512 * nrb : 0));
       if constexpr (FMT == FMT_BITPLANE) {
 #pragma unroll
         for (int p = 0; p < BITS; ++p)
-          bulk_g2s(smem_u32(cs + p * (kFr * 256)), d.codes + p * d.plane_stride + ((long long)ch * MF + rf0) * 256,
-                   256 * nfr, c_full + 8 * slot);
+          bulk_g2s(smem_u32(cs + p * 2048), d.codes + p * d.plane_stride + bidx * 1024, 1024 * nrb, c_full + 8 * slot);
       } else {
-        bulk_g2s(smem_u32(cs), d.codes + ((long long)ch * MF + rf0) * CB, CB * nfr, c_full + 8 * slot);
+        bulk_g2s(smem_u32(cs), d.codes + bidx * kBlk, kBlk * nrb, c_full + 8 * slot);
       }
-      if constexpr (FMT == FMT_INT) {
-#pragma unroll
-        for (int gi = 0; gi < GPC; ++gi)
-          bulk_g2s(smem_u32(cs + kFr * 1024 + gi * 1024), d.sz + ((long long)(ch * GPC + gi) * MF + rf0) * 16,
-                   64 * nfr, c_full + 8 * slot);
-      }
+      if constexpr (FMT == FMT_INT)
+        bulk_g2s(smem_u32(cs + 8192), d.sz + (long long)(i * 64 / GROUP) * a.M + rb0 * 128, 512 * nrb,
+                 c_full + 8 * slot);
       ++issued_c;
     }
     // activation tiles of stage i
@@ -184,7 +130,7 @@ __device__ void mma_issuer(const Ctx& c, uint8_t* sm, uint32_t bars, uint32_t tm
     for (int k16 = 0; k16 < kBK / 16; ++k16) {
       const uint64_t bdesc = sw128_desc(bbase + k16 * 32);
       for (int t = 0; t < c.ntile_live; ++t)
-        mma_f16(tmem + t * kBN, sw128_desc(abase + t * kATile + k16 * 32), bdesc, kIdesc, (i > 0 || k16 > 0));
+        mma_f16_ss(tmem + t * kBN, sw128_desc(abase + t * kATile + k16 * 32), bdesc, kIdesc, (i > 0 || k16 > 0));
     }
     mma_commit(a_empty + 8 * sa);
     mma_commit(b_empty + 8 * sb);
@@ -196,16 +142,20 @@ template <int FMT, int BITS, int GROUP>
 __device__ void dequant_and_epilogue(const PrefillArgs& a, const BlockDesc& d, const Ctx& c, uint8_t* sm,
                                      uint32_t bars, uint32_t tmem, volatile int* abort_flag) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int dw = warp - 2;  // 0..7
-  const int g = lane >> 2, cc = lane & 3;
+  const int dw = warp - 2;               // 0..7
+  const int t = threadIdx.x - 64;        // weight row of the tile, 0..255
   const uint32_t b_full = bars + 8 * 2 * kSA, b_empty = b_full + 8 * kSB;
   const uint32_t c_full = bars + 8 * (2 * kSA + 2 * kSB), c_empty = c_full + 8 * kSC;
   const uint32_t acc_full = bars + 8 * (2 * kSA + 2 * kSB + 2 * kSC);
-  const int MF = a.M / 16;
-  const int rf0 = c.rt * kFr;
-  const int nfr = min(kFr, MF - rf0);
+  const int RB = a.M / 128;
+  const int rb = c.rt * 2 + (t >> 7);    // this thread's 128-row block
+  const bool rvalid = rb < RB;
+  const int R = c.rt * kBN + t;          // internal row
+  const int nfr = min(kFr, a.M / 16 - c.rt * kFr);
+  constexpr int kBlk = 128 * 8 * BITS;
   LutRegs lut;
   if constexpr (FMT == FMT_BITPLANE) lut = load_lut(d.lut, BITS);
+  const int RS2 = d.rank / 2;
   bool ok = true;
   for (int i = 0; i < c.nk && ok; ++i) {
     const int sb = i % kSB;
@@ -214,98 +164,38 @@ __device__ void dequant_and_epilogue(const PrefillArgs& a, const BlockDesc& d, c
       break;
     }
     uint8_t* bt = sm + kSmemB + sb * kBSlot;
-    if ((i >> 1) < c.KC) {
-      const int ch = i >> 1, cs_slot = ch % kSC, half = i & 1;
-      if (!mbar_wait(c_full + 8 * cs_slot, (ch / kSC) & 1, a.status)) {
+    uint32_t v[32];
+    if (i < c.KC) {
+      const int cs_slot = i % kSC;
+      if (!mbar_wait(c_full + 8 * cs_slot, (i / kSC) & 1, a.status)) {
         ok = false;
         break;
       }
       const uint8_t* cs = sm + kSmemC + cs_slot * kCSlot;
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int rl = dw * 2 + r;  // local row fragment 0..15
+      if (rvalid) {
         uint32_t w[8];
-        if (rl < nfr) {
-          if constexpr (FMT == FMT_INT && BITS == 4) {
-            const uint4* p = reinterpret_cast<const uint4*>(cs + rl * 1024);
-            const uint4 v0 = p[lane], v1 = p[32 + lane];
-            w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-            w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
-          } else if constexpr (FMT == FMT_INT) {
-            const uint8_t* ws = cs + rl * (256 * BITS);
-            const uint4 v0 = reinterpret_cast<const uint4*>(ws)[lane];
-            w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-            if constexpr (BITS == 3) {
-              const uint2 h = reinterpret_cast<const uint2*>(ws + 512)[lane];
-              w[4] = h.x; w[5] = h.y;
-            }
-          } else {
-#pragma unroll
-            for (int p = 0; p < BITS; ++p) {
-              const uint2 v = reinterpret_cast<const uint2*>(cs + p * (kFr * 256) + rl * 256)[lane];
-              w[2 * p] = v.x; w[2 * p + 1] = v.y;
-            }
-          }
+        uint32_t sz = 0;
+        if constexpr (FMT == FMT_INT) {
+          load_row_words_int(cs + (t >> 7) * kBlk, t & 127, BITS, w);
+          sz = reinterpret_cast<const uint32_t*>(cs + 8192)[t];
         } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) w[q] = 0u;
+          load_row_planes<BITS>(cs + (t >> 7) * 1024, 2048, t & 127, w);
         }
-        uint32_t sA = 0, nA = 0, sB = 0, nB = 0;
+        decode_row64<FMT, BITS>(w, sz, lut, v);
+      } else {
 #pragma unroll
-        for (int s4 = 0; s4 < 4; ++s4) {
-          const int s = half * 4 + s4;  // step within the 128-wide chunk
-          uint32_t av[4];
-          if constexpr (FMT == FMT_INT) {
-            if (s4 == 0 || (16 * s) % GROUP == 0) {
-              const int gs = (16 * s) / GROUP;
-              const uint2 z2 = rl < nfr ? *reinterpret_cast<const uint2*>(cs + kFr * 1024 + gs * 1024 + rl * 64 + g * 8)
-                                        : make_uint2(0u, 0u);
-              sA = prmt(z2.x, z2.x, 0x1010u); nA = prmt(z2.x, z2.x, 0x3232u);
-              sB = prmt(z2.y, z2.y, 0x1010u); nB = prmt(z2.y, z2.y, 0x3232u);
-            }
-            uint32_t q[4];
-            if (half == 0) int_codes<BITS>(w, s4, q);
-            else int_codes<BITS>(w, 4 + s4, q);
-            av[0] = hfma2u(q[0], sA, nA);
-            av[1] = hfma2u(q[1], sB, nB);
-            av[2] = hfma2u(q[2], sA, nA);
-            av[3] = hfma2u(q[3], sB, nB);
-          } else {
-            if (half == 0) lut_decode<BITS>(plane_codes<BITS>(w, s4), lut, av);
-            else lut_decode<BITS>(plane_codes<BITS>(w, 4 + s4), lut, av);
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int row = rl * 16 + g + 8 * (j & 1);
-            const int k = 16 * s4 + 2 * cc + 8 * (j >> 1);
-            *reinterpret_cast<uint32_t*>(bt + sw128_off(row, k)) = av[j];
-          }
-        }
+        for (int q = 0; q < 32; ++q) v[q] = 0u;
       }
-      if (half == 1) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(c_empty + 8 * cs_slot);
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(c_empty + 8 * cs_slot);
     } else {
-      // compensator stage: B factor columns [0, r), zeros up to 64
-      const int RS = d.rank / 16;
+      // compensator stage: the row's B values (pairs), zero past the rank
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int rl = dw * 2 + r;
-#pragma unroll
-        for (int s4 = 0; s4 < 4; ++s4) {
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (s4 < RS && rl < nfr) v = d.bfrag[((long long)(rf0 + rl) * RS + s4) * 32 + lane];
-          const uint32_t av[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int row = rl * 16 + g + 8 * (j & 1);
-            const int k = 16 * s4 + 2 * cc + 8 * (j >> 1);
-            *reinterpret_cast<uint32_t*>(bt + sw128_off(row, k)) = av[j];
-          }
-        }
-      }
+      for (int q = 0; q < 32; ++q) v[q] = (rvalid && q < RS2) ? d.brow[(long long)q * a.M + R] : 0u;
     }
+#pragma unroll
+    for (int s8 = 0; s8 < 8; ++s8)
+      *reinterpret_cast<uint4*>(bt + sw128_off(t, 8 * s8)) = make_uint4(v[4 * s8], v[4 * s8 + 1], v[4 * s8 + 2], v[4 * s8 + 3]);
     fence_proxy_async();
     __syncwarp();
     if (lane == 0) mbar_arrive(b_full + 8 * sb);
@@ -314,6 +204,7 @@ __device__ void dequant_and_epilogue(const PrefillArgs& a, const BlockDesc& d, c
     *abort_flag = 1;
     return;
   }
+  const int rf0 = c.rt * kFr;
   // ---- epilogue
   if (!mbar_wait(acc_full, 0, a.status)) {
     *abort_flag = 1;
@@ -322,6 +213,7 @@ __device__ void dequant_and_epilogue(const PrefillArgs& a, const BlockDesc& d, c
   tc_fence_after();
   const int quarter = warp & 3;        // TMEM lanes 32*quarter .. +31
   const int chalf = dw >> 2;           // column half handled by this warp
+  (void)nfr;
   for (int t = 0; t < c.ntile_live; ++t) {
     const int n = c.pair * 2 * kTileM + t * kTileM + quarter * 32 + lane;  // token within the expert
     const bool live = n < c.n_e;
@@ -382,7 +274,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_gemm_kernel(const __g
   c.ntile_live = (c.n_e - c.pair * 2 * pf::kTileM) > pf::kTileM ? 2 : 1;
   c.prow0 = a.poffsets[c.e];
   c.rt = blockIdx.x;
-  c.KC = a.K / kChunkK;
+  c.KC = a.K / pf::kBK;
   const BlockDesc d = a.experts[c.e].blk[a.block];
   c.nk = a.K / pf::kBK + (d.rank > 0 ? 1 : 0);
   const uint32_t bars = smem_u32(sm + pf::kSmemBar);
@@ -404,13 +296,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_gemm_kernel(const __g
     abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;\n" ::"r"(smem_u32(&tmem_slot)));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
-  }
-  pf::tc_fence_before();
+  if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), 512);
+  tc_fence_before();
   __syncthreads();
-  pf::tc_fence_after();
+  tc_fence_after();
   const uint32_t tmem = tmem_slot;
   volatile int* ab = &abort_flag;
   bool ran = true;
@@ -435,11 +324,11 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_gemm_kernel(const __g
     ran = false;
   }
   if (!ran && threadIdx.x == 0) atomicOr(a.status, ST_BOUNDS);
-  pf::tc_fence_before();
+  tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    pf::tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;\n" ::"r"(tmem));
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 

@@ -1,6 +1,7 @@
 // Load-time re-layout of canonical weight formats into the internal
-// fragment-ordered layouts (see common.cuh), and the debug unpack that runs
-// the GEMM kernels' own decode routine backwards to canonical order.
+// row-per-thread block layout (see common.cuh), and the debug unpack that runs
+// the GEMM kernels' own decode routine and writes the codes back in canonical
+// order.
 #include "kernels.h"
 #include "decode_frag.cuh"
 
@@ -14,156 +15,166 @@ __device__ __forceinline__ int read_code(const uint8_t* row, int rowbytes, int b
   return (int)((v >> sh) & ((1u << bits) - 1u));
 }
 
-// one thread per (rf, kc, lane)
-__global__ void relayout_int_kernel(const uint8_t* __restrict__ canon, uint8_t* __restrict__ out, int M, int K,
-                                    int bits, int block, int N) {
-  const int KC = K / kChunkK, MF = M / 16;
-  const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-  if (tid >= (long long)MF * KC * 32) return;
-  const int lane = (int)(tid & 31);
-  const long long ch = tid >> 5;
-  const int kc = (int)(ch % KC), rf = (int)(ch / KC);
-  const int rowbytes = K * bits / 8;
-  uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+// Packs the 64 codes c[k] (k = 8s + 2j + h) of one row-chunk into the words
+// the decode routine expects (see decode_frag.cuh).
+__device__ __forceinline__ void pack_int_words(const int (&c)[64], int bits, uint32_t (&w)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w[i] = 0u;
   for (int s = 0; s < 8; ++s)
     for (int j = 0; j < 4; ++j)
       for (int h = 0; h < 2; ++h) {
-        int r, k;
-        frag_elem(lane, s, j, h, r, k);
-        const int crow = canon_row(16 * rf + r, block, N);
-        const int q = read_code(canon + (long long)crow * rowbytes, rowbytes, bits, kc * kChunkK + k);
+        const int q = c[8 * s + 2 * j + h];
         if (bits == 4) {
           w[s] |= (uint32_t)q << (4 * (j + 4 * h));
         } else {
           const int p = 4 * (s & 1) + j;
-          const int pos = 2 * (p & 3) + 8 * (p >> 2) + 16 * h;
-          w[s >> 1] |= (uint32_t)(q & 3) << pos;
+          w[s >> 1] |= (uint32_t)(q & 3) << (2 * (p & 3) + 8 * (p >> 2) + 16 * h);
           if (bits == 3) {
-            const int t = s & 3;  // transform of hi word s>>2
+            const int t = s & 3;  // transform applied to hi word s>>2
             const int base = (h ? 18 : 2) + 2 * j;
             const int src = t == 0 ? base : t == 1 ? base + 1 : t == 2 ? (base + 8) & 31 : (base + 9) & 31;
             w[4 + (s >> 2)] |= (uint32_t)(q >> 2) << src;
           }
         }
       }
-  uint32_t* chunk = reinterpret_cast<uint32_t*>(out + ((long long)kc * MF + rf) * 256LL * bits);
+}
+
+// word-quad-major store of one row's words into a [128-row] block
+__device__ __forceinline__ void store_row_words(uint8_t* blk, int row, int bits, const uint32_t (&w)[8]) {
   if (bits == 4) {
-    for (int s = 0; s < 8; ++s) chunk[(s >> 2) * 128 + lane * 4 + (s & 3)] = w[s];
+    reinterpret_cast<uint4*>(blk)[row] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(blk + 2048)[row] = make_uint4(w[4], w[5], w[6], w[7]);
   } else {
-    for (int i = 0; i < 4; ++i) chunk[lane * 4 + i] = w[i];
-    if (bits == 3) {
-      chunk[128 + lane * 2 + 0] = w[4];
-      chunk[128 + lane * 2 + 1] = w[5];
-    }
+    reinterpret_cast<uint4*>(blk)[row] = make_uint4(w[0], w[1], w[2], w[3]);
+    if (bits == 3) reinterpret_cast<uint2*>(blk + 2048)[row] = make_uint2(w[4], w[5]);
   }
 }
 
-// one thread per (rf, group, g): half2(s, -z*s) for rows g and g+8
+// one thread per (chunk kc, internal row)
+__global__ void relayout_int_kernel(const uint8_t* __restrict__ canon, uint8_t* __restrict__ out, int M, int K,
+                                    int bits, int block, int N) {
+  const int KC = K / 64;
+  const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (tid >= (long long)KC * M) return;
+  const int row = (int)(tid % M), kc = (int)(tid / M);
+  const int crow = canon_row(row, block, N);
+  const int rowbytes = K * bits / 8;
+  int c[64];
+  for (int k = 0; k < 64; ++k) c[k] = read_code(canon + (long long)crow * rowbytes, rowbytes, bits, kc * 64 + k);
+  uint32_t w[8];
+  pack_int_words(c, bits, w);
+  uint8_t* blk = out + ((long long)kc * (M / 128) + row / 128) * block_bytes(FMT_INT, bits);
+  store_row_words(blk, row % 128, bits, w);
+}
+
+// one thread per (group, internal row): half2(s, -z*s)
 __global__ void relayout_sz_kernel(const __half* __restrict__ s, const __half* __restrict__ z,
                                    uint32_t* __restrict__ out, int M, int K, int group, int block, int N) {
-  const int G = K / group, MF = M / 16;
+  const int G = K / group;
   const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-  if (tid >= (long long)MF * G * 8) return;
-  const int g = (int)(tid & 7);
-  const long long t2 = tid >> 3;
-  const int gi = (int)(t2 % G), rf = (int)(t2 / G);
-  for (int hrow = 0; hrow < 2; ++hrow) {
-    const int crow = canon_row(16 * rf + g + 8 * hrow, block, N);
-    const float sv = __half2float(s[(long long)crow * G + gi]);
-    const float zv = __half2float(z[(long long)crow * G + gi]);
-    out[(((long long)gi * MF + rf) * 8 + g) * 2 + hrow] = pack_half2(sv, -zv * sv);
+  if (tid >= (long long)G * M) return;
+  const int row = (int)(tid % M), gi = (int)(tid / M);
+  const int crow = canon_row(row, block, N);
+  const float sv = __half2float(s[(long long)crow * G + gi]);
+  const float zv = __half2float(z[(long long)crow * G + gi]);
+  out[(long long)gi * M + row] = pack_half2(sv, -zv * sv);
+}
+
+// dense bf16 [M, K] (rows mapped by block/N) -> fp16 blocks: per (kc, rb),
+// 8 quads x [128 rows x 16 B], quad q of a row = k 8q..8q+7
+__global__ void relayout_dense_kernel(const __nv_bfloat16* __restrict__ src, uint8_t* __restrict__ out, int M, int K,
+                                      int block, int N) {
+  const int KC = K / 64;
+  const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (tid >= (long long)KC * M) return;
+  const int row = (int)(tid % M), kc = (int)(tid / M);
+  const int crow = canon_row(row, block, N);
+  uint8_t* blk = out + ((long long)kc * (M / 128) + row / 128) * block_bytes(FMT_DENSE, 16);
+  for (int q = 0; q < 8; ++q) {
+    uint32_t v[4];
+    for (int j = 0; j < 4; ++j) {
+      const int k = kc * 64 + 8 * q + 2 * j;
+      v[j] = pack_half2(__bfloat162float(src[(long long)crow * K + k]), __bfloat162float(src[(long long)crow * K + k + 1]));
+    }
+    reinterpret_cast<uint4*>(blk + q * 2048)[row % 128] = make_uint4(v[0], v[1], v[2], v[3]);
   }
 }
 
-// dense bf16 [rows, K] (row map by block/N, or identity when block < 0) ->
-// fp16 A fragments [MF][K/16][32] uint4
-__global__ void relayout_dense_kernel(const __nv_bfloat16* __restrict__ src, uint4* __restrict__ out, int M, int K,
-                                      int block, int N, long long src_ld, int chunked) {
-  const int S = K / 16, MF = M / 16;
+// compensator A [r, K] bf16 -> mma A-fragments [r/16][K/16][32] uint4 (fp16), r a multiple of 16
+__global__ void relayout_afrag_kernel(const __nv_bfloat16* __restrict__ src, uint4* __restrict__ out, int r, int K) {
+  const int S = K / 16;
   const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-  if (tid >= (long long)MF * S * 32) return;
+  if (tid >= (long long)(r / 16) * S * 32) return;
   const int lane = (int)(tid & 31);
   const long long t2 = tid >> 5;
   const int st = (int)(t2 % S), rf = (int)(t2 / S);
+  const int g = lane >> 2, c = lane & 3;
   uint32_t v[4];
   for (int j = 0; j < 4; ++j) {
-    float e[2];
-    for (int h = 0; h < 2; ++h) {
-      int r, k;
-      frag_elem(lane, 0, j, h, r, k);
-      const int row = 16 * rf + r;
-      const int crow = block < 0 ? row : canon_row(row, block, N);
-      e[h] = __bfloat162float(src[(long long)crow * src_ld + 16 * st + k]);
-    }
-    v[j] = pack_half2(e[0], e[1]);
+    const int row = 16 * rf + g + 8 * (j & 1);
+    const int k = 16 * st + 2 * c + 8 * (j >> 1);
+    v[j] = pack_half2(__bfloat162float(src[(long long)row * K + k]), __bfloat162float(src[(long long)row * K + k + 1]));
   }
-  // chunked: [kc][rf][8 steps][32] (the GEMM weight layout); else [rf][K/16][32]
-  const long long o = chunked ? ((((long long)(st >> 3) * MF + rf) * 8 + (st & 7)) * 32 + lane) : tid;
-  out[o] = make_uint4(v[0], v[1], v[2], v[3]);
+  out[tid] = make_uint4(v[0], v[1], v[2], v[3]);
 }
 
-// bit-planes [4][M][K/32] u32 -> per plane [MF][KC][32] uint2
+// compensator B [M, r] bf16 -> fp16 pairs [r/2][M] in internal row order
+__global__ void relayout_brow_kernel(const __nv_bfloat16* __restrict__ src, uint32_t* __restrict__ out, int M, int r,
+                                     int block, int N) {
+  const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (tid >= (long long)(r / 2) * M) return;
+  const int row = (int)(tid % M), cp = (int)(tid / M);
+  const int crow = canon_row(row, block, N);
+  out[tid] = pack_half2(__bfloat162float(src[(long long)crow * r + 2 * cp]),
+                        __bfloat162float(src[(long long)crow * r + 2 * cp + 1]));
+}
+
+// bit-planes [4][M][K/32] u32 -> per plane [kc][rb][128 rows x 8 B]
 __global__ void relayout_planes_kernel(const uint32_t* __restrict__ canon, uint32_t* __restrict__ out, int M, int K,
                                        int block, int N) {
-  const int KC = K / kChunkK, MF = M / 16, KW = K / 32;
-  const long long per_plane = (long long)MF * KC * 32;
+  const int KC = K / 64, KW = K / 32;
+  const long long per_plane = (long long)KC * M;
   const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (tid >= per_plane * 4) return;
   const int p = (int)(tid / per_plane);
   const long long t = tid % per_plane;
-  const int lane = (int)(t & 31);
-  const long long ch = t >> 5;
-  const int kc = (int)(ch % KC), rf = (int)(ch / KC);
-  uint32_t w[2] = {0, 0};
+  const int row = (int)(t % M), kc = (int)(t / M);
+  const int crow = canon_row(row, block, N);
+  uint32_t w[2] = {0u, 0u};
   for (int s = 0; s < 8; ++s)
     for (int j = 0; j < 4; ++j)
       for (int h = 0; h < 2; ++h) {
-        int r, k;
-        frag_elem(lane, s, j, h, r, k);
-        const int crow = canon_row(16 * rf + r, block, N);
-        const int kk = kc * kChunkK + k;
+        const int kk = kc * 64 + 8 * s + 2 * j + h;
         const uint32_t word = canon[((long long)p * M + crow) * KW + (kk >> 5)];
-        const uint32_t bit = (word >> (kk & 31)) & 1u;
-        w[s >> 2] |= bit << (4 * (2 * j + h) + (s & 3));
+        w[s >> 2] |= ((word >> (kk & 31)) & 1u) << (4 * (2 * j + h) + (s & 3));
       }
-  const long long o = (((long long)p * KC + kc) * MF + rf) * 32 + lane;
-  out[o * 2 + 0] = w[0];
-  out[o * 2 + 1] = w[1];
+  const long long o = ((long long)p * KC + kc) * (M / 128) + row / 128;  // block index
+  reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(out) + o * 1024)[row % 128] = make_uint2(w[0], w[1]);
 }
 
 // ---------------------------------------------------------------------------
-// debug unpack: the GEMM's decode of each (rf, kc, lane), written back to
+// debug unpack: the GEMM's decode of each (chunk, row), written back to
 // canonical [M, K] order as uint8 codes.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int half_to_int(uint16_t h) { return (int)__half2float(__ushort_as_half(h)); }
 
 __global__ void debug_unpack_kernel(BlockDesc d, uint8_t* __restrict__ out, int block, int N) {
-  const int KC = d.K / kChunkK, MF = d.M / 16;
+  const int KC = d.K / 64;
   const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-  if (tid >= (long long)MF * KC * 32) return;
-  const int lane = (int)(tid & 31);
-  const long long ch = tid >> 5;
-  const int kc = (int)(ch % KC), rf = (int)(ch / KC);
+  if (tid >= (long long)KC * d.M) return;
+  const int row = (int)(tid % d.M), kc = (int)(tid / d.M);
+  const long long bidx = (long long)kc * (d.M / 128) + row / 128;
   uint32_t w[8];
   if (d.fmt == FMT_INT) {
-    const uint32_t* chunk = reinterpret_cast<const uint32_t*>(d.codes + ((long long)kc * MF + rf) * 256LL * d.bits);
-    if (d.bits == 4) {
-      for (int s = 0; s < 8; ++s) w[s] = chunk[(s >> 2) * 128 + lane * 4 + (s & 3)];
-    } else {
-      for (int i = 0; i < 4; ++i) w[i] = chunk[lane * 4 + i];
-      if (d.bits == 3) {
-        w[4] = chunk[128 + lane * 2];
-        w[5] = chunk[128 + lane * 2 + 1];
-      }
-    }
+    load_row_words_int(d.codes + bidx * block_bytes(FMT_INT, d.bits), row % 128, d.bits, w);
   } else {
     for (int p = 0; p < d.bits; ++p) {
-      const uint32_t* pl = reinterpret_cast<const uint32_t*>(d.codes + p * d.plane_stride);
-      const long long o = ((long long)kc * MF + rf) * 32 + lane;
-      w[2 * p] = pl[o * 2];
-      w[2 * p + 1] = pl[o * 2 + 1];
+      const uint2 v = reinterpret_cast<const uint2*>(d.codes + p * d.plane_stride + bidx * 1024)[row % 128];
+      w[2 * p] = v.x;
+      w[2 * p + 1] = v.y;
     }
   }
+  const int crow = canon_row(row, block, N);
   for (int s = 0; s < 8; ++s) {
     uint32_t q[4];
     uint32_t nib = 0;
@@ -176,13 +187,10 @@ __global__ void debug_unpack_kernel(BlockDesc d, uint8_t* __restrict__ out, int 
     }
     for (int j = 0; j < 4; ++j)
       for (int h = 0; h < 2; ++h) {
-        int r, k;
-        frag_elem(lane, s, j, h, r, k);
-        const int crow = canon_row(16 * rf + r, block, N);
         int code;
         if (d.fmt == FMT_INT) code = half_to_int((uint16_t)(h ? (q[j] >> 16) : (q[j] & 0xFFFF)));
         else code = (int)((nib >> (4 * (2 * j + h))) & 0xF);
-        out[(long long)crow * d.K + kc * kChunkK + k] = (uint8_t)code;
+        out[(long long)crow * d.K + kc * 64 + 8 * s + 2 * j + h] = (uint8_t)code;
       }
   }
 }
@@ -192,31 +200,35 @@ static inline unsigned grid_for(long long n, int bs) { return (unsigned)((n + bs
 
 cudaError_t launch_relayout_int(const uint8_t* canon, uint8_t* out, int M, int K, int bits, int block, int N,
                                 cudaStream_t st) {
-  const long long n = (long long)(M / 16) * (K / kChunkK) * 32;
-  relayout_int_kernel<<<grid_for(n, 256), 256, 0, st>>>(canon, out, M, K, bits, block, N);
+  relayout_int_kernel<<<grid_for((long long)(K / 64) * M, 256), 256, 0, st>>>(canon, out, M, K, bits, block, N);
   return cudaGetLastError();
 }
 cudaError_t launch_relayout_sz(const __half* s, const __half* z, uint32_t* out, int M, int K, int group, int block,
                                int N, cudaStream_t st) {
-  const long long n = (long long)(M / 16) * (K / group) * 8;
-  relayout_sz_kernel<<<grid_for(n, 256), 256, 0, st>>>(s, z, out, M, K, group, block, N);
+  relayout_sz_kernel<<<grid_for((long long)(K / group) * M, 256), 256, 0, st>>>(s, z, out, M, K, group, block, N);
   return cudaGetLastError();
 }
-cudaError_t launch_relayout_dense(const __nv_bfloat16* src, uint4* out, int M, int K, int block, int N,
-                                  long long ld, int chunked, cudaStream_t st) {
-  const long long n = (long long)(M / 16) * (K / 16) * 32;
-  relayout_dense_kernel<<<grid_for(n, 256), 256, 0, st>>>(src, out, M, K, block, N, ld, chunked);
+cudaError_t launch_relayout_dense(const __nv_bfloat16* src, uint8_t* out, int M, int K, int block, int N,
+                                  cudaStream_t st) {
+  relayout_dense_kernel<<<grid_for((long long)(K / 64) * M, 256), 256, 0, st>>>(src, out, M, K, block, N);
+  return cudaGetLastError();
+}
+cudaError_t launch_relayout_afrag(const __nv_bfloat16* src, uint4* out, int r, int K, cudaStream_t st) {
+  relayout_afrag_kernel<<<grid_for((long long)(r / 16) * (K / 16) * 32, 256), 256, 0, st>>>(src, out, r, K);
+  return cudaGetLastError();
+}
+cudaError_t launch_relayout_brow(const __nv_bfloat16* src, uint32_t* out, int M, int r, int block, int N,
+                                 cudaStream_t st) {
+  relayout_brow_kernel<<<grid_for((long long)(r / 2) * M, 256), 256, 0, st>>>(src, out, M, r, block, N);
   return cudaGetLastError();
 }
 cudaError_t launch_relayout_planes(const uint32_t* canon, uint32_t* out, int M, int K, int block, int N,
                                    cudaStream_t st) {
-  const long long n = (long long)(M / 16) * (K / kChunkK) * 32 * 4;
-  relayout_planes_kernel<<<grid_for(n, 256), 256, 0, st>>>(canon, out, M, K, block, N);
+  relayout_planes_kernel<<<grid_for((long long)(K / 64) * M * 4, 256), 256, 0, st>>>(canon, out, M, K, block, N);
   return cudaGetLastError();
 }
 cudaError_t launch_debug_unpack(const BlockDesc& d, uint8_t* out, int block, int N, cudaStream_t st) {
-  const long long n = (long long)(d.M / 16) * (d.K / kChunkK) * 32;
-  debug_unpack_kernel<<<grid_for(n, 256), 256, 0, st>>>(d, out, block, N);
+  debug_unpack_kernel<<<grid_for((long long)(d.K / 64) * d.M, 256), 256, 0, st>>>(d, out, block, N);
   return cudaGetLastError();
 }
 

@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_topk_kernel(RouteArgs a) 
 // grid: (token blocks of route_topk, K slices). Ranks within the block come
 // from per-expert token bitmasks; slice 0 writes perm/inv_pos; every CTA
 // gathers its K slice of the block's routed rows (bf16 -> fp16) into the
-// activation buffer, in the layout of the chosen GEMM path.
+// row-major fp16 activation buffer.
 __global__ void __launch_bounds__(kRouteThreads) route_permute_kernel(RouteArgs a) {
   __shared__ unsigned mask[kMaxExperts];
   __shared__ int prow_s[kRouteTokensPerCta * kMaxTopK];
@@ -179,28 +179,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_permute_kernel(RouteArgs 
   // gather of this CTA's K slice
   const int Kq = a.K;
   const int ks0 = (int)((long long)Kq * blockIdx.y / gridDim.y), ks1 = (int)((long long)Kq * (blockIdx.y + 1) / gridDim.y);
-  if (a.act_layout == ACT_FRAG) {
-    // one item = one uint4 of B fragments: (routed row, 32-wide k block, c)
-    const int kb0 = ks0 / 32, nkb = ks1 / 32 - kb0;
-    const int items = nt * a.k * nkb * 4;
-    for (int it = threadIdx.x; it < items; it += blockDim.x) {
-      const int c = it & 3;
-      const int rest = it >> 2;
-      const int kb = kb0 + rest % nkb;
-      const int i = rest / nkb;
-      const int t = t0 + i / a.k;
-      const long long prow = prow_s[i];
-      const __nv_bfloat16* x = a.X + (long long)t * Kq;
-      uint32_t v[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(x + 32 * kb + 2 * c + 8 * q);
-        v[q] = pack_half2(__bfloat162float(b2.x), __bfloat162float(b2.y));
-      }
-      uint4* dst = reinterpret_cast<uint4*>(a.act) + act_frag_u4(prow >> 3, kb, a.nt8cap, (int)(prow & 7) * 4 + c);
-      *dst = make_uint4(v[0], v[1], v[2], v[3]);
-    }
-  } else {
+  {
     // one item = 8 consecutive elements of a routed row
     const int k80 = ks0 / 8, nk8 = ks1 / 8 - k80;
     const int items = nt * a.k * nk8;
