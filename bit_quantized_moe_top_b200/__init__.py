@@ -24,7 +24,8 @@ FLAG_NO_TOPK_RENORM = 1
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 
 # every symbol the header declares
-EXPORTS = ["moe_layer_create", "moe_layer_set_expert_weights", "moe_layer_set_bits", "moe_layer_set_path",
+EXPORTS = ["moe_layer_create", "moe_layer_set_expert_weights", "moe_layer_set_bits", "moe_layer_set_comp_top_n",
+           "moe_layer_set_path",
            "moe_layer_forward", "moe_layer_forward_host", "moe_layer_get_routing", "moe_layer_debug_unpack",
            "moe_layer_sync_status", "moe_layer_last_launch_count", "moe_layer_set_profiling",
            "moe_layer_kernel_times", "moe_route_topk_noalloc", "moe_status_string", "moe_layer_destroy"]
@@ -56,6 +57,7 @@ def _lib() -> ctypes.CDLL:
         lib.moe_layer_set_expert_weights.argtypes = [P, I, I, P, P, P, P, P, I]
         lib.moe_layer_set_bits.argtypes = [P, I, I, I]
         lib.moe_layer_set_path.argtypes = [P, I]
+        lib.moe_layer_set_comp_top_n.argtypes = [P, I]
         lib.moe_layer_forward.argtypes = [P, P, P, I, I, P, P]
         lib.moe_layer_forward_host.argtypes = [P, P, P, I, I, P, P]
         lib.moe_layer_get_routing.argtypes = [P, P, P, P, P, P, P]
@@ -109,6 +111,10 @@ def moe_layer_set_expert_weights(layer: int, expert: int, block: int, codes, sca
 
 def moe_layer_set_bits(layer: int, expert: int, block: int, bits: int) -> None:
     _check(_lib().moe_layer_set_bits(layer, expert, block, bits), "moe_layer_set_bits")
+
+
+def moe_layer_set_comp_top_n(layer: int, n: int) -> None:
+    _check(_lib().moe_layer_set_comp_top_n(layer, n), "moe_layer_set_comp_top_n")
 
 
 def moe_layer_set_path(layer: int, path: int) -> None:
@@ -202,6 +208,9 @@ class MoELayer:
 
     def set_bits(self, expert, block, bits):
         moe_layer_set_bits(self.handle, expert, block, bits)
+
+    def set_comp_top_n(self, n):
+        moe_layer_set_comp_top_n(self.handle, n)
 
     def set_path(self, path):
         moe_layer_set_path(self.handle, path)

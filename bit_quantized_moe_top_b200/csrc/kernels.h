@@ -26,6 +26,7 @@ struct RouteArgs {
   int* perm_token;            // [T*k]
   int* inv_pos;               // [T, k]
   int* pinv;                  // [T, k] padded row
+  int* pslot;                 // [padded rows] routing slot of each routed row
   void* act;                  // activation buffer, fp16 row-major [rows, Kpad]
   int Kpad;
   unsigned* status;
@@ -66,6 +67,8 @@ struct LowrankArgs {
   long long part_ks_stride;
   int* sem;                   // [E][sem_stride], zero between launches
   long long sem_stride;
+  const int* pslot;           // routing slot of each padded row
+  int comp_top_n;             // > 0: rows in slots >= comp_top_n get U = 0 (no compensation)
   unsigned* status;
 };
 

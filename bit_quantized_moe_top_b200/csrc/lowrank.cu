@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
   }
   // acc[t][q]: row rbase + g + 8*(q>>1), column j = 8t + 2c + (q&1)
   auto store_u = [&](int n, int j, float v) {
+    // only the first comp_top_n routing slots of a token are compensated
+    if (a.comp_top_n > 0 && a.pslot[prow0 + n] >= a.comp_top_n) v = 0.f;
     a.act[(long long)(prow0 + n) * a.Kpad + a.K + j] = __float2half_rn(v);
   };
   if (a.KS == 1) {

@@ -65,7 +65,8 @@ struct moe_layer {
   long long rows_pad_max = 0, nt8cap = 0;
   int nb_max = 0, ks2_max = 1, kslr_max = 1;
   long long sem_stride = 0;
-  DevBuf idx, w, counts, offsets, poffsets, active, n_active, ticket, perm, inv_pos, pinv;
+  DevBuf idx, w, counts, offsets, poffsets, active, n_active, ticket, perm, inv_pos, pinv, pslot;
+  int comp_top_n = 0;
   DevBuf block_counts, block_base, pblock_base, sem, status;
   DevBuf xact, zact, obuf, part;
   DevBuf hx, hl, hy;  // device buffers for forward_host
@@ -171,7 +172,7 @@ void moe_layer_destroy(moe_layer_t* L) {
   if (!L) return;
   for (auto& s : L->store) free_block(s);
   DevBuf* bufs[] = {&L->d_experts, &L->idx, &L->w, &L->counts, &L->offsets, &L->poffsets, &L->active,
-                    &L->n_active, &L->ticket, &L->perm, &L->inv_pos, &L->pinv, &L->block_counts,
+                    &L->n_active, &L->ticket, &L->perm, &L->inv_pos, &L->pinv, &L->pslot, &L->block_counts,
                     &L->block_base, &L->pblock_base, &L->sem, &L->status, &L->xact, &L->zact, &L->obuf,
                     &L->part, &L->hx, &L->hl, &L->hy};
   for (DevBuf* b : bufs) dfree(*b);
@@ -245,6 +246,7 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   A(L->perm, sizeof(int) * rows);
   A(L->inv_pos, sizeof(int) * rows);
   A(L->pinv, sizeof(int) * rows);
+  A(L->pslot, sizeof(int) * (size_t)L->rows_pad_max);
   A(L->block_counts, sizeof(int) * (size_t)L->nb_max * E);
   A(L->block_base, sizeof(int) * (size_t)L->nb_max * E);
   A(L->pblock_base, sizeof(int) * (size_t)L->nb_max * E);
@@ -428,6 +430,12 @@ moe_status_t moe_layer_set_bits(moe_layer_t* L, int e, int block, int bits) {
   return upload_desc(L, e);
 }
 
+moe_status_t moe_layer_set_comp_top_n(moe_layer_t* L, int n) {
+  if (!L || n < 0 || n > L->max_top_k) return MOE_ERR_INVALID_ARG;
+  L->comp_top_n = n;
+  return MOE_OK;
+}
+
 moe_status_t moe_layer_set_path(moe_layer_t* L, int path) {
   if (!L || path < MOE_PATH_AUTO || path > MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
   L->path = path;
@@ -508,6 +516,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
   ra.perm_token = static_cast<int*>(L->perm.p);
   ra.inv_pos = static_cast<int*>(L->inv_pos.p);
   ra.pinv = static_cast<int*>(L->pinv.p);
+  ra.pslot = static_cast<int*>(L->pslot.p);
   ra.act = L->xact.p;
   ra.Kpad = L->Kpad_x;
   ra.status = static_cast<unsigned*>(L->status.p);
@@ -538,6 +547,8 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     ks = std::max(1, std::min(ks, std::min(L->kslr_max, Kin / 256)));
     la.KS = ks;
     la.sem_stride = L->sem_stride;
+    la.pslot = ra.pslot;
+    la.comp_top_n = L->comp_top_n;
     la.part = static_cast<float*>(L->part.p);
     la.part_ks_stride = (long long)L->rows_pad_max * kMaxRank;
     la.sem = static_cast<int*>(L->sem.p);

@@ -128,6 +128,14 @@ moe_status_t moe_layer_set_expert_weights(moe_layer_t* layer, int expert, int bl
  * MOE_ERR_UNSUPPORTED. Must not be called while a forward is in flight. */
 moe_status_t moe_layer_set_bits(moe_layer_t* layer, int expert, int block, int bits);
 
+/* Router-guided compensation: with n > 0, only the first n routing slots of
+ * each token (its n highest-logit experts) get the low-rank compensator; the
+ * other slots run on the quantised weights alone (Bandwidth-Efficient
+ * Adaptive Mixture-of-Experts via Low-Rank Compensation, abstract: Top-n
+ * (n < k) compensation per token). n = 0 (default) compensates every slot.
+ * 0 <= n <= max_top_k, else MOE_ERR_INVALID_ARG. */
+moe_status_t moe_layer_set_comp_top_n(moe_layer_t* layer, int n);
+
 /* Choose the kernel path (MOE_PATH_*). */
 moe_status_t moe_layer_set_path(moe_layer_t* layer, int path);
 

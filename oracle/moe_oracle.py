@@ -206,14 +206,18 @@ def expert_ffn(x: np.ndarray, W1: np.ndarray, W2: np.ndarray, N: int,
 
 def moe_forward(X: np.ndarray, logits: np.ndarray, top_k: int,
                 expert: Callable[[int], Dict], N: int, renorm: bool = True,
-                rows: Optional[Sequence[int]] = None) -> Dict:
+                rows: Optional[Sequence[int]] = None, comp_top_n: int = 0) -> Dict:
     """The layer's forward pass.
 
     ``expert(e)`` returns a dict with fp64 arrays W1 [2N, K], W2 [K, N] and
     optional A1, B1, A2, B2 (it is called only for experts that receive
     tokens). ``rows`` restricts the output to those tokens (routing and
-    bucketing are still computed for all tokens). Returns a dict with Y fp64
-    ([T, K] or [len(rows), K]) and the routing arrays.
+    bucketing are still computed for all tokens). ``comp_top_n`` > 0 applies
+    the compensators only to the first n routing slots of each token and runs
+    the other slots' experts on their quantised weights alone (Bandwidth-
+    Efficient Adaptive Mixture-of-Experts via Low-Rank Compensation, abstract:
+    compensation for the Top-n (n < k) experts of each token). Returns a dict
+    with Y fp64 ([T, K] or [len(rows), K]) and the routing arrays.
     """
     X64 = np.asarray(X, np.float64)
     T, K = X64.shape
@@ -222,6 +226,7 @@ def moe_forward(X: np.ndarray, logits: np.ndarray, top_k: int,
     counts, offsets, perm, inv = bucket(idx, E)
     want = np.arange(T) if rows is None else np.asarray(rows, np.int64)
     wanted = set(int(t) for t in want)
+    slot = {int(inv[t, j]): j for t in range(T) for j in range(top_k)}
     O = {}
     for e in range(E):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
@@ -229,10 +234,17 @@ def moe_forward(X: np.ndarray, logits: np.ndarray, top_k: int,
         if not ps:
             continue
         ex = expert(e)
-        xs = X64[perm[ps]]
-        o = expert_ffn(xs, ex["W1"], ex["W2"], N, ex.get("A1"), ex.get("B1"), ex.get("A2"), ex.get("B2"))
-        for i, p in enumerate(ps):
-            O[p] = o[i]
+        comp = [p for p in ps if comp_top_n <= 0 or slot[p] < comp_top_n]
+        plain = [p for p in ps if not (comp_top_n <= 0 or slot[p] < comp_top_n)]
+        if comp:
+            o = expert_ffn(X64[perm[comp]], ex["W1"], ex["W2"], N, ex.get("A1"), ex.get("B1"), ex.get("A2"),
+                           ex.get("B2"))
+            for i, p in enumerate(comp):
+                O[p] = o[i]
+        if plain:
+            o = expert_ffn(X64[perm[plain]], ex["W1"], ex["W2"], N)
+            for i, p in enumerate(plain):
+                O[p] = o[i]
     Y = np.zeros((len(want), K), np.float64)
     for i, t in enumerate(want):
         for j in range(top_k):

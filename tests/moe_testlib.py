@@ -95,10 +95,11 @@ class OracleExperts:
         return self.cache[e]
 
 
-def oracle_forward(cfg, blocks, X, logits, top_k, rows=None, renorm=True, bits_override=None):
+def oracle_forward(cfg, blocks, X, logits, top_k, rows=None, renorm=True, bits_override=None, comp_top_n=0):
     Xn = X.float().cpu().numpy().astype(np.float64)
     Ln = logits.cpu().numpy()
-    return orc.moe_forward(Xn, Ln, top_k, OracleExperts(blocks, bits_override), cfg.N, renorm=renorm, rows=rows)
+    return orc.moe_forward(Xn, Ln, top_k, OracleExperts(blocks, bits_override), cfg.N, renorm=renorm, rows=rows,
+                           comp_top_n=comp_top_n)
 
 
 def row_errors(Y: torch.Tensor, Yref: np.ndarray):

@@ -176,3 +176,21 @@ def test_dsv3_bitplane_decode_full_size_sampled_rows():
                           bits_override=newbits)
     assert_parity(Y2[rows], ref2["Y"], "dsv3 decode after set_bits")
     L.close()
+
+
+@pytest.mark.parametrize("path,T", [(1, 48), (2, 300)])
+def test_top_n_compensation(path, T):
+    """BEAM-style compensation of only the first n routing slots, both paths."""
+    cfg = _cfg(mult=10.0, top_k=3)
+    L, blocks, X, logits, Y = _run(cfg, T, path)
+    L.set_comp_top_n(1)
+    Y1 = L.forward(X, logits, cfg.top_k)
+    assert L.sync_status() == 0
+    ref1 = oracle_forward(cfg, blocks, X, logits, cfg.top_k, comp_top_n=1)
+    assert_parity(Y1, ref1["Y"], "top-n 1")
+    ref = oracle_forward(cfg, blocks, X, logits, cfg.top_k)
+    assert np.max(np.abs(ref1["Y"] - ref["Y"])) > 0.05 * np.max(np.abs(ref["Y"]))
+    L.set_comp_top_n(0)
+    Y0 = L.forward(X, logits, cfg.top_k)
+    assert torch.equal(Y0, Y)
+    L.close()

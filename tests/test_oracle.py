@@ -226,9 +226,10 @@ def test_truncated_svd_eckart_young():
 
 # --------------------------------------------------------------------------- O2 / O6 / O7
 
-def _brute_force(X, L, k, experts, N, renorm=True):
+def _brute_force(X, L, k, experts, N, renorm=True, comp_top_n=0):
     """Every expert on every token, combined with a 0/1 selection mask; the
-    selection uses a stable argsort (no bucketing, no permutation)."""
+    selection uses a stable argsort (no bucketing, no permutation). With
+    comp_top_n > 0 only the experts ranked below n keep their compensators."""
     T = X.shape[0]
     E = L.shape[1]
     Y = np.zeros_like(X, dtype=np.float64)
@@ -236,12 +237,15 @@ def _brute_force(X, L, k, experts, N, renorm=True):
         order = np.argsort(-L[t].astype(np.float64), kind="stable")[:k]
         sel = np.zeros(E, bool)
         sel[order] = True
+        rank = {int(e): j for j, e in enumerate(order)}
         p = np.exp(L[t].astype(np.float64) - L[t].astype(np.float64).max())
         wts = p * sel / ((p * sel).sum() if renorm else p.sum())
         for e in range(E):
             ex = experts[e]
-            o = orc.expert_ffn(X[t:t + 1], ex["W1"], ex["W2"], N, ex.get("A1"), ex.get("B1"),
-                               ex.get("A2"), ex.get("B2"))[0]
+            use = comp_top_n <= 0 or rank.get(e, k) < comp_top_n
+            o = orc.expert_ffn(X[t:t + 1], ex["W1"], ex["W2"], N, ex.get("A1") if use else None,
+                               ex.get("B1") if use else None, ex.get("A2") if use else None,
+                               ex.get("B2") if use else None)[0]
             Y[t] += wts[e] * o
     return Y
 
@@ -275,6 +279,23 @@ def test_brute_force_agrees(k, renorm):
     out = orc.moe_forward(X, L, k, lambda e: experts[e], N, renorm=renorm)
     Yb = _brute_force(X, L, k, experts, N, renorm)
     assert np.max(np.abs(out["Y"] - Yb)) <= 1e-13 * max(1.0, np.max(np.abs(Yb)))
+
+
+@pytest.mark.parametrize("n", [1, 2])
+def test_top_n_compensation_brute_force(n):
+    """Compensators only on the first n routing slots (BEAM abstract)."""
+    E, K, N, T, k = 4, 64, 64, 7, 3
+    experts = _quantized_experts(E, K, N, 3, 32, 8, 51)
+    g = np.random.default_rng(12)
+    X = g.normal(size=(T, K))
+    L = g.normal(size=(T, E)).astype(np.float32)
+    out = orc.moe_forward(X, L, k, lambda e: experts[e], N, comp_top_n=n)
+    Yb = _brute_force(X, L, k, experts, N, comp_top_n=n)
+    assert np.max(np.abs(out["Y"] - Yb)) <= 1e-13 * max(1.0, np.max(np.abs(Yb)))
+    full = orc.moe_forward(X, L, k, lambda e: experts[e], N)["Y"]
+    assert np.max(np.abs(out["Y"] - full)) > 1e-6  # the compensators do matter here
+    same = orc.moe_forward(X, L, k, lambda e: experts[e], N, comp_top_n=k)["Y"]
+    assert np.array_equal(same, full)
 
 
 def test_dense16_rank0_is_dense_matmul():
