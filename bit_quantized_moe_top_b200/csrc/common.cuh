@@ -8,11 +8,12 @@
 //    gate and up values of one SwiGLU column sit 8 rows (8 TMEM lanes) apart.
 //  * Codes are stored per 64-wide K chunk kc and 128-row block rb, chunk-major
 //    ([kc][rb]), so the rows a CTA streams for one chunk are one contiguous
-//    range. Inside a block, row i's 64 codes are "words" in the order one
-//    thread consumes them: step s (0..7) holds pairs j (0..3) of codes
-//    (k = 8s + 2j, 8s + 2j + 1). Words are stored word-quad-major
-//    ([quad][row][16 B]) so that a thread per row reads them conflict-free.
-//    A block holds 128 * 8 * b bytes (b = bits; 16 for dense fp16).
+//    range. Inside a block, row i's 64 codes are two halves of 16 pairs
+//    (k = 32h + 2p, 32h + 2p + 1) packed into the words that the decode
+//    routines consume (field positions in decode_frag.cuh), stored so that
+//    consecutive rows are consecutive 4, 8 or 16-byte units (conflict-free
+//    for a thread per row). A block holds 128 * 8 * b bytes (b = bits; 16
+//    for dense fp16).
 //  * Activations are row-major fp16 [rows, Kpad]: routed rows bucketed per
 //    expert, each expert's range padded to a multiple of 8 rows; the rank
 //    columns U = A x sit after column K.
@@ -31,12 +32,12 @@ constexpr int kMaxExperts = 256;
 enum : int { FMT_INT = 0, FMT_BITPLANE = 1, FMT_DENSE = 2 };
 
 // device status word bits
-enum : unsigned { ST_BOUNDS = 1u, ST_TIMEOUT = 2u, ST_ROUTE = 4u };
+enum : unsigned { ST_BOUNDS = 1u, ST_TIMEOUT = 2u, ST_ROUTE = 4u, ST_RANGE = 8u };
 
 // One expert linear block as the kernels see it.
 struct BlockDesc {
   const uint8_t* codes;   // code blocks [K/64][M/128][block] (INT / DENSE) or plane 0 (BITPLANE)
-  const uint32_t* sz;     // INT: [K/g][M] half2(s, -z*s), internal row order
+  const uint32_t* sz;     // INT: [K/g][M] half2(s, z), internal row order
   const uint32_t* lut;    // BITPLANE: 28 fp16 as 14 u32
   const uint32_t* brow;   // compensator B as fp16 pairs [r/2][M] (column-pair-major)
   const uint4* afrag;     // compensator A [r, K] as mma A-fragments [r/16][K/16][32] uint4 (fp16)
@@ -54,6 +55,14 @@ struct ExpertDesc {
 // ---------------------------------------------------------------------------
 // PTX helpers
 // ---------------------------------------------------------------------------
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while its predecessor finishes; pdl_wait() blocks
+// until every prerequisite grid has completed and its writes are visible (a
+// no-op for a normally serialized launch), pdl_trigger() lets the dependent
+// grid launch once every CTA of this grid has triggered or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -94,6 +103,14 @@ __device__ __forceinline__ uint32_t hfma2u(uint32_t a, uint32_t b, uint32_t c) {
   asm("fma.rn.f16x2 %0, %1, %2, %3;\n" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
+
+__device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;\n" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hneg2u(uint32_t a) { return a ^ 0x80008000u; }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);

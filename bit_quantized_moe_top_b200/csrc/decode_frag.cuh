@@ -1,73 +1,117 @@
-// Register-level unpack + dequantisation of packed codes into fp16 pairs.
-// One thread owns one weight row; a 64-wide K chunk of that row is 8 "steps"
-// of 4 pairs, pair j of step s being the codes at k = 8s+2j and 8s+2j+1.
+// Register-level unpack of packed codes into fp16 pairs.
+//
+// A 64-wide K chunk of one weight row is two halves of 32 codes; half h is
+// 16 pairs, pair i holding the codes at k = 32h + 2i (low 16 bits) and
+// k = 32h + 2i + 1 (high 16 bits). One routine decodes one half, so a row's
+// chunk can be shared by two threads or walked by one.
 //
 // Integer codes become fp16 through the exponent-bias trick: a b-bit field
-// OR-ed into the mantissa of a power of two P whose mantissa ulp is 1 reads as
-// P + q exactly; subtracting P gives q exactly; one fp16 FMA with the group's
-// scale s and the pre-rounded -z*s gives (q - z) * s with one rounding.
-// The field positions inside each 32-bit word are chosen so that no word
-// needs more than one shift per step; see the layout notes in common.cuh.
+// q OR-ed into the mantissa of a power of two P whose mantissa unit at the
+// field's position is 1 reads as P + q exactly. The "raw" value P_i + q is
+// what the tensor-core path multiplies (the P_i term is removed per group
+// through extra K columns); the dequantising path subtracts P_i exactly and
+// applies one fp16 FMA with the group's scale and -z*s. P_i depends only on
+// the pair index i (both halves of a word use the same bit position), so
+// each format has a fixed table of P_i (int_magic) and of P_i / 1024
+// (int_pfac, used to precompute the correction sums).
+//
+// Field positions per format (per 16-bit half of a word; P = 2^(10 - pos)):
+//   INT4: word s (0..3) holds pairs 4s..4s+3: nibbles 0 and 1 of each byte
+//         after a shift of 0 or 8, P = 1024, 64, 1024, 64.
+//   INT2: word u (0..1) holds pairs 8u..8u+7: 2-bit fields at 0,2,4,6 after a
+//         shift of 0 or 8, P = 1024, 256, 64, 16.
+//   INT3: words a, b, c hold pairs 5w..5w+4 as 3-bit fields at 0,3,6 and at
+//         9,12 (read after a shift of 6 as 3,6): P = 1024, 128, 16, 128, 16.
+//         Pair 15 takes its three bits from bit 15 of a (lsb), b and c.
 #pragma once
 #include "common.cuh"
 
 namespace moeq {
 
-// fp16x2 powers of two whose mantissa ulp is 1 for a field at bit 0, 2, 4, 6
-__device__ __forceinline__ uint32_t magic2(int pos) {
-  return pos == 0 ? 0x64006400u : pos == 1 ? 0x5C005C00u : pos == 2 ? 0x54005400u : 0x4C004C00u;
-}
+// ---- integer formats --------------------------------------------------------
 
-// ---- integer formats: produce the exact codes q as fp16x2 (q_k, q_k+1) ----
-
-// INT4: word s of the chunk; slot j lives in nibbles j and j+4.
-__device__ __forceinline__ void int4_codes(uint32_t w, uint32_t (&q)[4]) {
-  const uint32_t w8 = w >> 8;
-  q[0] = hsub2u(lop3_and_or(w, 0x000F000Fu, 0x64006400u), 0x64006400u);
-  q[1] = hsub2u(lop3_and_or(w, 0x00F000F0u, 0x54005400u), 0x54005400u);
-  q[2] = hsub2u(lop3_and_or(w8, 0x000F000Fu, 0x64006400u), 0x64006400u);
-  q[3] = hsub2u(lop3_and_or(w8, 0x00F000F0u, 0x54005400u), 0x54005400u);
-}
-
-// INT2: word s/2 of the chunk; step parity selects the byte half.
-__device__ __forceinline__ void int2_codes(uint32_t w, int s, uint32_t (&q)[4]) {
-  const uint32_t b = (s & 1) ? (w >> 8) : w;
-  q[0] = hsub2u(lop3_and_or(b, 0x00030003u, 0x64006400u), 0x64006400u);
-  q[1] = hsub2u(lop3_and_or(b, 0x000C000Cu, 0x5C005C00u), 0x5C005C00u);
-  q[2] = hsub2u(lop3_and_or(b, 0x00300030u, 0x54005400u), 0x54005400u);
-  q[3] = hsub2u(lop3_and_or(b, 0x00C000C0u, 0x4C004C00u), 0x4C004C00u);
-}
-
-// INT3: low two bits as INT2 (word s/2), the third bit from hi word s/4 after
-// the transform (s & 3): identity, >>1, rotate-right 8, rotate-right 9.
-__device__ __forceinline__ uint32_t int3_hi_transform(uint32_t h, int t) {
-  return t == 0 ? h : t == 1 ? (h >> 1) : t == 2 ? __funnelshift_r(h, h, 8) : __funnelshift_r(h, h, 9);
-}
-__device__ __forceinline__ void int3_codes(uint32_t lo, uint32_t hi, int s, uint32_t (&q)[4]) {
-  const uint32_t b = (s & 1) ? (lo >> 8) : lo;
-  const uint32_t t = int3_hi_transform(hi, s & 3);
-  q[0] = hsub2u(lop3_and_or(lop3_sel(b, t, 0x00030003u), 0x00070007u, 0x64006400u), 0x64006400u);
-  q[1] = hsub2u(lop3_and_or(lop3_sel(b, t, 0x000C000Cu), 0x001C001Cu, 0x5C005C00u), 0x5C005C00u);
-  q[2] = hsub2u(lop3_and_or(lop3_sel(b, t, 0x00300030u), 0x00700070u, 0x54005400u), 0x54005400u);
-  q[3] = hsub2u(lop3_and_or(lop3_sel(b, t, 0x00C000C0u), 0x01C001C0u, 0x4C004C00u), 0x4C004C00u);
-}
-
-// codes of step s (4 fp16x2 pairs) from the row's chunk words (in registers)
-//   INT2: w[0..3]   INT3: w[0..3] lo + w[4..5] hi   INT4: w[0..7]
 template <int BITS>
-__device__ __forceinline__ void int_codes(const uint32_t* w, int s, uint32_t (&q)[4]) {
+__host__ __device__ __forceinline__ uint32_t int_magic(int i) {
+  if (BITS == 4) return (i & 1) ? 0x54005400u : 0x64006400u;
+  if (BITS == 2) {
+    const int j = i & 3;
+    return j == 0 ? 0x64006400u : j == 1 ? 0x5C005C00u : j == 2 ? 0x54005400u : 0x4C004C00u;
+  }
+  if (i == 15) return 0x48004800u;
+  const int f = i % 5;
+  return f == 0 ? 0x64006400u : (f & 1) ? 0x58005800u : 0x4C004C00u;
+}
+
+// P / 1024 of the code at position kk (0..63) of a chunk
+__host__ __device__ __forceinline__ float int_pfac(int bits, int kk) {
+  const int i = (kk >> 1) & 15;
+  if (bits == 4) return (i & 1) ? 0.0625f : 1.f;
+  if (bits == 2) {
+    const int j = i & 3;
+    return j == 0 ? 1.f : j == 1 ? 0.25f : j == 2 ? 0.0625f : 0.015625f;
+  }
+  if (i == 15) return 0.0078125f;
+  const int f = i % 5;
+  return f == 0 ? 1.f : (f & 1) ? 0.125f : 0.015625f;
+}
+
+// number of 32-bit code words per half chunk of one row
+__host__ __device__ __forceinline__ int int_half_words(int bits) { return bits == 4 ? 4 : bits == 3 ? 3 : 2; }
+
+// raw pairs P_i + q of one half chunk from its code words
+//   INT4: w[0..3]   INT3: w[0..2]   INT2: w[0..1]
+template <int BITS>
+__device__ __forceinline__ void int_raw_half(const uint32_t* w, uint32_t (&r)[16]) {
   if constexpr (BITS == 4) {
-    int4_codes(w[s], q);
-  } else if constexpr (BITS == 3) {
-    int3_codes(w[s >> 1], w[4 + (s >> 2)], s, q);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const uint32_t w8 = w[s] >> 8;
+      r[4 * s + 0] = lop3_and_or(w[s], 0x000F000Fu, 0x64006400u);
+      r[4 * s + 1] = lop3_and_or(w[s], 0x00F000F0u, 0x54005400u);
+      r[4 * s + 2] = lop3_and_or(w8, 0x000F000Fu, 0x64006400u);
+      r[4 * s + 3] = lop3_and_or(w8, 0x00F000F0u, 0x54005400u);
+    }
+  } else if constexpr (BITS == 2) {
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const uint32_t b = (s & 1) ? (w[s >> 1] >> 8) : w[s >> 1];
+      r[4 * s + 0] = lop3_and_or(b, 0x00030003u, 0x64006400u);
+      r[4 * s + 1] = lop3_and_or(b, 0x000C000Cu, 0x5C005C00u);
+      r[4 * s + 2] = lop3_and_or(b, 0x00300030u, 0x54005400u);
+      r[4 * s + 3] = lop3_and_or(b, 0x00C000C0u, 0x4C004C00u);
+    }
   } else {
-    int2_codes(w[s >> 1], s, q);
+    uint32_t w6[3];
+#pragma unroll
+    for (int v = 0; v < 3; ++v) {
+      w6[v] = w[v] >> 6;
+      r[5 * v + 0] = lop3_and_or(w[v], 0x00070007u, 0x64006400u);
+      r[5 * v + 1] = lop3_and_or(w[v], 0x00380038u, 0x58005800u);
+      r[5 * v + 2] = lop3_and_or(w[v], 0x01C001C0u, 0x4C004C00u);
+      r[5 * v + 3] = lop3_and_or(w6[v], 0x00380038u, 0x58005800u);
+      r[5 * v + 4] = lop3_and_or(w6[v], 0x01C001C0u, 0x4C004C00u);
+    }
+    // pair 15: bit 15 of a -> bit 7, of b -> bit 8, of c -> bit 9 (each half)
+    const uint32_t t = lop3_sel(w[0] >> 8, w[1] >> 7, 0x00800080u);
+    const uint32_t t2 = lop3_sel(t, w6[2], 0x01800180u);
+    r[15] = lop3_and_or(t2, 0x03800380u, 0x48004800u);
   }
 }
 
-// ---- bit-plane + LUT: 4-bit layout per plane word: bit 4*(2j+h) + (s&3) of
-// word s>>2 is element (step s, slot j, half h).  Codes are built as prmt
-// nibble selectors; the LUT is split in a low-byte and a high-byte table. ----
+// (q - z) * s of one half: raw - P exactly, then one fp16 FMA with
+// s2 = (s, s) and n2 = (-z*s, -z*s)
+template <int BITS>
+__device__ __forceinline__ void int_dequant_half(const uint32_t (&raw)[16], uint32_t s2, uint32_t n2,
+                                                 uint32_t (&out)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) out[i] = hfma2u(hsub2u(raw[i], int_magic<BITS>(i)), s2, n2);
+}
+
+// ---- bit-plane + LUT ---------------------------------------------------------
+// Per plane, a half chunk is one 32-bit word: bit 4*(2j+h) + s of it is the
+// plane bit of element (step s, slot j, half h), step s = 0..3 covering pairs
+// 4s..4s+3. Codes are built as prmt nibble selectors; the LUT is split in a
+// low-byte and a high-byte table.
 
 struct LutRegs {
   // low / high bytes of LUT entries 0..7 (a) and 8..15 (b, 4-bit only)
@@ -101,24 +145,20 @@ __device__ __forceinline__ LutRegs load_lut(const uint32_t* lut28, int bits) {
   return r;
 }
 
-// b-bit code nibbles of step s (8 elements: nibble 2j+h) from the plane words
-// of word s>>2; bit 3 of every nibble is left 0 (b<=3) or holds the MSB (b=4).
+// b-bit code nibbles of step s (8 elements: nibble 2j+h) from the half's
+// plane words pw[p] (p = 0 is the MSB plane); bit 3 of every nibble is 0
+// (b <= 3) or holds the MSB (b = 4).
 template <int BITS>
 __device__ __forceinline__ uint32_t plane_codes(const uint32_t* pw, int s) {
-  const int q = s & 3;
-  const int w = s >> 2;
   uint32_t c = 0;
 #pragma unroll
-  for (int p = 0; p < BITS; ++p) {
-    const uint32_t bit = (pw[2 * p + w] >> q) & 0x11111111u;
-    c |= bit << (BITS - 1 - p);
-  }
+  for (int p = 0; p < BITS; ++p) c |= ((pw[p] >> s) & 0x11111111u) << (BITS - 1 - p);
   return c;
 }
 
-// LUT lookup of the 8 codes of step s: out[j] = (LUT[c(j,0)], LUT[c(j,1)])
+// LUT lookup of the 8 codes of one step: a[j] = (LUT[c(j,0)], LUT[c(j,1)])
 template <int BITS>
-__device__ __forceinline__ void lut_decode(uint32_t codes, const LutRegs& L, uint32_t (&a)[4]) {
+__device__ __forceinline__ void lut_decode(uint32_t codes, const LutRegs& L, uint32_t* a) {
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     const uint32_t sel = half ? (codes >> 16) : (codes & 0xFFFFu);
@@ -138,54 +178,71 @@ __device__ __forceinline__ void lut_decode(uint32_t codes, const LutRegs& L, uin
   }
 }
 
-// ---- whole 64-wide chunk of one row ----
-
-// words of row `row` of a [128-row] code block (global or shared memory)
-__device__ __forceinline__ void load_row_words_int(const uint8_t* blk, int row, int bits, uint32_t (&w)[8]) {
-  const uint4 v0 = reinterpret_cast<const uint4*>(blk)[row];
-  w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-  w[4] = w[5] = w[6] = w[7] = 0u;
-  if (bits == 4) {
-    const uint4 v1 = reinterpret_cast<const uint4*>(blk + 2048)[row];
-    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
-  } else if (bits == 3) {
-    const uint2 h = reinterpret_cast<const uint2*>(blk + 2048)[row];
-    w[4] = h.x; w[5] = h.y;
-  }
-}
-
-// bit-plane words of row `row`: plane p at blk + p * plane_bytes
+// LUT values of one half from its plane words pw[0..BITS-1]
 template <int BITS>
-__device__ __forceinline__ void load_row_planes(const uint8_t* blk, int plane_bytes, int row, uint32_t (&w)[8]) {
+__device__ __forceinline__ void lut_half(const uint32_t* pw, const LutRegs& L, uint32_t (&out)[16]) {
 #pragma unroll
-  for (int p = 0; p < BITS; ++p) {
-    const uint2 v = reinterpret_cast<const uint2*>(blk + p * plane_bytes)[row];
-    w[2 * p] = v.x; w[2 * p + 1] = v.y;
+  for (int s = 0; s < 4; ++s) lut_decode<BITS>(plane_codes<BITS>(pw, s), L, out + 4 * s);
+}
+
+// ---- code blocks in memory (global or shared) --------------------------------
+// INT4: words 0..3 of all rows ([128] x 16 B), then words 4..7.
+// INT2: words 0..3 of all rows ([128] x 16 B).
+// INT3: word-major, [6][128] x 4 B.
+// BITPLANE: per plane [128] x 8 B (word 0 = half 0), planes plane_bytes apart.
+
+// half h's code words of row `row`
+template <int BITS>
+__device__ __forceinline__ void load_half_words_int(const uint8_t* blk, int row, int h, uint32_t (&w)[4]) {
+  if constexpr (BITS == 4) {
+    const uint4 v = reinterpret_cast<const uint4*>(blk + 2048 * h)[row];
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (BITS == 2) {
+    const uint2 v = reinterpret_cast<const uint2*>(blk + 16 * row + 8 * h)[0];
+    w[0] = v.x; w[1] = v.y; w[2] = w[3] = 0u;
+  } else {
+    const uint32_t* b32 = reinterpret_cast<const uint32_t*>(blk);
+    w[0] = b32[(3 * h + 0) * 128 + row];
+    w[1] = b32[(3 * h + 1) * 128 + row];
+    w[2] = b32[(3 * h + 2) * 128 + row];
+    w[3] = 0u;
   }
 }
 
-// 32 fp16 pairs (k = 0..63) of one row chunk: out[4s+j] = pair (8s+2j, 8s+2j+1)
-// INT: w^ = (q - z) * s with sz = half2(s, -z*s); bit-plane: LUT_b[code].
+template <int BITS>
+__device__ __forceinline__ void load_half_planes(const uint8_t* blk, int plane_bytes, int row, int h,
+                                                 uint32_t (&pw)[4]) {
+#pragma unroll
+  for (int p = 0; p < 4; ++p)
+    pw[p] = p < BITS ? reinterpret_cast<const uint32_t*>(blk + p * plane_bytes)[2 * row + h] : 0u;
+}
+
+// 32 dequantised fp16 pairs (k = 0..63) of one row chunk: out[16h + i] = pair i of half h
+// INT: (q - z) * s with sz = half2(s, z); bit-plane: LUT_b[code].
 template <int FMT, int BITS>
-__device__ __forceinline__ void decode_row64(const uint32_t (&w)[8], uint32_t sz, const LutRegs& lut,
-                                             uint32_t (&out)[32]) {
+__device__ __forceinline__ void decode_row64(const uint8_t* blk, int plane_bytes, int row, uint32_t sz,
+                                             const LutRegs& lut, uint32_t (&out)[32]) {
+  uint32_t s2 = 0, n2 = 0;
   if constexpr (FMT == FMT_INT) {
-    const uint32_t s2 = prmt(sz, sz, 0x1010u), n2 = prmt(sz, sz, 0x3232u);
+    s2 = prmt(sz, sz, 0x1010u);
+    const uint32_t z2 = prmt(sz, sz, 0x3232u);
+    n2 = hmul2u(hneg2u(z2), s2);
+  }
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      uint32_t q[4];
-      int_codes<BITS>(w, s, q);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) out[4 * s + j] = hfma2u(q[j], s2, n2);
+  for (int h = 0; h < 2; ++h) {
+    uint32_t v[16];
+    if constexpr (FMT == FMT_INT) {
+      uint32_t w[4], raw[16];
+      load_half_words_int<BITS>(blk, row, h, w);
+      int_raw_half<BITS>(w, raw);
+      int_dequant_half<BITS>(raw, s2, n2, v);
+    } else {
+      uint32_t pw[4];
+      load_half_planes<BITS>(blk, plane_bytes, row, h, pw);
+      lut_half<BITS>(pw, lut, v);
     }
-  } else {
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      uint32_t av[4];
-      lut_decode<BITS>(plane_codes<BITS>(w, s), lut, av);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) out[4 * s + j] = av[j];
-    }
+    for (int i = 0; i < 16; ++i) out[16 * h + i] = v[i];
   }
 }
 

@@ -1,84 +1,129 @@
 // Grouped expert GEMM for small per-expert batches (the decode path), on the
-// 5th-generation tensor cores with the dequantised weights in TMEM.
+// 5th-generation tensor cores with the unpacked weights in TMEM.
 //
 // The decode matmuls stream weights: every packed code is read once per
 // token pass, so the kernel is bound by HBM bandwidth and by the ALU work of
-// unpacking. One CTA owns 128 weight rows of one expert (one row per TMEM
-// lane) and a range of 64-wide K chunks:
-//   warp 4     producer: per chunk, the 128 rows' packed codes (one contiguous
-//              block), their scales, and the expert's routed activation rows
-//              (TMA 2-D boxes of 16 rows, 128-byte swizzle, no multicast);
-//   warps 0-3  one thread per weight row unpacks and dequantises the row's 64
-//              codes in registers to fp16 and stores them into a TMEM buffer
-//              (tcgen05.st) that is the A operand of the MMA;
-//   warp 5     allocates TMEM and issues tcgen05.mma kind::f16 with A from
+// unpacking. A CTA owns 128 weight rows of one expert (one row per TMEM
+// lane) and a group-aligned range of 64-wide K chunks; CTAs are persistent
+// and walk the (expert, row block, K split) tiles round-robin.
+//   warp 8     producer: per chunk, the 128 rows' packed codes (one contiguous
+//              block), at a group's first chunk its scales and zero points
+//              and the routed rows' correction columns, and the expert's
+//              routed activation rows (TMA 2-D boxes of 16 rows, no multicast);
+//   warps 0-7  two threads per weight row (warps w and w+4 share TMEM lane
+//              quarter w, one K half each) unpack the codes in registers and
+//              store them into a TMEM buffer (tcgen05.st), the MMA's A operand;
+//   warp 9     allocates TMEM and issues tcgen05.mma kind::f16 with A from
 //              TMEM (M = 128 weight rows), B = activations from shared memory
-//              (N = tokens, 16..128), D accumulated in TMEM.
-// No accumulator lives in registers, so several CTAs share an SM. The rank-r
-// compensator is one more 64-wide stage: the B factor's row values as A
-// against the U = A x columns stored after the activations' K (MiLo abstract:
-// low-rank compensators of the quantised experts; TileQ abstract: low-rank
-// terms in the same pass as the quantised GEMM).
+//              (N = tokens, 16..64), D in TMEM.
 //
-// Epilogues (warps 0-3, tcgen05.ld): SwiGLU of the gate/up rows 8 lanes apart
-// (W1, fp16 rows of the down projection's input), or fp32 partial outputs per
-// K split (W2, summed by the combine kernel in a fixed order). Every wait is
-// bounded; a timeout sets the status word and the CTA unwinds.
+// Integer codes are not dequantised per weight. The A operand holds the raw
+// fp16 values P_k + q_k of the exponent-bias unpack (exact small integers
+// offset by a per-position power of two), and each quantisation group g gets
+// its own accumulator:
+//   acc_g = sum_{k in g} (P_k + q_k) x_k + 1024 (-XP_g) + z_g (-X_g)
+//         = sum_{k in g} (q_k - z_g) x_k,
+// the two extra terms being one more K = 16 MMA step per group whose A
+// columns are (1024, 1024, z_g, z_g, 0...) and whose B columns are the
+// routed row's precomputed sums XP_g = sum (P_k/1024) x_k and X_g = sum x_k,
+// each split into fp16 value + fp16 remainder. The epilogue of a group is
+// y += s_g * acc_g in fp32 registers (two threads per row, one half of the
+// tokens each). Per pair of weights this leaves one or two logic ops and no
+// fp16 arithmetic. Bit-plane (LUT) and dense blocks store their fp16 weight
+// values as A and use one accumulator for the whole K range.
+//
+// The rank-r compensator is one more 64-wide stage (its own accumulator,
+// scale 1): the B factor's row values as A against the U = A x columns stored
+// after the activations' K (MiLo abstract: low-rank compensators of the
+// quantised experts; TileQ abstract: low-rank terms in the same pass as the
+// quantised GEMM).
+//
+// Outputs: SwiGLU of the gate/up rows 8 lanes apart (W1, fp16 rows of the
+// down projection's input), or fp32 partial outputs per K split (W2, summed
+// by the combine kernel in a fixed order). Every wait is bounded; a timeout
+// sets the status word and the CTA unwinds.
+#include <algorithm>
+
 #include "kernels.h"
 #include "decode_frag.cuh"
 #include "tc.cuh"
+#include "corr.cuh"
 
 namespace moeq {
 namespace dk {
 
-constexpr int kThreads = 192;
+constexpr int kDqWarps = 8;
+constexpr int kThreads = 32 * (kDqWarps + 2);
 constexpr int kRows = 128;
 constexpr int kStages = 4;
 constexpr int kABufs = 2;
-constexpr int kActBox = 16;  // rows per TMA box
+constexpr int kACols = 40;        // per A buffer: 32 code columns + 8 correction columns
+constexpr int kActBox = 16;       // rows per TMA box
+constexpr int kTmemCols = 256;    // accumulators at [0, 2 NTOK), A buffers at [128, 208)
+constexpr int kABase = 128;
+constexpr uint32_t kOne1024 = 0x64006400u;  // fp16 pair (1024, 1024)
 
 __host__ __device__ inline int code_bytes(int maxbits) { return maxbits >= 16 ? 16384 : 4096; }
+// stage: [act NTOK x 128 B][corr NTOK x 32 B][codes][scales 512 B]
 __host__ __device__ inline int stage_bytes(int ntok, int maxbits) {
-  const int b = ntok * 128 + code_bytes(maxbits) + 512;
+  const int b = ntok * 160 + code_bytes(maxbits) + 512;
   return (b + 1023) & ~1023;
-}
-__host__ __device__ inline int tmem_cols(int ntok) {
-  const int need = ntok + kABufs * 32;
-  return need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
 }
 
 struct Ctx {
-  int n_e, prow0, rb, ks, kc0, nmain, next, npass, cbytes;
+  int n_e, prow0, rb, ks, kc0, nmain, next, npass;
+};
+struct Cnt {
+  int it = 0;  // chunk (stage and A buffer) counter
+  int gc = 0;  // accumulator group counter
 };
 
+// group position of chunk i of a pass: first / last chunk of its accumulator group
+template <int FMT, int GROUP>
+__device__ __forceinline__ void group_pos(const Ctx& c, int i, bool& first, bool& last) {
+  if (i >= c.nmain) {
+    first = last = true;  // compensator stage
+  } else if (FMT == FMT_INT) {
+    constexpr int cpg = GROUP / 64;
+    first = (i % cpg) == 0;
+    last = (i % cpg) == cpg - 1;
+  } else {
+    first = i == 0;
+    last = i == c.nmain - 1;
+  }
+}
+
 template <int NTOK, int FMT, int BITS, int GROUP>
-__device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, uint8_t* sm, int stage_b,
-                         uint32_t bars, volatile int* abort_flag) {
+__device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, uint8_t* sm, int stage_b, int cbytes,
+                         uint32_t bars, Cnt& cnt, volatile int* abort_flag) {
   const uint32_t full = bars, empty = bars + 8 * kStages;
   const int RB = a.M / kRows;
   constexpr int kBlk = (FMT == FMT_DENSE) ? 16384 : 128 * 8 * BITS;  // bytes of one code block (per plane: 1 KiB)
-  int it = 0, issued = 0;
   for (int p = 0; p < c.npass && !*abort_flag; ++p) {
     const int n_pass = min(NTOK, c.n_e - p * NTOK);
     const int nbox = (n_pass + kActBox - 1) / kActBox;
-    for (int i = 0; i < c.nmain + c.next; ++i, ++it) {
-      const int slot = it % kStages;
-      if (*abort_flag || (it >= kStages && !mbar_wait(empty + 8 * slot, ((it / kStages) & 1) ^ 1, a.status))) {
+    const int row0 = c.prow0 + p * NTOK;
+    for (int i = 0; i < c.nmain + c.next; ++i, ++cnt.it) {
+      const int slot = cnt.it % kStages;
+      if (*abort_flag || !mbar_wait(empty + 8 * slot, ((cnt.it / kStages) & 1) ^ 1, a.status)) {
         *abort_flag = 1;
-        break;
+        return;
       }
+      bool first, last;
+      group_pos<FMT, GROUP>(c, i, first, last);
       uint8_t* st = sm + slot * stage_b;
       const bool main = i < c.nmain;
       const int kc = c.kc0 + i;
+      const bool corr = FMT == FMT_INT && main && first;
       uint32_t bytes = nbox * kActBox * 128;
-      if (main) bytes += kBlk + (FMT == FMT_INT ? 512 : 0);
+      if (main) bytes += (FMT == FMT_BITPLANE ? BITS * 1024 : kBlk);
+      if (corr) bytes += nbox * kActBox * 32 + 512;
       mbar_expect_tx(full + 8 * slot, bytes);
       const int kx = main ? kc * 64 : a.K;
       for (int b = 0; b < nbox; ++b)
-        tma_load_2d(smem_u32(st + b * kActBox * 128), &a.tmap_act, kx, c.prow0 + p * NTOK + b * kActBox,
-                    full + 8 * slot);
+        tma_load_2d(smem_u32(st + b * kActBox * 128), &a.tmap_act, kx, row0 + b * kActBox, full + 8 * slot);
       if (main) {
-        uint8_t* cs = st + NTOK * 128;
+        uint8_t* cs = st + NTOK * 160;
         const long long bidx = (long long)kc * RB + c.rb;
         if constexpr (FMT == FMT_BITPLANE) {
 #pragma unroll
@@ -87,260 +132,377 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
         } else {
           bulk_g2s(smem_u32(cs), d.codes + bidx * kBlk, kBlk, full + 8 * slot);
         }
-        if constexpr (FMT == FMT_INT)
-          bulk_g2s(smem_u32(cs + c.cbytes), d.sz + (long long)(kc * 64 / GROUP) * a.M + c.rb * kRows, 512,
-                   full + 8 * slot);
+        if (corr) {
+          const int g = kc * 64 / GROUP;
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(smem_u32(st + NTOK * 128 + b * kActBox * 32), &a.tmap_corr, 16 * g, row0 + b * kActBox,
+                        full + 8 * slot);
+          bulk_g2s(smem_u32(cs + cbytes), d.sz + (long long)g * a.M + c.rb * kRows, 512, full + 8 * slot);
+        }
       }
-      ++issued;
     }
   }
-  // drain: every issued stage must land before the CTA may exit
-  for (int k = max(0, issued - kStages); k < issued; ++k)
-    if (!mbar_wait(full + 8 * (k % kStages), (k / kStages) & 1, a.status)) break;
 }
 
-template <int NTOK>
-__device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int stage_b, uint32_t bars,
-                           uint32_t tmem, volatile int* abort_flag) {
+// every issued stage must land before the CTA may exit
+__device__ void producer_drain(const DecodeArgs& a, uint32_t bars, const Cnt& cnt) {
+  for (int k = max(0, cnt.it - kStages); k < cnt.it; ++k)
+    if (!mbar_wait(bars + 8 * (k % kStages), (k / kStages) & 1, a.status)) break;
+}
+
+template <int NTOK, int FMT, int GROUP>
+__device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int stage_b, uint32_t bars, uint32_t tmem,
+                           Cnt& cnt, volatile int* abort_flag) {
   const uint32_t full = bars, empty = bars + 8 * kStages;
   const uint32_t afull = bars + 16 * kStages, aempty = afull + 8 * kABufs;
-  const uint32_t accfull = aempty + 8 * kABufs, dfree = accfull + 8;
-  int it = 0;
+  const uint32_t accfull = aempty + 8 * kABufs, accfree = accfull + 16;
   for (int p = 0; p < c.npass; ++p) {
     const int n_pass = min(NTOK, c.n_e - p * NTOK);
     const int npad = (n_pass + 15) & ~15;
     const uint32_t idesc = idesc_f16(128, npad);
-    if (p > 0 && !mbar_wait(dfree, (p - 1) & 1, a.status)) {  // previous pass's epilogue is done with D
-      *abort_flag = 1;
-      break;
-    }
-    bool ok = true;
-    for (int i = 0; i < c.nmain + c.next; ++i, ++it) {
-      const int slot = it % kStages, buf = it % kABufs;
-      if (*abort_flag || !mbar_wait(full + 8 * slot, (it / kStages) & 1, a.status) ||
-          !mbar_wait(afull + 8 * buf, (it / kABufs) & 1, a.status)) {
-        ok = false;
-        break;
+    for (int i = 0; i < c.nmain + c.next; ++i, ++cnt.it) {
+      const int slot = cnt.it % kStages, buf = cnt.it % kABufs;
+      bool first, last;
+      group_pos<FMT, GROUP>(c, i, first, last);
+      const int ab = cnt.gc & 1;
+      if (*abort_flag || !mbar_wait(full + 8 * slot, (cnt.it / kStages) & 1, a.status) ||
+          !mbar_wait(afull + 8 * buf, (cnt.it / kABufs) & 1, a.status) ||
+          (first && !mbar_wait(accfree + 8 * ab, ((cnt.gc >> 1) & 1) ^ 1, a.status))) {
+        *abort_flag = 1;
+        return;
       }
       tc_fence_after();
       const uint32_t bt = smem_u32(sm + slot * stage_b);
+      const uint32_t acc = tmem + ab * NTOK;
+      const uint32_t ta = tmem + kABase + buf * kACols;
+      const bool corr = FMT == FMT_INT && i < c.nmain && first;
+      if (corr) mma_f16_ts(acc, ta + 32, sw32_desc(bt + NTOK * 128), idesc, 0);
 #pragma unroll
       for (int k16 = 0; k16 < 4; ++k16)
-        mma_f16_ts(tmem, tmem + NTOK + buf * 32 + k16 * 8, sw128_desc(bt + k16 * 32), idesc, (i > 0 || k16 > 0));
+        mma_f16_ts(acc, ta + k16 * 8, sw128_desc(bt + k16 * 32), idesc, (corr || !first || k16 > 0) ? 1 : 0);
       mma_commit(empty + 8 * slot);
       mma_commit(aempty + 8 * buf);
-    }
-    mma_commit(accfull);
-    if (!ok) {
-      *abort_flag = 1;
-      break;
+      if (last) {
+        mma_commit(accfull + 8 * ab);
+        ++cnt.gc;
+      }
     }
   }
 }
 
-template <int NTOK, int FMT, int BITS>
+// y[t] += scale * acc[t] for this thread's half of the tokens of group gq
+template <int NTOK>
+__device__ __forceinline__ bool group_epilogue(const DecodeArgs& a, uint32_t bars, uint32_t tmem, uint32_t lane_base,
+                                               int h, int gq, float scale, float (&y)[NTOK / 2]) {
+  const uint32_t accfull = bars + 16 * kStages + 16 * kABufs, accfree = accfull + 16;
+  const int ab = gq & 1;
+  if (!__all_sync(0xffffffffu, mbar_wait(accfull + 8 * ab, (gq >> 1) & 1, a.status))) return false;
+  tc_fence_after();
+  uint32_t v[NTOK / 2];
+  tmem_ld<NTOK / 2>(tmem + lane_base + ab * NTOK + h * (NTOK / 2), v);
+#pragma unroll
+  for (int t = 0; t < NTOK / 2; ++t) y[t] = fmaf(scale, __uint_as_float(v[t]), y[t]);
+  tc_fence_before();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(accfree + 8 * ab);
+  return true;
+}
+
+template <int NTOK, int FMT, int BITS, int GROUP>
 __device__ void dequant_epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, uint8_t* sm, int stage_b,
-                                 uint32_t bars, uint32_t tmem, volatile int* abort_flag) {
+                                 int cbytes, uint32_t bars, uint32_t tmem, Cnt& cnt, volatile int* abort_flag) {
   const uint32_t full = bars, empty = bars + 8 * kStages;
   const uint32_t afull = bars + 16 * kStages, aempty = afull + 8 * kABufs;
-  const uint32_t accfull = aempty + 8 * kABufs, dfree = accfull + 8;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = threadIdx.x;       // 0..127 = TMEM lane
-  const int R = c.rb * kRows + row;  // internal row of the block
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const int q = warp & 3, h = warp >> 2;      // TMEM lane quarter, K half / token half
+  const int row = q * 32 + lane;              // TMEM lane
+  const int R = c.rb * kRows + row;           // internal row of the block
+  const uint32_t lane_base = (uint32_t)(q * 32) << 16;
   LutRegs lut;
   if constexpr (FMT == FMT_BITPLANE) lut = load_lut(d.lut, BITS);
   const int RS2 = d.rank / 2;  // compensator column pairs
-  int it = 0;
+  constexpr int NH = NTOK / 2;
   for (int p = 0; p < c.npass; ++p) {
     const int n_pass = min(NTOK, c.n_e - p * NTOK);
-    const int npad = (n_pass + 15) & ~15;
-    for (int i = 0; i < c.nmain + c.next; ++i, ++it) {
-      const int slot = it % kStages, buf = it % kABufs;
-      if (*abort_flag || !mbar_wait(full + 8 * slot, (it / kStages) & 1, a.status) ||
-          !mbar_wait(aempty + 8 * buf, ((it / kABufs) & 1) ^ 1, a.status)) {
+    float y[NH];
+#pragma unroll
+    for (int t = 0; t < NH; ++t) y[t] = 0.f;
+    int pending = -1;        // group whose epilogue is deferred by one chunk
+    float pend_scale = 1.f;
+    float s_cur = 1.f;
+    for (int i = 0; i < c.nmain + c.next; ++i, ++cnt.it) {
+      const int slot = cnt.it % kStages, buf = cnt.it % kABufs;
+      bool first, last;
+      group_pos<FMT, GROUP>(c, i, first, last);
+      // warp-uniform waits: every lane must reach the .sync.aligned TMEM stores
+      const bool ok = !*abort_flag && mbar_wait(full + 8 * slot, (cnt.it / kStages) & 1, a.status) &&
+                      mbar_wait(aempty + 8 * buf, ((cnt.it / kABufs) & 1) ^ 1, a.status);
+      if (!__all_sync(0xffffffffu, ok)) {
         *abort_flag = 1;
         return;
       }
-      uint32_t v[32];
-      if (i < c.nmain) {
-        const uint8_t* cs = sm + slot * stage_b + NTOK * 128;
-        if constexpr (FMT == FMT_DENSE) {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint4 x = reinterpret_cast<const uint4*>(cs + q * 2048)[row];
-            v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+      const uint32_t ta = tmem + lane_base + kABase + buf * kACols;
+      uint32_t v[16];
+      const bool main = i < c.nmain;
+      if (main) {
+        const uint8_t* cs = sm + slot * stage_b + NTOK * 160;
+        if constexpr (FMT == FMT_INT) {
+          if (first) {
+            const uint32_t sz = reinterpret_cast<const uint32_t*>(cs + cbytes)[row];
+            s_cur = __half2float(__ushort_as_half((uint16_t)(sz & 0xFFFFu)));
+            if (h == 0) tmem_st1_nw(ta + 33, prmt(sz, sz, 0x3232u));  // (z, z) against (-X_hi, -X_lo)
           }
+          uint32_t w[4];
+          load_half_words_int<BITS>(cs, row, h, w);
+          int_raw_half<BITS>(w, v);
+        } else if constexpr (FMT == FMT_BITPLANE) {
+          uint32_t pw[4];
+          load_half_planes<BITS>(cs, 1024, row, h, pw);
+          lut_half<BITS>(pw, lut, v);
         } else {
-          uint32_t w[8];
-          uint32_t sz = 0;
-          if constexpr (FMT == FMT_INT) {
-            load_row_words_int(cs, row, BITS, w);
-            sz = reinterpret_cast<const uint32_t*>(cs + c.cbytes)[row];
-          } else {
-            load_row_planes<BITS>(cs, 1024, row, w);
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) {
+            const uint4 x = reinterpret_cast<const uint4*>(cs + (4 * h + qd) * 2048)[row];
+            v[4 * qd] = x.x; v[4 * qd + 1] = x.y; v[4 * qd + 2] = x.z; v[4 * qd + 3] = x.w;
           }
-          decode_row64<FMT, BITS>(w, sz, lut, v);
         }
       } else {
         // compensator stage: the row's B values (pairs), zero past the rank
 #pragma unroll
-        for (int q = 0; q < 32; ++q) v[q] = q < RS2 ? d.brow[(long long)q * a.M + R] : 0u;
+        for (int j = 0; j < 16; ++j) v[j] = (16 * h + j) < RS2 ? d.brow[(long long)(16 * h + j) * a.M + R] : 0u;
       }
-      tmem_st32(tmem + lane_base + NTOK + buf * 32, v);
+      tmem_st16_nw(ta + 16 * h, v);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(afull + 8 * buf);
         mbar_arrive(empty + 8 * slot);
       }
+      // the previous group's accumulator, while this chunk's MMAs queue
+      if (pending >= 0) {
+        if (!group_epilogue<NTOK>(a, bars, tmem, lane_base, h, pending, pend_scale, y)) {
+          *abort_flag = 1;
+          return;
+        }
+        pending = -1;
+      }
+      if (last) {
+        pending = cnt.gc++;
+        pend_scale = (FMT == FMT_INT && main) ? s_cur : 1.f;
+      }
     }
-    // ---- epilogue of pass p
-    if (!mbar_wait(accfull, p & 1, a.status)) {
+    if (pending >= 0 && !group_epilogue<NTOK>(a, bars, tmem, lane_base, h, pending, pend_scale, y)) {
       *abort_flag = 1;
       return;
     }
-    tc_fence_after();
-    const int tok0 = p * NTOK;
-    for (int cb = 0; cb < npad / 16; ++cb) {
-      uint32_t acc[16];
-      tmem_ld16(tmem + lane_base + cb * 16, acc);
-      if (a.mode == MODE_SWIGLU) {
-        // gate rows are lanes 16f..16f+7 of each 16-row group, up rows 8 lanes later
-        float up[16];
+    // ---- outputs of pass p: tokens p*NTOK + h*NH + t
+    const int tok0 = p * NTOK + h * NH;
+    const int nt = n_pass - h * NH;  // valid tokens of this half
+    if (a.mode == MODE_SWIGLU) {
+      // gate rows are lanes 16f..16f+7 of each 16-row group, up rows 8 lanes later
+      float up[NH];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) up[t] = __shfl_down_sync(0xffffffffu, __uint_as_float(acc[t]), 8);
-        if ((R & 15) < 8) {
-          const int col = 8 * (R >> 4) + (R & 7);
+      for (int t = 0; t < NH; ++t) up[t] = __shfl_down_sync(0xffffffffu, y[t], 8);
+      if ((R & 15) < 8) {
+        const int col = 8 * (R >> 4) + (R & 7);
 #pragma unroll
-          for (int t = 0; t < 16; ++t) {
-            const int n = cb * 16 + t;
-            if (n < n_pass) {
-              const float gt = __uint_as_float(acc[t]);
-              a.zout[(long long)(c.prow0 + tok0 + n) * a.ldz + col] = __float2half_rn(gt / (1.f + expf(-gt)) * up[t]);
-            }
+        for (int t = 0; t < NH; ++t) {
+          if (t < nt) {
+            const float gt = y[t];
+            a.zout[(long long)(c.prow0 + tok0 + t) * a.ldz + col] = __float2half_rn(gt / (1.f + expf(-gt)) * up[t]);
           }
         }
-      } else {
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const int n = cb * 16 + t;
-          if (n < n_pass)
-            a.out[c.ks * a.out_ks_stride + (long long)(c.prow0 + tok0 + n) * a.M + R] = __uint_as_float(acc[t]);
-        }
       }
+    } else {
+#pragma unroll
+      for (int t = 0; t < NH; ++t)
+        if (t < nt) a.out[c.ks * a.out_ks_stride + (long long)(c.prow0 + tok0 + t) * a.M + R] = y[t];
     }
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(dfree);
+  }
+}
+
+template <int NTOK, int FMT, int BITS, int GROUP>
+__device__ void decode_tile(const DecodeArgs& a, const BlockDesc& d, const Ctx& c0, uint8_t* sm, int stage_b,
+                            int cbytes, uint32_t bars, uint32_t tmem, Cnt& cnt, volatile int* ab) {
+  // group-aligned K range of this split
+  Ctx c = c0;
+  const int KC = a.K / 64;
+  if constexpr (FMT == FMT_INT) {
+    constexpr int cpg = GROUP / 64;
+    const int NG = KC / cpg;
+    const int g0 = (int)((long long)NG * c.ks / a.KS), g1 = (int)((long long)NG * (c.ks + 1) / a.KS);
+    c.kc0 = g0 * cpg;
+    c.nmain = (g1 - g0) * cpg;
+  } else {
+    c.kc0 = (int)((long long)KC * c.ks / a.KS);
+    c.nmain = (int)((long long)KC * (c.ks + 1) / a.KS) - c.kc0;
+  }
+  const int warp = threadIdx.x >> 5;
+  if (warp < kDqWarps) {
+    dequant_epilogue<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, tmem, cnt, ab);
+  } else if (warp == kDqWarps) {
+    if ((threadIdx.x & 31) == 0) producer<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, cnt, ab);
+  } else {
+    if ((threadIdx.x & 31) == 0) mma_issuer<NTOK, FMT, GROUP>(a, c, sm, stage_b, bars, tmem, cnt, ab);
   }
 }
 
 }  // namespace dk
 
-template <int NTOK, int FMT, int BITS, int GROUP>
-__device__ void decode_tile(const DecodeArgs& a, const BlockDesc& d, const dk::Ctx& c, uint8_t* sm, int stage_b,
-                            uint32_t bars, uint32_t tmem, volatile int* ab) {
-  const int warp = threadIdx.x >> 5;
-  if (warp < 4) {
-    dk::dequant_epilogue<NTOK, FMT, BITS>(a, d, c, sm, stage_b, bars, tmem, ab);
-  } else if (warp == 4) {
-    if ((threadIdx.x & 31) == 0) dk::producer<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, bars, ab);
-  } else {
-    if ((threadIdx.x & 31) == 0) dk::mma_issuer<NTOK>(a, c, sm, stage_b, bars, tmem, ab);
-  }
-}
-
 template <int NTOK>
-__global__ void __launch_bounds__(dk::kThreads, 1) decode_gemm_kernel(const __grid_constant__ DecodeArgs a,
+__global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __grid_constant__ DecodeArgs a,
                                                                         int stage_b, int cbytes) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) unsigned long long bars[2 * dk::kStages + 2 * dk::kABufs + 2];
+  // full, empty [stages]; afull, aempty [A bufs]; accfull, accfree [2]; done
+  __shared__ __align__(8) unsigned long long bars[2 * dk::kStages + 2 * dk::kABufs + 5];
   __shared__ int abort_flag;
   __shared__ uint32_t tmem_slot;
-  const int slot = blockIdx.y;
-  if (slot >= *a.n_active) return;
-  const int e = a.active[slot];
-  dk::Ctx c;
-  c.n_e = a.counts[e];
-  if (c.n_e <= 0) return;
-  c.prow0 = a.poffsets[e];
-  c.rb = blockIdx.x / a.KS;
-  c.ks = blockIdx.x % a.KS;
-  const int KC = a.K / 64;
-  c.kc0 = (int)((long long)KC * c.ks / a.KS);
-  c.nmain = (int)((long long)KC * (c.ks + 1) / a.KS) - c.kc0;
-  const BlockDesc d = a.experts[e].blk[a.block];
-  c.next = (c.ks == 0 && d.rank > 0) ? 1 : 0;
-  c.npass = (c.n_e + NTOK - 1) / NTOK;
-  c.cbytes = cbytes;
   const uint32_t b0 = smem_u32(bars);
+  const uint32_t done_bar = b0 + 8 * (2 * dk::kStages + 2 * dk::kABufs + 4);
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int i = 0; i < dk::kStages; ++i) {
-      mbar_init(b0 + 8 * i, 1);                  // full: producer arrival + tx bytes
-      mbar_init(b0 + 8 * (dk::kStages + i), 5);  // empty: 4 dequant warps + MMA commit
+      mbar_init(b0 + 8 * i, 1);                                  // full: producer arrival + tx bytes
+      mbar_init(b0 + 8 * (dk::kStages + i), dk::kDqWarps + 1);   // empty: dequant warps + MMA commit
     }
     for (int i = 0; i < dk::kABufs; ++i) {
-      mbar_init(b0 + 8 * (2 * dk::kStages + i), 4);               // A buffer written (4 warps)
+      mbar_init(b0 + 8 * (2 * dk::kStages + i), dk::kDqWarps);    // A buffer written
       mbar_init(b0 + 8 * (2 * dk::kStages + dk::kABufs + i), 1);  // A buffer free (MMA commit)
     }
-    mbar_init(b0 + 8 * (2 * dk::kStages + 2 * dk::kABufs), 1);      // accumulator complete
-    mbar_init(b0 + 8 * (2 * dk::kStages + 2 * dk::kABufs + 1), 4);  // accumulator drained
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(b0 + 8 * (2 * dk::kStages + 2 * dk::kABufs + i), 1);                 // accumulator complete
+      mbar_init(b0 + 8 * (2 * dk::kStages + 2 * dk::kABufs + 2 + i), dk::kDqWarps);  // accumulator read
+    }
+    mbar_init(done_bar, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) tmem_alloc(smem_u32(&tmem_slot), dk::tmem_cols(NTOK));
+  if (warp == dk::kDqWarps + 1) tmem_alloc(smem_u32(&tmem_slot), dk::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  volatile int* ab = &abort_flag;
-  bool ran = true;
-  if (d.fmt == FMT_INT) {
-    switch (d.bits * 1000 + d.group) {
-      case 2064: decode_tile<NTOK, FMT_INT, 2, 64>(a, d, c, sm, stage_b, b0, tmem, ab); break;
-      case 2128: decode_tile<NTOK, FMT_INT, 2, 128>(a, d, c, sm, stage_b, b0, tmem, ab); break;
-      case 3064: decode_tile<NTOK, FMT_INT, 3, 64>(a, d, c, sm, stage_b, b0, tmem, ab); break;
-      case 3128: decode_tile<NTOK, FMT_INT, 3, 128>(a, d, c, sm, stage_b, b0, tmem, ab); break;
-      case 4064: decode_tile<NTOK, FMT_INT, 4, 64>(a, d, c, sm, stage_b, b0, tmem, ab); break;
-      case 4128: decode_tile<NTOK, FMT_INT, 4, 128>(a, d, c, sm, stage_b, b0, tmem, ab); break;
-      default: ran = false; break;
-    }
-  } else if (d.fmt == FMT_BITPLANE) {
-    switch (d.bits) {
-      case 2: decode_tile<NTOK, FMT_BITPLANE, 2, 64>(a, d, c, sm, stage_b, b0, tmem, ab); break;
-      case 3: decode_tile<NTOK, FMT_BITPLANE, 3, 64>(a, d, c, sm, stage_b, b0, tmem, ab); break;
-      case 4: decode_tile<NTOK, FMT_BITPLANE, 4, 64>(a, d, c, sm, stage_b, b0, tmem, ab); break;
-      default: ran = false; break;
-    }
-  } else if (d.fmt == FMT_DENSE) {
-    decode_tile<NTOK, FMT_DENSE, 16, 64>(a, d, c, sm, stage_b, b0, tmem, ab);
-  } else {
-    ran = false;
+  if (warp < 4) {
+    // constant correction columns of both A buffers: (1024, 1024), then zeros
+    const uint32_t lb = (uint32_t)(warp * 32) << 16;
+    const uint32_t cz[8] = {dk::kOne1024, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    for (int b = 0; b < dk::kABufs; ++b) tmem_st8_nw(tmem + lb + dk::kABase + b * dk::kACols + 32, cz);
+    tmem_wait_st();
   }
-  if (!ran && threadIdx.x == 0) atomicOr(a.status, ST_BOUNDS);
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
-    tc_fence_after();
-    tmem_dealloc(tmem, dk::tmem_cols(NTOK));
+  tc_fence_after();
+  // everything above overlaps the previous kernel's tail
+  pdl_wait();
+  pdl_trigger();
+  const int RB = a.M / dk::kRows;
+  const int total = *a.n_active * RB * a.KS;
+  volatile int* ab = &abort_flag;
+  dk::Cnt cnt;
+  for (int tile = blockIdx.x; tile < total && !*ab; tile += gridDim.x) {
+    const int slot = tile / (RB * a.KS);
+    const int rem = tile % (RB * a.KS);
+    const int e = a.active[slot];
+    dk::Ctx c;
+    c.n_e = a.counts[e];
+    if (c.n_e <= 0) continue;
+    c.prow0 = a.poffsets[e];
+    c.rb = rem / a.KS;
+    c.ks = rem % a.KS;
+    const BlockDesc& d = a.experts[e].blk[a.block];
+    c.next = (c.ks == 0 && d.rank > 0) ? 1 : 0;
+    c.npass = (c.n_e + NTOK - 1) / NTOK;
+    c.kc0 = c.nmain = 0;
+    bool ran = true;
+    if (d.fmt == FMT_INT) {
+      switch (d.bits * 1000 + d.group) {
+        case 2064: dk::decode_tile<NTOK, FMT_INT, 2, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
+        case 2128: dk::decode_tile<NTOK, FMT_INT, 2, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
+        case 3064: dk::decode_tile<NTOK, FMT_INT, 3, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
+        case 3128: dk::decode_tile<NTOK, FMT_INT, 3, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
+        case 4064: dk::decode_tile<NTOK, FMT_INT, 4, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
+        case 4128: dk::decode_tile<NTOK, FMT_INT, 4, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
+        default: ran = false; break;
+      }
+    } else if (d.fmt == FMT_BITPLANE) {
+      switch (d.bits) {
+        case 2: dk::decode_tile<NTOK, FMT_BITPLANE, 2, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
+        case 3: dk::decode_tile<NTOK, FMT_BITPLANE, 3, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
+        case 4: dk::decode_tile<NTOK, FMT_BITPLANE, 4, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
+        default: ran = false; break;
+      }
+    } else if (d.fmt == FMT_DENSE) {
+      dk::decode_tile<NTOK, FMT_DENSE, 16, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab);
+    } else {
+      ran = false;
+    }
+    if (!ran) {
+      if (threadIdx.x == 0) atomicOr(a.status, ST_BOUNDS);
+      break;
+    }
   }
+  if (warp == dk::kDqWarps && (threadIdx.x & 31) == 0) dk::producer_drain(a, b0, cnt);
+  if (warp == dk::kDqWarps + 1 && (threadIdx.x & 31) == 0) {
+    // every issued MMA must complete before TMEM is released
+    mma_commit(done_bar);
+    mbar_wait(done_bar, 0, a.status);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == dk::kDqWarps + 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, dk::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// per-group correction sums (one warp per routed row x group)
+
+__global__ void __launch_bounds__(256) act_corr_kernel(const CorrArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  act_corr_rows(a, blockIdx.y, blockIdx.x, gridDim.x);
+}
+
+int act_corr_ctas(int rows_per_expert, int K) {
+  const long long items = (long long)rows_per_expert * (K / 64);
+  return (int)std::max<long long>(1, std::min<long long>((items + 7) / 8, 256));
+}
+
+cudaError_t launch_act_corr(const CorrArgs& a, int rows_per_expert, int grid_y, cudaStream_t st, int* launches) {
+  const cudaError_t err =
+      launch_kernel(act_corr_kernel, dim3(act_corr_ctas(rows_per_expert, a.K), grid_y), dim3(256), 0, st, true, a);
+  if (launches) ++*launches;
+  return err;
 }
 
 int decode_rows_per_cta() { return dk::kRows; }
 
+static int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
 template <int NTOK>
 static cudaError_t launch_ntok(const DecodeArgs& a, int maxbits, int grid_y, cudaStream_t st) {
   const int stage_b = dk::stage_bytes(NTOK, maxbits);
-  const size_t smem = (size_t)dk::kStages * stage_b + 1024;
+  // at least 80 KiB so that at most two CTAs (2 x 256 TMEM columns) share an SM
+  const size_t smem = std::max<size_t>((size_t)dk::kStages * stage_b + 1024, 80 * 1024);
   cudaError_t err = cudaFuncSetAttribute(decode_gemm_kernel<NTOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
   if (err != cudaSuccess) return err;
-  dim3 grid((a.M / dk::kRows) * a.KS, grid_y);
-  decode_gemm_kernel<NTOK><<<grid, dk::kThreads, smem, st>>>(a, stage_b, dk::code_bytes(maxbits));
-  return cudaGetLastError();
+  const long long tiles = (long long)grid_y * (a.M / dk::kRows) * a.KS;
+  const int grid = (int)std::min<long long>(tiles, 2LL * num_sms());
+  return launch_kernel(decode_gemm_kernel<NTOK>, dim3(grid), dim3(dk::kThreads), smem, st, true, a, stage_b,
+                       dk::code_bytes(maxbits));
 }
 
 cudaError_t launch_decode_gemm(const DecodeArgs& a, int ntok, int maxbits, int grid_y, cudaStream_t st,
@@ -348,8 +510,7 @@ cudaError_t launch_decode_gemm(const DecodeArgs& a, int ntok, int maxbits, int g
   if (launches) ++*launches;
   if (ntok <= 16) return launch_ntok<16>(a, maxbits, grid_y, st);
   if (ntok <= 32) return launch_ntok<32>(a, maxbits, grid_y, st);
-  if (ntok <= 64) return launch_ntok<64>(a, maxbits, grid_y, st);
-  return launch_ntok<128>(a, maxbits, grid_y, st);
+  return launch_ntok<64>(a, maxbits, grid_y, st);
 }
 
 }  // namespace moeq

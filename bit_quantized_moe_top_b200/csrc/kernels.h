@@ -4,9 +4,29 @@
 #include <cuda_runtime.h>
 #include "common.cuh"
 
+#include <utility>
+
 namespace moeq {
 
 enum : int { MODE_SWIGLU = 0, MODE_OUT = 1 };
+
+// Kernel launch on `st`, with programmatic stream serialization when `pdl`
+// (the kernel then calls pdl_wait() before it reads what earlier kernels wrote).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                 bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 struct RouteArgs {
   const float* logits;        // [T, E]
@@ -34,6 +54,7 @@ struct RouteArgs {
 
 struct DecodeArgs {
   CUtensorMap tmap_act;       // activations [rows, Kpad] fp16 row-major; box 64 x 16, 128-byte swizzle
+  CUtensorMap tmap_corr;      // per-group correction columns [rows, 16 * groups] fp16; box 16 x 16, 32-byte swizzle
   const ExpertDesc* experts;
   int block;                  // 0 = W1, 1 = W2
   const int* active;
@@ -51,7 +72,29 @@ struct DecodeArgs {
   unsigned* status;
 };
 
+// Per-group correction columns of the activations for the integer-code
+// decode GEMM: for routed row p and group g of an INT block,
+// corr[p][16g .. 16g+15] = (-XP_hi, -XP_lo, -X_hi, -X_lo, 0 x 12) in fp16, with
+// XP = sum_k (P_k / 1024) x_pk and X = sum_k x_pk over the group, each split
+// into an fp16 value and its fp16 remainder.
+struct CorrArgs {
+  const ExpertDesc* experts;
+  int block;
+  const int* active;
+  const int* n_active;
+  const int* counts;
+  const int* poffsets;
+  const __half* act;          // activations [rows, lda] fp16
+  long long lda;
+  int K;                      // input features of the block
+  __half* corr;               // [rows, ldc] fp16
+  long long ldc;
+  unsigned* status;
+};
+
 struct LowrankArgs {
+  CorrArgs corr;              // corr.act != nullptr: CTAs past the low-rank grid compute correction sums
+  int corr_ctas;
   const ExpertDesc* experts;
   int block;
   const int* active;
@@ -116,6 +159,8 @@ cudaError_t launch_route_topk(const RouteArgs& a, cudaStream_t st, int* launches
 cudaError_t launch_route_permute(const RouteArgs& a, cudaStream_t st, int* launches);
 int route_num_blocks(int T);
 
+cudaError_t launch_act_corr(const CorrArgs& a, int rows_per_expert, int grid_y, cudaStream_t st, int* launches);
+int act_corr_ctas(int rows_per_expert, int K);
 int decode_rows_per_cta();
 cudaError_t launch_decode_gemm(const DecodeArgs& a, int ntok, int maxbits, int grid_y, cudaStream_t st,
                                int* launches);

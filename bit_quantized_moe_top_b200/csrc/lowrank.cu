@@ -9,26 +9,41 @@
 // combine_kernel: y_t = sum_j w[t, j] * o_(t, j), slots in a fixed order, the
 // K-split partials of o summed first; bf16 out.
 #include "kernels.h"
+#include "corr.cuh"
 
 namespace moeq {
 
 constexpr int kLrWarps = 4;    // each warp: 16 routed rows (tokens) x all r columns
 constexpr int kLrRows = 16 * kLrWarps;
+constexpr int kCombineThreads = 128;
 
 // grid: (KS x token tiles of 64 rows, expert slots). Tokens are the MMA's M:
 // a warp's A fragments are 16 routed rows of the activations, its B
 // fragments come straight from the factor's dense fragments (two n8 tiles per
-// uint4). With KS == 1 the result is written directly; otherwise each CTA
+// uint4). A tile with few rows (small decode batches) spreads its K range over
+// the CTA's warps instead of its rows, so every warp keeps loads in flight;
+// the warps' partial products meet in shared memory and are summed in a fixed
+// order. With KS == 1 the result is written directly; otherwise each CTA
 // writes an fp32 partial and the last CTA of a (expert, token tile) sums the
 // partials in a fixed order.
 __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
   __shared__ int is_last;
+  __shared__ float red[kLrWarps][16][kMaxRank + 1];
+  pdl_wait();
+  pdl_trigger();
   const int slot = blockIdx.y;
+  const int lr_ctas = a.KS * a.tiles;
+  if ((int)blockIdx.x >= lr_ctas) {
+    // the same launch also computes the decode GEMM's correction sums
+    act_corr_rows(a.corr, slot, blockIdx.x - lr_ctas, a.corr_ctas);
+    return;
+  }
   if (slot >= *a.n_active) return;
   const int e = a.active[slot];
   const int n_e = a.counts[e];
   const int ks = blockIdx.x % a.KS, tile = blockIdx.x / a.KS;
-  if (tile * kLrRows >= n_e) return;
+  const int nrows = min(kLrRows, n_e - tile * kLrRows);
+  if (nrows <= 0) return;
   const BlockDesc& dd = a.experts[e].blk[a.block];
   const int r = dd.rank;
   if (r <= 0) return;
@@ -36,10 +51,14 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
   const int RF = r / 16;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, c = lane & 3;
+  // warps along K: 4 for one 16-row sub-tile, 2 for two, 1 otherwise
+  const int wk = nrows <= 16 ? 4 : nrows <= 32 ? 2 : 1;
+  const int rsub = warp / wk, kw = warp % wk;
   const int S16 = a.K / 16;
-  const int s0 = (int)((long long)S16 * ks / a.KS), s1 = (int)((long long)S16 * (ks + 1) / a.KS);
+  const int c0 = (int)((long long)S16 * ks / a.KS), c1 = (int)((long long)S16 * (ks + 1) / a.KS);
+  const int s0 = c0 + (c1 - c0) * kw / wk, s1 = c0 + (c1 - c0) * (kw + 1) / wk;
   const int prow0 = a.poffsets[e];
-  const int rbase = tile * kLrRows + warp * 16;  // first row (within the expert) of this warp
+  const int rbase = tile * kLrRows + rsub * 16;  // first row (within the expert) of this warp
   const uint32_t* act32 = reinterpret_cast<const uint32_t*>(a.act);
   float acc[8][4];
 #pragma unroll
@@ -47,11 +66,12 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) acc[t][q] = 0.f;
   if (rbase < n_e) {
+    // rows past the expert's count read the padded slack rows of the buffer
     const long long ra = prow0 + rbase + g, rb = ra + 8;  // rows of a0a1/a4a5 and a2a3/a6a7
+    const long long ldw = a.Kpad >> 1;                    // row pitch in u32
 #pragma unroll 4
     for (int S = s0; S < s1; ++S) {
       uint32_t av[4];
-      const long long ldw = a.Kpad >> 1;  // row pitch in u32
       av[0] = act32[ra * ldw + 8 * S + c];
       av[1] = act32[rb * ldw + 8 * S + c];
       av[2] = act32[ra * ldw + 8 * S + c + 4];
@@ -66,33 +86,36 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
       }
     }
   }
-  // acc[t][q]: row rbase + g + 8*(q>>1), column j = 8t + 2c + (q&1)
+  // acc[t][q]: row g + 8*(q>>1) of the sub-tile, column j = 8t + 2c + (q&1)
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    if (t >= 2 * RF) break;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) red[warp][g + 8 * (q >> 1)][8 * t + 2 * c + (q & 1)] = acc[t][q];
+  }
+  __syncthreads();
   auto store_u = [&](int n, int j, float v) {
     // only the first comp_top_n routing slots of a token are compensated
     if (a.comp_top_n > 0 && a.pslot[prow0 + n] >= a.comp_top_n) v = 0.f;
     a.act[(long long)(prow0 + n) * a.Kpad + a.K + j] = __float2half_rn(v);
   };
+  // the CTA's value for tile row i, column j: the K-warps' partials in order
+  auto cta_value = [&](int i, int j) {
+    const int sub = i >> 4;
+    float v = 0.f;
+    for (int w = 0; w < wk; ++w) v += red[sub * wk + w][i & 15][j];
+    return v;
+  };
   if (a.KS == 1) {
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      if (t >= 2 * RF) break;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int n = rbase + g + 8 * (q >> 1);
-        if (n < n_e) store_u(n, 8 * t + 2 * c + (q & 1), acc[t][q]);
-      }
+    for (int idx = threadIdx.x; idx < nrows * r; idx += blockDim.x) {
+      const int i = idx / r, j = idx % r;
+      store_u(tile * kLrRows + i, j, cta_value(i, j));
     }
     return;
   }
-#pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    if (t >= 2 * RF) break;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int n = rbase + g + 8 * (q >> 1);
-      if (n < n_e)
-        a.part[ks * a.part_ks_stride + (long long)(prow0 + n) * kMaxRank + 8 * t + 2 * c + (q & 1)] = acc[t][q];
-    }
+  for (int idx = threadIdx.x; idx < nrows * r; idx += blockDim.x) {
+    const int i = idx / r, j = idx % r;
+    a.part[ks * a.part_ks_stride + (long long)(prow0 + tile * kLrRows + i) * kMaxRank + j] = cta_value(i, j);
   }
   __threadfence();
   __syncthreads();
@@ -101,7 +124,6 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  const int nrows = min(kLrRows, n_e - tile * kLrRows);
   for (int idx = threadIdx.x; idx < nrows * r; idx += blockDim.x) {
     const int n = tile * kLrRows + idx / r, j = idx % r;
     float sum = 0.f;
@@ -112,7 +134,9 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
   if (threadIdx.x == 0) *sem = 0;
 }
 
-__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   float wt[kMaxTopK];
   long long pr[kMaxTopK];
@@ -120,10 +144,12 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
     wt[j] = a.w[(long long)t * a.k + j];
     pr[j] = a.pinv[(long long)t * a.k + j];
   }
-  for (int k = threadIdx.x * 4; k < a.K; k += blockDim.x * 4) {
+  // this CTA's slice of the token's K columns, 4 per thread
+  for (int k = (blockIdx.y * blockDim.x + threadIdx.x) * 4; k < a.K; k += gridDim.y * blockDim.x * 4) {
     float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < a.k; ++j) {
       float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
       for (int s = 0; s < a.KS; ++s) {
         const float4 v = *reinterpret_cast<const float4*>(a.O + s * a.ks_stride + pr[j] * a.K + k);
         o.x += v.x; o.y += v.y; o.z += v.z; o.w += v.w;
@@ -140,16 +166,17 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
 }
 
 cudaError_t launch_lowrank(const LowrankArgs& a, int grid_y, cudaStream_t st, int* launches) {
-  dim3 grid(a.KS * a.tiles, grid_y);
-  lowrank_kernel<<<grid, kLrWarps * 32, 0, st>>>(a);
+  dim3 grid(a.KS * a.tiles + (a.corr.act ? a.corr_ctas : 0), grid_y);
+  const cudaError_t err = launch_kernel(lowrank_kernel, grid, dim3(kLrWarps * 32), 0, st, true, a);
   if (launches) ++*launches;
-  return cudaGetLastError();
+  return err;
 }
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st, int* launches) {
-  combine_kernel<<<a.T, 256, 0, st>>>(a);
+  const int ky = (a.K + 4 * kCombineThreads - 1) / (4 * kCombineThreads);
+  const cudaError_t err = launch_kernel(combine_kernel, dim3(a.T, ky), dim3(kCombineThreads), 0, st, true, a);
   if (launches) ++*launches;
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace moeq

@@ -68,10 +68,12 @@ struct moe_layer {
   DevBuf idx, w, counts, offsets, poffsets, active, n_active, ticket, perm, inv_pos, pinv, pslot;
   int comp_top_n = 0;
   DevBuf block_counts, block_base, pblock_base, sem, status;
-  DevBuf xact, zact, obuf, part;
+  DevBuf xact, zact, obuf, part, corr_x, corr_z;
+  int ldc_x = 0, ldc_z = 0;  // correction columns per row: 16 per group of 64 (the smallest group)
   DevBuf hx, hl, hy;  // device buffers for forward_host
   CUtensorMap tmap_x, tmap_z;    // activation buffers, 128-row boxes (prefill GEMMs)
   CUtensorMap tmap_xd, tmap_zd;  // activation buffers, 16-row boxes (decode GEMMs)
+  CUtensorMap tmap_cx, tmap_cz;  // correction columns, 16 x 16 boxes (decode GEMMs)
   bool have_tmaps = false;
   int last_T = 0, last_k = 0, last_launches = 0;
   cudaStream_t last_stream = nullptr;
@@ -105,7 +107,8 @@ static moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_O
 
 // 2-D tensor map over a row-major fp16 [rows, cols] buffer: box 64 columns x
 // box_rows rows, 128-byte swizzle, zero fill outside the buffer.
-static bool encode_act_map(CUtensorMap* map, void* base, int cols, long long rows, int box_rows) {
+static bool encode_map(CUtensorMap* map, void* base, int cols, long long rows, int box_cols, int box_rows,
+                       CUtensorMapSwizzle swz) {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     cudaDriverEntryPointQueryResult q;
@@ -117,11 +120,14 @@ static bool encode_act_map(CUtensorMap* map, void* base, int cols, long long row
   }
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// activation rows: boxes of 64 columns (128 B, 128-byte swizzle)
+static bool encode_act_map(CUtensorMap* map, void* base, int cols, long long rows, int box_rows) {
+  return encode_map(map, base, cols, rows, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 static bool valid_desc(const moe_expert_desc_t& d, int K, int N) {
@@ -174,7 +180,7 @@ void moe_layer_destroy(moe_layer_t* L) {
   DevBuf* bufs[] = {&L->d_experts, &L->idx, &L->w, &L->counts, &L->offsets, &L->poffsets, &L->active,
                     &L->n_active, &L->ticket, &L->perm, &L->inv_pos, &L->pinv, &L->pslot, &L->block_counts,
                     &L->block_base, &L->pblock_base, &L->sem, &L->status, &L->xact, &L->zact, &L->obuf,
-                    &L->part, &L->hx, &L->hl, &L->hy};
+                    &L->part, &L->corr_x, &L->corr_z, &L->hx, &L->hl, &L->hy};
   for (DevBuf* b : bufs) dfree(*b);
   for (cudaEvent_t ev : L->events) cudaEventDestroy(ev);
   delete L;
@@ -257,6 +263,10 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   A(L->zact, sizeof(__half) * (size_t)L->rows_pad_max * L->Kpad_z);
   A(L->obuf, sizeof(float) * (size_t)o_elems * K);
   A(L->part, sizeof(float) * (size_t)L->kslr_max * L->rows_pad_max * kMaxRank);
+  L->ldc_x = 16 * (K / 64);
+  L->ldc_z = 16 * (N / 64);
+  A(L->corr_x, sizeof(__half) * (size_t)L->rows_pad_max * L->ldc_x);
+  A(L->corr_z, sizeof(__half) * (size_t)L->rows_pad_max * L->ldc_z);
   A(L->hx, sizeof(__nv_bfloat16) * (size_t)max_tokens * K);
   A(L->hl, sizeof(float) * (size_t)max_tokens * E);
   A(L->hy, sizeof(__nv_bfloat16) * (size_t)max_tokens * K);
@@ -265,7 +275,8 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
     return st;
   }
   cudaError_t ce = cudaSuccess;
-  DevBuf* zero[] = {&L->ticket, &L->sem, &L->status, &L->xact, &L->zact, &L->n_active, &L->counts};
+  DevBuf* zero[] = {&L->ticket, &L->sem, &L->status, &L->xact, &L->zact, &L->n_active, &L->counts, &L->corr_x,
+                    &L->corr_z};
   for (DevBuf* b : zero)
     if (ce == cudaSuccess) ce = cudaMemset(b->p, 0, b->n);
   if (ce == cudaSuccess)
@@ -278,7 +289,9 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   L->have_tmaps = encode_act_map(&L->tmap_x, L->xact.p, L->Kpad_x, L->rows_pad_max, 128) &&
                   encode_act_map(&L->tmap_z, L->zact.p, L->Kpad_z, L->rows_pad_max, 128) &&
                   encode_act_map(&L->tmap_xd, L->xact.p, L->Kpad_x, L->rows_pad_max, 16) &&
-                  encode_act_map(&L->tmap_zd, L->zact.p, L->Kpad_z, L->rows_pad_max, 16);
+                  encode_act_map(&L->tmap_zd, L->zact.p, L->Kpad_z, L->rows_pad_max, 16) &&
+                  encode_map(&L->tmap_cx, L->corr_x.p, L->ldc_x, L->rows_pad_max, 16, 16, CU_TENSOR_MAP_SWIZZLE_32B) &&
+                  encode_map(&L->tmap_cz, L->corr_z.p, L->ldc_z, L->rows_pad_max, 16, 16, CU_TENSOR_MAP_SWIZZLE_32B);
   if (!L->have_tmaps) {
     moe_layer_destroy(L);
     return MOE_ERR_CUDA;
@@ -482,10 +495,12 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int E = L->E, K = L->K, N = L->N;
   int maxbits[2] = {0, 0}, rmax = 0;
+  bool any_int[2] = {false, false};
   for (int e = 0; e < E; ++e) {
     for (int b = 0; b < 2; ++b) {
       const int bb = L->hdesc[e].blk[b].bits;
       maxbits[b] = bb > maxbits[b] ? bb : maxbits[b];
+      any_int[b] = any_int[b] || L->hdesc[e].blk[b].fmt == FMT_INT;
     }
     rmax = L->hdesc[e].blk[0].rank > rmax ? L->hdesc[e].blk[0].rank : rmax;
   }
@@ -528,9 +543,38 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
 
   const ExpertDesc* dexp = static_cast<const ExpertDesc*>(L->d_experts.p);
   const long long prows = (rows + 7LL * E + 7) / 8 * 8;
-  auto lowrank = [&](int block, __half* act, int Kpad, int Kin) {
-    if (ce != cudaSuccess || rmax == 0) return;
+  // per-group correction sums of a block's input rows (decode path, integer-code blocks)
+  auto make_corr = [&](int block, const __half* act, long long lda, int Kin, __half* corr, long long ldc) {
+    CorrArgs ca{};
+    if (prefill || !any_int[block]) return ca;  // ca.act == nullptr: nothing to compute
+    ca.experts = dexp;
+    ca.block = block;
+    ca.active = ra.active;
+    ca.n_active = ra.n_active;
+    ca.counts = ra.counts;
+    ca.poffsets = ra.poffsets;
+    ca.act = act;
+    ca.lda = lda;
+    ca.K = Kin;
+    ca.corr = corr;
+    ca.ldc = ldc;
+    ca.status = ra.status;
+    return ca;
+  };
+  const int corr_rows = (int)std::min<long long>(T, rows);
+  // the low-rank down-projection, with the correction sums in the same launch
+  auto lowrank = [&](int block, __half* act, int Kpad, int Kin, const CorrArgs& corr) {
+    if (ce != cudaSuccess) return;
+    if (rmax == 0) {
+      if (corr.act) {
+        prof_mark(L, st, block == 0 ? "act_corr_w1" : "act_corr_w2");
+        ce = launch_act_corr(corr, corr_rows, grid_y, st, &launches);
+      }
+      return;
+    }
     LowrankArgs la{};
+    la.corr = corr;
+    la.corr_ctas = corr.act ? act_corr_ctas(corr_rows, Kin) : 0;
     la.experts = dexp;
     la.block = block;
     la.active = ra.active;
@@ -542,8 +586,9 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     la.K = Kin;
     // token tiles of 64 rows per expert; split K only while the grid is small
     la.tiles = (int)std::min<long long>((T + 63) / 64, (rows + 63) / 64);
+    // about eight CTAs per SM: rows / 64 tiles plus the experts' ragged tails
     const long long ctas = (rows + 63) / 64 + grid_y / 2;
-    int ks = (int)std::max<long long>(1, 296 / std::max<long long>(1, ctas));
+    int ks = (int)std::max<long long>(1, (1184 + ctas - 1) / std::max<long long>(1, ctas));
     ks = std::max(1, std::min(ks, std::min(L->kslr_max, Kin / 256)));
     la.KS = ks;
     la.sem_stride = L->sem_stride;
@@ -557,7 +602,9 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     ce = launch_lowrank(la, grid_y, st, &launches);
   };
   // W1 side compensator U1 = X A1^T
-  lowrank(0, static_cast<__half*>(L->xact.p), L->Kpad_x, K);
+  lowrank(0, static_cast<__half*>(L->xact.p), L->Kpad_x, K,
+          make_corr(0, static_cast<const __half*>(L->xact.p), L->Kpad_x, K, static_cast<__half*>(L->corr_x.p),
+                    L->ldc_x));
   int ks2 = 1;
   if (prefill) {
     // tcgen05 path: one launch per block, CTAs over (row tile, 256-token pair, expert)
@@ -584,7 +631,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
       ce = launch_prefill_gemm(pa, pairs, grid_y, st, &launches);
     };
     prefill_gemm(0, L->tmap_x, K, 2 * N, MODE_SWIGLU);
-    lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N);
+    lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N, CorrArgs{});
     prefill_gemm(1, L->tmap_z, N, K, MODE_OUT);
   } else {
     // tokens per pass: cover the expected per-expert batch (mean + 3 sd);
@@ -592,11 +639,13 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     const double avg = (double)rows / E;
     const int want = (int)std::ceil(avg + 3.0 * std::sqrt(avg) + 1.0);
     const int ntok = std::min(64, std::min(T, want) <= 16 ? 16 : std::min(T, want) <= 32 ? 32 : 64);
-    auto decode_gemm = [&](int block, const CUtensorMap& map, int Kin, int M, int mode, int KS) {
+    auto decode_gemm = [&](int block, const CUtensorMap& map, const CUtensorMap& cmap, int Kin, int M, int mode,
+                           int KS) {
       if (ce != cudaSuccess) return;
       DecodeArgs da;
       std::memset(&da, 0, sizeof(da));
       da.tmap_act = map;
+      da.tmap_corr = cmap;
       da.experts = dexp;
       da.block = block;
       da.active = ra.active;
@@ -615,14 +664,16 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
       prof_mark(L, st, block == 0 ? "decode_gemm_w1_swiglu" : "decode_gemm_w2");
       ce = launch_decode_gemm(da, ntok, maxbits[block], grid_y, st, &launches);
     };
-    decode_gemm(0, L->tmap_xd, K, 2 * N, MODE_SWIGLU, 1);
-    lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N);
+    decode_gemm(0, L->tmap_xd, L->tmap_cx, K, 2 * N, MODE_SWIGLU, 1);
+    lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N,
+            make_corr(1, static_cast<const __half*>(L->zact.p), L->Kpad_z, N, static_cast<__half*>(L->corr_z.p),
+                      L->ldc_z));
     // split the down projection's K while its grid is small (fixed-order sum in the combine)
     const int row_tiles = K / decode_rows_per_cta();
     ks2 = std::max(1, 600 / std::max(1, row_tiles * grid_y));
     ks2 = std::min(ks2, std::min(L->ks2_max, N / 256));
     if (rows > 1024) ks2 = 1;
-    decode_gemm(1, L->tmap_zd, N, K, MODE_OUT, ks2);
+    decode_gemm(1, L->tmap_zd, L->tmap_cz, N, K, MODE_OUT, ks2);
   }
   if (ce == cudaSuccess) {
     CombineArgs ca{};

@@ -173,15 +173,12 @@ __device__ void dequant_and_epilogue(const PrefillArgs& a, const BlockDesc& d, c
       }
       const uint8_t* cs = sm + kSmemC + cs_slot * kCSlot;
       if (rvalid) {
-        uint32_t w[8];
-        uint32_t sz = 0;
         if constexpr (FMT == FMT_INT) {
-          load_row_words_int(cs + (t >> 7) * kBlk, t & 127, BITS, w);
-          sz = reinterpret_cast<const uint32_t*>(cs + 8192)[t];
+          decode_row64<FMT, BITS>(cs + (t >> 7) * kBlk, 0, t & 127, reinterpret_cast<const uint32_t*>(cs + 8192)[t],
+                                  lut, v);
         } else {
-          load_row_planes<BITS>(cs + (t >> 7) * 1024, 2048, t & 127, w);
+          decode_row64<FMT, BITS>(cs + (t >> 7) * 1024, 2048, t & 127, 0u, lut, v);
         }
-        decode_row64<FMT, BITS>(w, sz, lut, v);
       } else {
 #pragma unroll
         for (int q = 0; q < 32; ++q) v[q] = 0u;
@@ -264,6 +261,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1) prefill_gemm_kernel(const __g
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ int abort_flag;
   __shared__ uint32_t tmem_slot;
+  pdl_wait();
+  pdl_trigger();
   const int slot = blockIdx.z;
   if (slot >= *a.n_active) return;
   pf::Ctx c;
@@ -341,9 +340,10 @@ cudaError_t launch_prefill_gemm(const PrefillArgs& a, int grid_y, int grid_z, cu
     attr_set = true;
   }
   const int row_tiles = (a.M + pf::kBN - 1) / pf::kBN;
-  prefill_gemm_kernel<<<dim3(row_tiles, grid_y, grid_z), pf::kThreads, pf::kSmemAlloc, st>>>(a);
+  cudaError_t err = launch_kernel(prefill_gemm_kernel, dim3(row_tiles, grid_y, grid_z), dim3(pf::kThreads),
+                                  (size_t)pf::kSmemAlloc, st, true, a);
   if (launches) ++*launches;
-  return cudaGetLastError();
+  return err;
 }
 
 int prefill_smem_bytes() { return pf::kSmemAlloc; }

@@ -15,38 +15,43 @@ __device__ __forceinline__ int read_code(const uint8_t* row, int rowbytes, int b
   return (int)((v >> sh) & ((1u << bits) - 1u));
 }
 
-// Packs the 64 codes c[k] (k = 8s + 2j + h) of one row-chunk into the words
-// the decode routine expects (see decode_frag.cuh).
+// Packs the 64 codes c[k] of one row chunk into the words the decode
+// routines consume (field positions in decode_frag.cuh): half hh holds pairs
+// i = 0..15 of codes (32hh + 2i, 32hh + 2i + 1), the even code in bits 0..15.
 __device__ __forceinline__ void pack_int_words(const int (&c)[64], int bits, uint32_t (&w)[8]) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) w[i] = 0u;
-  for (int s = 0; s < 8; ++s)
-    for (int j = 0; j < 4; ++j)
+  for (int hh = 0; hh < 2; ++hh)
+    for (int i = 0; i < 16; ++i)
       for (int h = 0; h < 2; ++h) {
-        const int q = c[8 * s + 2 * j + h];
+        const uint32_t q = (uint32_t)c[32 * hh + 2 * i + h];
+        const int hs = 16 * h;
         if (bits == 4) {
-          w[s] |= (uint32_t)q << (4 * (j + 4 * h));
+          // word 4hh + i/4: slot j = i%4 at nibble 0/1 of byte 0/1 of the half
+          const int j = i & 3;
+          w[4 * hh + (i >> 2)] |= q << (hs + 4 * (j & 1) + 8 * (j >> 1));
+        } else if (bits == 2) {
+          // word 2hh + i/8: step i/4 (parity = byte), 2-bit field i%4
+          w[2 * hh + (i >> 3)] |= q << (hs + 8 * ((i >> 2) & 1) + 2 * (i & 3));
+        } else if (i < 15) {
+          // word 3hh + i/5: fields at bits 0, 3, 6, 9, 12 of the half
+          w[3 * hh + i / 5] |= q << (hs + 3 * (i % 5));
         } else {
-          const int p = 4 * (s & 1) + j;
-          w[s >> 1] |= (uint32_t)(q & 3) << (2 * (p & 3) + 8 * (p >> 2) + 16 * h);
-          if (bits == 3) {
-            const int t = s & 3;  // transform applied to hi word s>>2
-            const int base = (h ? 18 : 2) + 2 * j;
-            const int src = t == 0 ? base : t == 1 ? base + 1 : t == 2 ? (base + 8) & 31 : (base + 9) & 31;
-            w[4 + (s >> 2)] |= (uint32_t)(q >> 2) << src;
-          }
+          // pair 15: bit 0 in word a, bit 1 in word b, bit 2 in word c, at bit 15 of the half
+          for (int v = 0; v < 3; ++v) w[3 * hh + v] |= ((q >> v) & 1u) << (hs + 15);
         }
       }
 }
 
-// word-quad-major store of one row's words into a [128-row] block
+// store of one row's words into a [128-row] block (layouts in decode_frag.cuh)
 __device__ __forceinline__ void store_row_words(uint8_t* blk, int row, int bits, const uint32_t (&w)[8]) {
   if (bits == 4) {
     reinterpret_cast<uint4*>(blk)[row] = make_uint4(w[0], w[1], w[2], w[3]);
     reinterpret_cast<uint4*>(blk + 2048)[row] = make_uint4(w[4], w[5], w[6], w[7]);
-  } else {
+  } else if (bits == 2) {
     reinterpret_cast<uint4*>(blk)[row] = make_uint4(w[0], w[1], w[2], w[3]);
-    if (bits == 3) reinterpret_cast<uint2*>(blk + 2048)[row] = make_uint2(w[4], w[5]);
+  } else {
+    for (int v = 0; v < 6; ++v) reinterpret_cast<uint32_t*>(blk)[v * 128 + row] = w[v];
   }
 }
 
@@ -67,7 +72,7 @@ __global__ void relayout_int_kernel(const uint8_t* __restrict__ canon, uint8_t* 
   store_row_words(blk, row % 128, bits, w);
 }
 
-// one thread per (group, internal row): half2(s, -z*s)
+// one thread per (group, internal row): half2(s, z)
 __global__ void relayout_sz_kernel(const __half* __restrict__ s, const __half* __restrict__ z,
                                    uint32_t* __restrict__ out, int M, int K, int group, int block, int N) {
   const int G = K / group;
@@ -75,9 +80,8 @@ __global__ void relayout_sz_kernel(const __half* __restrict__ s, const __half* _
   if (tid >= (long long)G * M) return;
   const int row = (int)(tid % M), gi = (int)(tid / M);
   const int crow = canon_row(row, block, N);
-  const float sv = __half2float(s[(long long)crow * G + gi]);
-  const float zv = __half2float(z[(long long)crow * G + gi]);
-  out[(long long)gi * M + row] = pack_half2(sv, -zv * sv);
+  const __half2 v = __halves2half2(s[(long long)crow * G + gi], z[(long long)crow * G + gi]);
+  out[(long long)gi * M + row] = *reinterpret_cast<const uint32_t*>(&v);
 }
 
 // dense bf16 [M, K] (rows mapped by block/N) -> fp16 blocks: per (kc, rb),
@@ -158,40 +162,51 @@ __global__ void relayout_planes_kernel(const uint32_t* __restrict__ canon, uint3
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int half_to_int(uint16_t h) { return (int)__half2float(__ushort_as_half(h)); }
 
+template <int BITS>
+__device__ void unpack_int_half(const uint8_t* blk, int row, int h, int (&code)[32]) {
+  uint32_t w[4], raw[16];
+  load_half_words_int<BITS>(blk, row, h, w);
+  int_raw_half<BITS>(w, raw);
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t q = hsub2u(raw[i], int_magic<BITS>(i));
+    code[2 * i] = half_to_int((uint16_t)(q & 0xFFFF));
+    code[2 * i + 1] = half_to_int((uint16_t)(q >> 16));
+  }
+}
+
+template <int BITS>
+__device__ void unpack_plane_half(const uint8_t* blk, int plane_bytes, int row, int h, int (&code)[32]) {
+  uint32_t pw[4];
+  load_half_planes<BITS>(blk, plane_bytes, row, h, pw);
+  for (int s = 0; s < 4; ++s) {
+    const uint32_t nib = plane_codes<BITS>(pw, s);
+    for (int j = 0; j < 4; ++j)
+      for (int hh = 0; hh < 2; ++hh) code[8 * s + 2 * j + hh] = (int)((nib >> (4 * (2 * j + hh))) & 0xF);
+  }
+}
+
 __global__ void debug_unpack_kernel(BlockDesc d, uint8_t* __restrict__ out, int block, int N) {
   const int KC = d.K / 64;
   const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (tid >= (long long)KC * d.M) return;
   const int row = (int)(tid % d.M), kc = (int)(tid / d.M);
   const long long bidx = (long long)kc * (d.M / 128) + row / 128;
-  uint32_t w[8];
-  if (d.fmt == FMT_INT) {
-    load_row_words_int(d.codes + bidx * block_bytes(FMT_INT, d.bits), row % 128, d.bits, w);
-  } else {
-    for (int p = 0; p < d.bits; ++p) {
-      const uint2 v = reinterpret_cast<const uint2*>(d.codes + p * d.plane_stride + bidx * 1024)[row % 128];
-      w[2 * p] = v.x;
-      w[2 * p + 1] = v.y;
-    }
-  }
   const int crow = canon_row(row, block, N);
-  for (int s = 0; s < 8; ++s) {
-    uint32_t q[4];
-    uint32_t nib = 0;
+  for (int h = 0; h < 2; ++h) {
+    int code[32];
     if (d.fmt == FMT_INT) {
-      if (d.bits == 4) int_codes<4>(w, s, q);
-      else if (d.bits == 3) int_codes<3>(w, s, q);
-      else int_codes<2>(w, s, q);
+      const uint8_t* blk = d.codes + bidx * block_bytes(FMT_INT, d.bits);
+      if (d.bits == 4) unpack_int_half<4>(blk, row % 128, h, code);
+      else if (d.bits == 3) unpack_int_half<3>(blk, row % 128, h, code);
+      else unpack_int_half<2>(blk, row % 128, h, code);
     } else {
-      nib = d.bits == 4 ? plane_codes<4>(w, s) : d.bits == 3 ? plane_codes<3>(w, s) : plane_codes<2>(w, s);
+      const uint8_t* blk = d.codes + bidx * 1024;
+      const int pb = (int)d.plane_stride;
+      if (d.bits == 4) unpack_plane_half<4>(blk, pb, row % 128, h, code);
+      else if (d.bits == 3) unpack_plane_half<3>(blk, pb, row % 128, h, code);
+      else unpack_plane_half<2>(blk, pb, row % 128, h, code);
     }
-    for (int j = 0; j < 4; ++j)
-      for (int h = 0; h < 2; ++h) {
-        int code;
-        if (d.fmt == FMT_INT) code = half_to_int((uint16_t)(h ? (q[j] >> 16) : (q[j] & 0xFFFF)));
-        else code = (int)((nib >> (4 * (2 * j + h))) & 0xF);
-        out[(long long)crow * d.K + kc * 64 + 8 * s + 2 * j + h] = (uint8_t)code;
-      }
+    for (int k = 0; k < 32; ++k) out[(long long)crow * d.K + kc * 64 + 32 * h + k] = (uint8_t)code[k];
   }
 }
 

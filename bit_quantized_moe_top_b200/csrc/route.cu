@@ -23,6 +23,8 @@ __device__ __forceinline__ bool better(float a, int ia, float b, int ib) {
 __global__ void __launch_bounds__(kRouteThreads) route_topk_kernel(RouteArgs a) {
   __shared__ int hist[kMaxExperts];
   __shared__ int is_last;
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int e = threadIdx.x; e < a.E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
@@ -150,6 +152,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_topk_kernel(RouteArgs a) 
 __global__ void __launch_bounds__(kRouteThreads) route_permute_kernel(RouteArgs a) {
   __shared__ unsigned mask[kMaxExperts];
   __shared__ int prow_s[kRouteTokensPerCta * kMaxTopK];
+  pdl_wait();
+  pdl_trigger();
   for (int e = threadIdx.x; e < a.E; e += blockDim.x) mask[e] = 0u;
   __syncthreads();
   const int t0 = blockIdx.x * kRouteTokensPerCta;
@@ -202,18 +206,19 @@ __global__ void __launch_bounds__(kRouteThreads) route_permute_kernel(RouteArgs 
 
 cudaError_t launch_route_topk(const RouteArgs& a, cudaStream_t st, int* launches) {
   const int nb = (a.T + kRouteTokensPerCta - 1) / kRouteTokensPerCta;
-  route_topk_kernel<<<nb, kRouteThreads, 0, st>>>(a);
+  // first kernel of a forward: normally serialized after whatever the stream ran before
+  const cudaError_t err = launch_kernel(route_topk_kernel, dim3(nb), dim3(kRouteThreads), 0, st, false, a);
   if (launches) ++*launches;
-  return cudaGetLastError();
+  return err;
 }
 
 cudaError_t launch_route_permute(const RouteArgs& a, cudaStream_t st, int* launches) {
   const int nb = (a.T + kRouteTokensPerCta - 1) / kRouteTokensPerCta;
   int gs = 296 / nb;
   gs = gs < 1 ? 1 : gs > a.K / 256 ? a.K / 256 : gs;
-  route_permute_kernel<<<dim3(nb, gs), kRouteThreads, 0, st>>>(a);
+  const cudaError_t err = launch_kernel(route_permute_kernel, dim3(nb, gs), dim3(kRouteThreads), 0, st, true, a);
   if (launches) ++*launches;
-  return cudaGetLastError();
+  return err;
 }
 
 int route_num_blocks(int T) { return (T + kRouteTokensPerCta - 1) / kRouteTokensPerCta; }
