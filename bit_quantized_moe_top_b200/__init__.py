@@ -28,7 +28,8 @@ EXPORTS = ["moe_layer_create", "moe_layer_set_expert_weights", "moe_layer_set_bi
            "moe_layer_set_path",
            "moe_layer_forward", "moe_layer_forward_host", "moe_layer_get_routing", "moe_layer_debug_unpack",
            "moe_layer_sync_status", "moe_layer_last_launch_count", "moe_layer_set_profiling",
-           "moe_layer_kernel_times", "moe_route_topk_noalloc", "moe_status_string", "moe_layer_destroy"]
+           "moe_layer_kernel_times", "moe_route_topk_noalloc", "moe_plan_reduce", "moe_plan_restore",
+           "moe_status_string", "moe_layer_destroy"]
 
 
 class MoEError(RuntimeError):
@@ -41,6 +42,12 @@ class MoEError(RuntimeError):
 class ExpertDesc(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int * 2), ("format", ctypes.c_int), ("group_size", ctypes.c_int),
                 ("rank", ctypes.c_int)]
+
+
+class PlanBlock(ctypes.Structure):
+    _fields_ = [("committed_bits", ctypes.c_int), ("floor_bits", ctypes.c_int), ("max_steps", ctypes.c_int),
+                ("plane_bytes", ctypes.c_longlong), ("sensitivity", ctypes.c_float * 5),
+                ("routing_mult", ctypes.c_float), ("prompt_factor", ctypes.c_float)]
 
 
 _LIB = None
@@ -67,6 +74,10 @@ def _lib() -> ctypes.CDLL:
         lib.moe_layer_set_profiling.argtypes = [P, I]
         lib.moe_layer_kernel_times.argtypes = [P, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float), I]
         lib.moe_route_topk_noalloc.argtypes = [P, I, I, I, U, P, P, P, P, P]
+        PB = ctypes.POINTER(PlanBlock)
+        IP, LP = ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_longlong)
+        lib.moe_plan_reduce.argtypes = [PB, I, ctypes.c_longlong, ctypes.c_float, IP, LP]
+        lib.moe_plan_restore.argtypes = [PB, I, IP, ctypes.c_longlong, ctypes.c_float, IP, LP]
         lib.moe_status_string.argtypes = [I]
         lib.moe_status_string.restype = ctypes.c_char_p
         lib.moe_layer_destroy.argtypes = [P]
@@ -178,6 +189,44 @@ def moe_route_topk_noalloc(logits, top_k: int, idx, w, counts, offsets, flags: i
     T, E = logits.shape
     _check(_lib().moe_route_topk_noalloc(_ptr(logits), T, E, top_k, flags, _ptr(idx), _ptr(w), _ptr(counts),
                                          _ptr(offsets), stream), "moe_route_topk_noalloc")
+
+
+def _plan_blocks(blocks):
+    arr = (PlanBlock * len(blocks))()
+    for i, b in enumerate(blocks):
+        arr[i].committed_bits = b["committed_bits"]
+        arr[i].floor_bits = b["floor_bits"]
+        arr[i].max_steps = b["max_steps"]
+        arr[i].plane_bytes = b["plane_bytes"]
+        for j, g in b["sensitivity"].items():
+            arr[i].sensitivity[j] = g
+        arr[i].routing_mult = b["routing_mult"]
+        arr[i].prompt_factor = b["prompt_factor"]
+    return arr
+
+
+def moe_plan_reduce(blocks, bytes_target: int, eps: float):
+    """Greedy reduction plan. ``blocks``: dicts with the moe_plan_block_t
+    fields (``sensitivity`` maps a bitwidth b to g of b -> b-1). Returns
+    (status, new_bits, bytes_released); status MOE_OK or MOE_ERR_TOO_LARGE."""
+    n = len(blocks)
+    out = (ctypes.c_int * max(n, 1))()
+    rel = ctypes.c_longlong(0)
+    st = _lib().moe_plan_reduce(_plan_blocks(blocks), n, bytes_target, eps, out, ctypes.byref(rel))
+    if st not in (MOE_OK, 9):
+        raise MoEError(st, "moe_plan_reduce")
+    return st, [out[i] for i in range(n)], rel.value
+
+
+def moe_plan_restore(blocks, max_bits, bytes_budget: int, eps: float):
+    """Greedy restore plan; returns (new_bits, bytes_used)."""
+    n = len(blocks)
+    out = (ctypes.c_int * max(n, 1))()
+    mb = (ctypes.c_int * max(n, 1))(*max_bits)
+    used = ctypes.c_longlong(0)
+    _check(_lib().moe_plan_restore(_plan_blocks(blocks), n, mb, bytes_budget, eps, out, ctypes.byref(used)),
+           "moe_plan_restore")
+    return [out[i] for i in range(n)], used.value
 
 
 def moe_status_string(status: int) -> str:

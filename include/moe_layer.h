@@ -49,9 +49,13 @@
  *   - moe_layer_forward is asynchronous on the given CUDA stream; device-side
  *     errors surface at moe_layer_sync_status or at the next call.
  *   - One layer is used from one stream at a time.
- *   - Arithmetic: fp16 tensor-core operands (X, dequantised weights, the
- *     SwiGLU output and the compensator terms are rounded to fp16), fp32
- *     accumulation, bf16 output. |X| and |z| must stay below 65504.
+ *   - Arithmetic: fp16 tensor-core operands (X, the SwiGLU output and the
+ *     compensator terms are rounded to fp16; dequantised weights too on the
+ *     prefill path, while the decode path multiplies the exact integer codes
+ *     and applies scale and zero per group in fp32), fp32 accumulation, bf16
+ *     output. |X| and |z| must stay below 65504, and on the decode path of an
+ *     INT_ASYM block so must the sum of |x| over each quantisation group
+ *     (otherwise moe_layer_sync_status reports MOE_ERR_DEVICE_CHECK).
  */
 #ifndef MOE_LAYER_H
 #define MOE_LAYER_H
@@ -98,7 +102,7 @@ typedef struct moe_layer moe_layer_t; /* opaque */
 
 /* paths for moe_layer_set_path */
 #define MOE_PATH_AUTO 0    /* by T: decode kernels for small batches, prefill kernels above */
-#define MOE_PATH_DECODE 1  /* register-dequant mma.sync grouped GEMM */
+#define MOE_PATH_DECODE 1  /* weight-streaming tcgen05 grouped GEMM, unpacked codes in TMEM */
 #define MOE_PATH_PREFILL 2 /* TMA + shared-memory dequant + tcgen05/TMEM grouped GEMM */
 
 /* Create a layer on the current CUDA device.
@@ -201,6 +205,45 @@ int moe_layer_kernel_times(moe_layer_t* layer, const char** names, float* ms, in
  * must be serialised by the caller. Calls no allocating routine. */
 moe_status_t moe_route_topk_noalloc(const float* router_logits, int T, int E, int top_k, unsigned flags, int* idx,
                                     float* w, int* counts, int* offsets, void* cuda_stream);
+
+/* ---- Bitwidth planner (host only) ----
+ * PagedWeight ("What carries the argument"): under memory pressure the planner
+ * lowers the bitwidths of expert linear blocks ("weight pages") greedily,
+ * taking the actions with the lowest predicted damage per released byte until
+ * the byte target is met; the predicted damage of an action is
+ * d = max(eps, mu * g * eta): g the block's offline sensitivity for that
+ * bitwidth transition, mu the multiplier of its routing-mass bucket, eta its
+ * exponentiated prompt residual. One action drops one bit-plane (b -> b-1) of
+ * one block; floors and per-plan depth caps bound the actions (the pages'
+ * bitwidth floor stages and depth caps). Reading where the pages are silent:
+ * equal damage per byte goes to the lower block index, and a block's next
+ * action becomes a candidate only after its previous one was taken. */
+typedef struct {
+  int committed_bits;    /* q_i: current bitwidth, 2..4 */
+  int floor_bits;        /* lowest bitwidth a plan may assign, 2..committed_bits */
+  int max_steps;         /* depth cap: planes one plan may drop (reduce) or restore (restore), >= 0 */
+  long long plane_bytes; /* device bytes one bit-plane of the block occupies, > 0 */
+  float sensitivity[5];  /* g_i^b for the transition b -> b-1, indices 3 and 4 (others unused) */
+  float routing_mult;    /* mu of the block's routing-mass bucket, >= 0 */
+  float prompt_factor;   /* eta_i, >= 0 */
+} moe_plan_block_t;
+
+/* Reduction plan: releases at least bytes_target bytes if the floors and caps
+ * allow. new_bits [n] receives each block's planned bitwidth, *bytes_released
+ * the bytes the plan frees. MOE_OK when the target is met, MOE_ERR_TOO_LARGE
+ * when every allowed action was taken and the target is still not met (the
+ * plan is still written), MOE_ERR_INVALID_ARG for bad arguments. */
+moe_status_t moe_plan_reduce(const moe_plan_block_t* blocks, int n, long long bytes_target, float eps,
+                             int* new_bits, long long* bytes_released);
+
+/* Restore plan (pressure released, PagedWeight Figure 4: pages are reloaded
+ * before a higher bitwidth is committed): undoes reductions, the action whose
+ * undo removes the most damage per byte first, up to max_bits[i] per block and
+ * while the restored bytes stay within bytes_budget. An action b-1 -> b costs
+ * plane_bytes and removes the damage of the transition b -> b-1. new_bits,
+ * *bytes_used as above; MOE_OK or MOE_ERR_INVALID_ARG. */
+moe_status_t moe_plan_restore(const moe_plan_block_t* blocks, int n, const int* max_bits, long long bytes_budget,
+                              float eps, int* new_bits, long long* bytes_used);
 
 const char* moe_status_string(moe_status_t status);
 
