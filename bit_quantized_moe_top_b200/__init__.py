@@ -29,6 +29,7 @@ EXPORTS = ["moe_layer_create", "moe_layer_set_expert_weights", "moe_layer_set_bi
            "moe_layer_forward", "moe_layer_forward_host", "moe_layer_get_routing", "moe_layer_debug_unpack",
            "moe_layer_sync_status", "moe_layer_last_launch_count", "moe_layer_set_profiling",
            "moe_layer_kernel_times", "moe_route_topk_noalloc", "moe_plan_reduce", "moe_plan_restore",
+           "moe_layer_release_planes", "moe_layer_reload_planes", "moe_layer_page_state",
            "moe_status_string", "moe_layer_destroy"]
 
 
@@ -74,6 +75,9 @@ def _lib() -> ctypes.CDLL:
         lib.moe_layer_set_profiling.argtypes = [P, I]
         lib.moe_layer_kernel_times.argtypes = [P, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_float), I]
         lib.moe_route_topk_noalloc.argtypes = [P, I, I, I, U, P, P, P, P, P]
+        lib.moe_layer_release_planes.argtypes = [P, I, I, I, P]
+        lib.moe_layer_reload_planes.argtypes = [P, I, I, I, P]
+        lib.moe_layer_page_state.argtypes = [P, I, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]
         PB = ctypes.POINTER(PlanBlock)
         IP, LP = ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_longlong)
         lib.moe_plan_reduce.argtypes = [PB, I, ctypes.c_longlong, ctypes.c_float, IP, LP]
@@ -191,6 +195,29 @@ def moe_route_topk_noalloc(logits, top_k: int, idx, w, counts, offsets, flags: i
                                          _ptr(offsets), stream), "moe_route_topk_noalloc")
 
 
+def moe_layer_release_planes(layer: int, expert: int, block: int, keep: int, stream: Optional[int] = None) -> None:
+    _check(_lib().moe_layer_release_planes(layer, expert, block, keep, _stream(stream)), "moe_layer_release_planes")
+
+
+def moe_layer_reload_planes(layer: int, expert: int, block: int, planes: int, stream: Optional[int] = None) -> None:
+    _check(_lib().moe_layer_reload_planes(layer, expert, block, planes, _stream(stream)), "moe_layer_reload_planes")
+
+
+def moe_layer_page_state(layer: int, expert: int, block: int):
+    """(committed_bits, resident_planes, host_planes) of (expert, block)."""
+    c, r, h = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(_lib().moe_layer_page_state(layer, expert, block, ctypes.byref(c), ctypes.byref(r), ctypes.byref(h)),
+           "moe_layer_page_state")
+    return c.value, r.value, h.value
+
+
+def _stream(stream):
+    if stream is not None:
+        return stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
 def _plan_blocks(blocks):
     arr = (PlanBlock * len(blocks))()
     for i, b in enumerate(blocks):
@@ -257,6 +284,15 @@ class MoELayer:
 
     def set_bits(self, expert, block, bits):
         moe_layer_set_bits(self.handle, expert, block, bits)
+
+    def release_planes(self, expert, block, keep, stream=None):
+        moe_layer_release_planes(self.handle, expert, block, keep, stream)
+
+    def reload_planes(self, expert, block, planes, stream=None):
+        moe_layer_reload_planes(self.handle, expert, block, planes, stream)
+
+    def page_state(self, expert, block):
+        return moe_layer_page_state(self.handle, expert, block)
 
     def set_comp_top_n(self, n):
         moe_layer_set_comp_top_n(self.handle, n)

@@ -36,12 +36,12 @@ enum : unsigned { ST_BOUNDS = 1u, ST_TIMEOUT = 2u, ST_ROUTE = 4u, ST_RANGE = 8u 
 
 // One expert linear block as the kernels see it.
 struct BlockDesc {
-  const uint8_t* codes;   // code blocks [K/64][M/128][block] (INT / DENSE) or plane 0 (BITPLANE)
+  const uint8_t* codes;   // code blocks [K/64][M/128][block] (INT / DENSE)
+  const uint8_t* plane[4];// BITPLANE: plane p as [K/64][M/128][1 KiB] (null while released to host)
   const uint32_t* sz;     // INT: [K/g][M] half2(s, z), internal row order
   const uint32_t* lut;    // BITPLANE: 28 fp16 as 14 u32
   const uint32_t* brow;   // compensator B as fp16 pairs [r/2][M] (column-pair-major)
   const uint4* afrag;     // compensator A [r, K] as mma A-fragments [r/16][K/16][32] uint4 (fp16)
-  long long plane_stride; // BITPLANE: bytes between planes ([K/64][M/128][1 KiB] each)
   int fmt, bits, group, rank;
   int M, K;
   int loaded;

@@ -128,7 +128,7 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
         if constexpr (FMT == FMT_BITPLANE) {
 #pragma unroll
           for (int q = 0; q < BITS; ++q)
-            bulk_g2s(smem_u32(cs + q * 1024), d.codes + q * d.plane_stride + bidx * 1024, 1024, full + 8 * slot);
+            bulk_g2s(smem_u32(cs + q * 1024), d.plane[q] + bidx * 1024, 1024, full + 8 * slot);
         } else {
           bulk_g2s(smem_u32(cs), d.codes + bidx * kBlk, kBlk, full + 8 * slot);
         }

@@ -151,7 +151,10 @@ cudaError_t launch_relayout_dense(const __nv_bfloat16* src, uint8_t* out, int M,
 cudaError_t launch_relayout_afrag(const __nv_bfloat16* src, uint4* out, int r, int K, cudaStream_t st);
 cudaError_t launch_relayout_brow(const __nv_bfloat16* src, uint32_t* out, int M, int r, int block, int N,
                                  cudaStream_t st);
-cudaError_t launch_relayout_planes(const uint32_t* canon, uint32_t* out, int M, int K, int block, int N,
+struct PlaneOut {
+  uint8_t* p[4];  // the four plane buffers, [K/64][M/128][1 KiB] each
+};
+cudaError_t launch_relayout_planes(const uint32_t* canon, PlaneOut out, int M, int K, int block, int N,
                                    cudaStream_t st);
 cudaError_t launch_debug_unpack(const BlockDesc& d, uint8_t* out, int block, int N, cudaStream_t st);
 

@@ -46,9 +46,34 @@ void dfree(DevBuf& b) {
   b.n = 0;
 }
 
+// Bit-plane pages of one block: each plane is its own stream-ordered device
+// allocation so it can be released to (and restored from) pinned host memory.
+struct PlaneStore {
+  void* dev[4] = {nullptr, nullptr, nullptr, nullptr};
+  void* host[4] = {nullptr, nullptr, nullptr, nullptr};  // pinned copies of released planes (kept as a cache)
+  size_t bytes = 0;                                     // bytes of one plane
+  int resident = 0;                                     // planes 0..resident-1 are (or are being made) resident
+  cudaEvent_t reload = nullptr;                         // completion of the last reload's copies
+  bool reload_pending = false;
+};
+
 struct BlockStore {
   DevBuf codes, sz, lut, afrag, brow;
+  PlaneStore planes;
 };
+
+void free_planes(PlaneStore& ps) {
+  for (int p = 0; p < 4; ++p) {
+    if (ps.dev[p]) cudaFree(ps.dev[p]);
+    if (ps.host[p]) cudaFreeHost(ps.host[p]);
+    ps.dev[p] = ps.host[p] = nullptr;
+  }
+  if (ps.reload) cudaEventDestroy(ps.reload);
+  ps.reload = nullptr;
+  ps.reload_pending = false;
+  ps.resident = 0;
+  ps.bytes = 0;
+}
 
 }  // namespace
 
@@ -77,6 +102,7 @@ struct moe_layer {
   bool have_tmaps = false;
   int last_T = 0, last_k = 0, last_launches = 0;
   cudaStream_t last_stream = nullptr;
+  cudaEvent_t fwd_done = nullptr;  // recorded at the end of every forward (page release orders after it)
   // profiling: events around each launch of the last forward
   bool profiling = false;
   std::vector<cudaEvent_t> events;
@@ -149,6 +175,7 @@ static bool valid_desc(const moe_expert_desc_t& d, int K, int N) {
 }
 
 static void free_block(BlockStore& s) {
+  free_planes(s.planes);
   dfree(s.codes);
   dfree(s.sz);
   dfree(s.lut);
@@ -183,6 +210,7 @@ void moe_layer_destroy(moe_layer_t* L) {
                     &L->part, &L->corr_x, &L->corr_z, &L->hx, &L->hl, &L->hy};
   for (DevBuf* b : bufs) dfree(*b);
   for (cudaEvent_t ev : L->events) cudaEventDestroy(ev);
+  if (L->fwd_done) cudaEventDestroy(L->fwd_done);
   delete L;
 }
 
@@ -281,6 +309,7 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
     if (ce == cudaSuccess) ce = cudaMemset(b->p, 0, b->n);
   if (ce == cudaSuccess)
     ce = cudaMemcpy(L->d_experts.p, L->hdesc.data(), sizeof(ExpertDesc) * E, cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess) ce = cudaEventCreateWithFlags(&L->fwd_done, cudaEventDisableTiming);
   if (ce == cudaSuccess) ce = cudaDeviceSynchronize();
   if (ce != cudaSuccess) {
     moe_layer_destroy(L);
@@ -357,11 +386,23 @@ moe_status_t moe_layer_set_expert_weights(moe_layer_t* L, int e, int block, cons
     const void* dl = nullptr;
     st = stage_in(t1, codes, nbytes, ptr_kind, &dc);
     if (st == MOE_OK) st = stage_in(t3, zeros_or_lut, 28 * sizeof(__half), ptr_kind, &dl);
-    if (st == MOE_OK) st = dalloc(S.codes, (size_t)4 * KC * RB * 1024);
+    PlaneStore& ps = S.planes;
+    ps.bytes = (size_t)KC * RB * 1024;
+    PlaneOut po;
+    for (int p = 0; p < 4 && st == MOE_OK; ++p) {
+      const int at = fail_alloc_at();
+      ++g_alloc_count;
+      if ((at >= 0 && g_alloc_count == at) || cudaMallocAsync(&ps.dev[p], ps.bytes, s0) != cudaSuccess) {
+        cudaGetLastError();
+        ps.dev[p] = nullptr;
+        st = MOE_ERR_OOM;
+      }
+      po.p[p] = static_cast<uint8_t*>(ps.dev[p]);
+    }
+    ps.resident = st == MOE_OK ? 4 : 0;
     if (st == MOE_OK) st = dalloc(S.lut, 28 * sizeof(__half));
     if (st == MOE_OK) {
-      ce = launch_relayout_planes(static_cast<const uint32_t*>(dc), static_cast<uint32_t*>(S.codes.p), M, Kin, block,
-                                  L->N, s0);
+      ce = launch_relayout_planes(static_cast<const uint32_t*>(dc), po, M, Kin, block, L->N, s0);
       if (ce == cudaSuccess) ce = cudaMemcpy(S.lut.p, dl, 28 * sizeof(__half), cudaMemcpyDeviceToDevice);
     }
   } else {
@@ -414,7 +455,7 @@ moe_status_t moe_layer_set_expert_weights(moe_layer_t* L, int e, int block, cons
   d.lut = static_cast<const uint32_t*>(S.lut.p);
   d.afrag = static_cast<const uint4*>(S.afrag.p);
   d.brow = static_cast<const uint32_t*>(S.brow.p);
-  d.plane_stride = (long long)KC * RB * 1024;
+  for (int p = 0; p < 4; ++p) d.plane[p] = static_cast<const uint8_t*>(S.planes.dev[p]);
   d.loaded = 1;
   return upload_desc(L, e);
 }
@@ -426,6 +467,18 @@ moe_status_t moe_layer_set_bits(moe_layer_t* L, int e, int block, int bits) {
   if (fmt == FMT_DENSE) return MOE_ERR_UNSUPPORTED;
   if (bits > 4) return MOE_ERR_BITS_UNAVAILABLE;
   if (bits < 2) return MOE_ERR_INVALID_ARG;
+  if (fmt == FMT_BITPLANE) {
+    // a bitwidth needs its planes resident; a pending reload completes first
+    for (int b = b0; b <= b1; ++b) {
+      PlaneStore& ps = L->store[2 * e + b].planes;
+      if (!L->hdesc[e].blk[b].loaded) continue;
+      if (bits > ps.resident) return MOE_ERR_BITS_UNAVAILABLE;
+      if (ps.reload_pending) {
+        if (cudaEventSynchronize(ps.reload) != cudaSuccess) return MOE_ERR_CUDA;
+        ps.reload_pending = false;
+      }
+    }
+  }
   for (int b = b0; b <= b1; ++b) {
     BlockDesc& d = L->hdesc[e].blk[b];
     if (d.bits == bits) continue;
@@ -441,6 +494,79 @@ moe_status_t moe_layer_set_bits(moe_layer_t* L, int e, int block, int bits) {
     }
   }
   return upload_desc(L, e);
+}
+
+moe_status_t moe_layer_release_planes(moe_layer_t* L, int e, int block, int keep, void* stream) {
+  if (!L || e < 0 || e >= L->E || block < 0 || block > 1 || keep < 2 || keep > 4) return MOE_ERR_INVALID_ARG;
+  BlockDesc& d = L->hdesc[e].blk[block];
+  if (d.fmt != FMT_BITPLANE) return MOE_ERR_UNSUPPORTED;
+  if (!d.loaded) return MOE_ERR_NOT_LOADED;
+  if (keep < d.bits) return MOE_ERR_INVALID_ARG;  // lower the committed bitwidth first
+  PlaneStore& ps = L->store[2 * e + block].planes;
+  if (keep >= ps.resident) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // after every forward issued so far (they may still read these planes)
+  cudaError_t ce = cudaStreamWaitEvent(st, L->fwd_done, 0);
+  if (ce == cudaSuccess && ps.reload_pending) ce = cudaStreamWaitEvent(st, ps.reload, 0);
+  for (int p = keep; p < ps.resident && ce == cudaSuccess; ++p) {
+    if (!ps.host[p]) {
+      if (cudaMallocHost(&ps.host[p], ps.bytes) != cudaSuccess) {
+        cudaGetLastError();
+        ps.host[p] = nullptr;
+        return MOE_ERR_OOM;
+      }
+      ce = cudaMemcpyAsync(ps.host[p], ps.dev[p], ps.bytes, cudaMemcpyDeviceToHost, st);
+    }
+    if (ce == cudaSuccess) ce = cudaFreeAsync(ps.dev[p], st);
+    if (ce == cudaSuccess) {
+      ps.dev[p] = nullptr;
+      d.plane[p] = nullptr;
+    }
+  }
+  if (ce != cudaSuccess) return MOE_ERR_CUDA;
+  ps.resident = keep;
+  return upload_desc(L, e);
+}
+
+moe_status_t moe_layer_reload_planes(moe_layer_t* L, int e, int block, int planes, void* stream) {
+  if (!L || e < 0 || e >= L->E || block < 0 || block > 1 || planes < 2 || planes > 4) return MOE_ERR_INVALID_ARG;
+  BlockDesc& d = L->hdesc[e].blk[block];
+  if (d.fmt != FMT_BITPLANE) return MOE_ERR_UNSUPPORTED;
+  if (!d.loaded) return MOE_ERR_NOT_LOADED;
+  PlaneStore& ps = L->store[2 * e + block].planes;
+  if (planes <= ps.resident) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t ce = cudaSuccess;
+  if (!ps.reload) ce = cudaEventCreateWithFlags(&ps.reload, cudaEventDisableTiming);
+  for (int p = ps.resident; p < planes && ce == cudaSuccess; ++p) {
+    if (!ps.host[p]) return MOE_ERR_BITS_UNAVAILABLE;
+    ce = cudaMallocAsync(&ps.dev[p], ps.bytes, st);
+    if (ce != cudaSuccess) {
+      cudaGetLastError();
+      ps.dev[p] = nullptr;
+      return MOE_ERR_OOM;
+    }
+    ce = cudaMemcpyAsync(ps.dev[p], ps.host[p], ps.bytes, cudaMemcpyHostToDevice, st);
+    d.plane[p] = static_cast<const uint8_t*>(ps.dev[p]);
+    ps.resident = p + 1;
+  }
+  if (ce == cudaSuccess) ce = cudaEventRecord(ps.reload, st);
+  if (ce != cudaSuccess) return MOE_ERR_CUDA;
+  ps.reload_pending = true;
+  return upload_desc(L, e);
+}
+
+moe_status_t moe_layer_page_state(moe_layer_t* L, int e, int block, int* committed_bits, int* resident_planes,
+                                  int* host_planes) {
+  if (!L || e < 0 || e >= L->E || block < 0 || block > 1) return MOE_ERR_INVALID_ARG;
+  const BlockDesc& d = L->hdesc[e].blk[block];
+  const PlaneStore& ps = L->store[2 * e + block].planes;
+  int nh = 0;
+  for (int p = 0; p < 4; ++p) nh += ps.host[p] ? 1 : 0;
+  if (committed_bits) *committed_bits = d.bits;
+  if (resident_planes) *resident_planes = d.fmt == FMT_BITPLANE ? ps.resident : (d.loaded ? d.bits : 0);
+  if (host_planes) *host_planes = nh;
+  return MOE_OK;
 }
 
 moe_status_t moe_layer_set_comp_top_n(moe_layer_t* L, int n) {
@@ -690,6 +816,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     ce = launch_combine(ca, st, &launches);
   }
   prof_end(L, st);
+  cudaEventRecord(L->fwd_done, st);
   L->last_T = T;
   L->last_k = top_k;
   L->last_launches = launches;

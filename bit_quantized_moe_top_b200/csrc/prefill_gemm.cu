@@ -81,7 +81,7 @@ __device__ void producer(const PrefillArgs& a, const BlockDesc& d, const Ctx& c,
       if constexpr (FMT == FMT_BITPLANE) {
 #pragma unroll
         for (int p = 0; p < BITS; ++p)
-          bulk_g2s(smem_u32(cs + p * 2048), d.codes + p * d.plane_stride + bidx * 1024, 1024 * nrb, c_full + 8 * slot);
+          bulk_g2s(smem_u32(cs + p * 2048), d.plane[p] + bidx * 1024, 1024 * nrb, c_full + 8 * slot);
       } else {
         bulk_g2s(smem_u32(cs), d.codes + bidx * kBlk, kBlk * nrb, c_full + 8 * slot);
       }

@@ -134,8 +134,8 @@ __global__ void relayout_brow_kernel(const __nv_bfloat16* __restrict__ src, uint
 }
 
 // bit-planes [4][M][K/32] u32 -> per plane [kc][rb][128 rows x 8 B]
-__global__ void relayout_planes_kernel(const uint32_t* __restrict__ canon, uint32_t* __restrict__ out, int M, int K,
-                                       int block, int N) {
+__global__ void relayout_planes_kernel(const uint32_t* __restrict__ canon, PlaneOut out, int M, int K, int block,
+                                       int N) {
   const int KC = K / 64, KW = K / 32;
   const long long per_plane = (long long)KC * M;
   const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
@@ -152,8 +152,8 @@ __global__ void relayout_planes_kernel(const uint32_t* __restrict__ canon, uint3
         const uint32_t word = canon[((long long)p * M + crow) * KW + (kk >> 5)];
         w[s >> 2] |= ((word >> (kk & 31)) & 1u) << (4 * (2 * j + h) + (s & 3));
       }
-  const long long o = ((long long)p * KC + kc) * (M / 128) + row / 128;  // block index
-  reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(out) + o * 1024)[row % 128] = make_uint2(w[0], w[1]);
+  const long long o = (long long)kc * (M / 128) + row / 128;  // block index within the plane
+  reinterpret_cast<uint2*>(out.p[p] + o * 1024)[row % 128] = make_uint2(w[0], w[1]);
 }
 
 // ---------------------------------------------------------------------------
@@ -175,9 +175,10 @@ __device__ void unpack_int_half(const uint8_t* blk, int row, int h, int (&code)[
 }
 
 template <int BITS>
-__device__ void unpack_plane_half(const uint8_t* blk, int plane_bytes, int row, int h, int (&code)[32]) {
+__device__ void unpack_plane_half(const BlockDesc& d, long long bidx, int row, int h, int (&code)[32]) {
   uint32_t pw[4];
-  load_half_planes<BITS>(blk, plane_bytes, row, h, pw);
+#pragma unroll
+  for (int p = 0; p < 4; ++p) pw[p] = p < BITS ? reinterpret_cast<const uint32_t*>(d.plane[p] + bidx * 1024)[2 * row + h] : 0u;
   for (int s = 0; s < 4; ++s) {
     const uint32_t nib = plane_codes<BITS>(pw, s);
     for (int j = 0; j < 4; ++j)
@@ -200,11 +201,9 @@ __global__ void debug_unpack_kernel(BlockDesc d, uint8_t* __restrict__ out, int 
       else if (d.bits == 3) unpack_int_half<3>(blk, row % 128, h, code);
       else unpack_int_half<2>(blk, row % 128, h, code);
     } else {
-      const uint8_t* blk = d.codes + bidx * 1024;
-      const int pb = (int)d.plane_stride;
-      if (d.bits == 4) unpack_plane_half<4>(blk, pb, row % 128, h, code);
-      else if (d.bits == 3) unpack_plane_half<3>(blk, pb, row % 128, h, code);
-      else unpack_plane_half<2>(blk, pb, row % 128, h, code);
+      if (d.bits == 4) unpack_plane_half<4>(d, bidx, row % 128, h, code);
+      else if (d.bits == 3) unpack_plane_half<3>(d, bidx, row % 128, h, code);
+      else unpack_plane_half<2>(d, bidx, row % 128, h, code);
     }
     for (int k = 0; k < 32; ++k) out[(long long)crow * d.K + kc * 64 + 32 * h + k] = (uint8_t)code[k];
   }
@@ -237,7 +236,7 @@ cudaError_t launch_relayout_brow(const __nv_bfloat16* src, uint32_t* out, int M,
   relayout_brow_kernel<<<grid_for((long long)(r / 2) * M, 256), 256, 0, st>>>(src, out, M, r, block, N);
   return cudaGetLastError();
 }
-cudaError_t launch_relayout_planes(const uint32_t* canon, uint32_t* out, int M, int K, int block, int N,
+cudaError_t launch_relayout_planes(const uint32_t* canon, PlaneOut out, int M, int K, int block, int N,
                                    cudaStream_t st) {
   relayout_planes_kernel<<<grid_for((long long)(K / 64) * M * 4, 256), 256, 0, st>>>(canon, out, M, K, block, N);
   return cudaGetLastError();

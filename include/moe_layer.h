@@ -132,6 +132,31 @@ moe_status_t moe_layer_set_expert_weights(moe_layer_t* layer, int expert, int bl
  * MOE_ERR_UNSUPPORTED. Must not be called while a forward is in flight. */
 moe_status_t moe_layer_set_bits(moe_layer_t* layer, int expert, int block, int bits);
 
+/* ---- Weight-page movement (BITPLANE_LUT blocks) ----
+ * PagedWeight ("What carries the argument"; Figure 4, asynchronous page
+ * movement): a weight page is one bit-plane of an expert linear block. Each
+ * plane is its own stream-ordered device allocation; released planes move to
+ * pinned host memory that the layer owns (and keeps as a cache until the
+ * block's weights are set again or the layer is destroyed).
+ *
+ * moe_layer_release_planes: keep planes 0..keep-1 on the device and release
+ * planes keep..3. Requires committed bits <= keep (lower them with
+ * moe_layer_set_bits first; 2 <= keep <= 4). On `cuda_stream`, after every
+ * forward issued so far: each released plane is copied to host (unless a host
+ * copy is already cached) and its device memory is freed. Asynchronous.
+ * moe_layer_reload_planes: make planes 0..planes-1 resident again: allocates
+ * and copies the missing planes back from host on `cuda_stream`
+ * (asynchronous). A later moe_layer_set_bits that needs them waits for these
+ * copies before it commits (the pages' rule: reload, then commit the higher
+ * bitwidth). moe_layer_set_bits with more bits than resident planes returns
+ * MOE_ERR_BITS_UNAVAILABLE. Other formats: MOE_ERR_UNSUPPORTED.
+ * moe_layer_page_state: committed bits, resident planes and host-cached planes
+ * of (expert, block); any output may be NULL. */
+moe_status_t moe_layer_release_planes(moe_layer_t* layer, int expert, int block, int keep, void* cuda_stream);
+moe_status_t moe_layer_reload_planes(moe_layer_t* layer, int expert, int block, int planes, void* cuda_stream);
+moe_status_t moe_layer_page_state(moe_layer_t* layer, int expert, int block, int* committed_bits,
+                                  int* resident_planes, int* host_planes);
+
 /* Router-guided compensation: with n > 0, only the first n routing slots of
  * each token (its n highest-logit experts) get the low-rank compensator; the
  * other slots run on the quantised weights alone (Bandwidth-Efficient
