@@ -56,12 +56,27 @@ constexpr int kDqWarps = 8;
 constexpr int kThreads = 32 * (kDqWarps + 2);
 constexpr int kRows = 128;
 constexpr int kStages = 4;
-constexpr int kABufs = 2;
 constexpr int kACols = 40;        // per A buffer: 32 code columns + 8 correction columns
 constexpr int kActBox = 16;       // rows per TMA box
-constexpr int kTmemCols = 256;    // accumulators at [0, 2 NTOK), A buffers at [128, 208)
-constexpr int kABase = 128;
+constexpr int kTmemCols = 256;
 constexpr uint32_t kOne1024 = 0x64006400u;  // fp16 pair (1024, 1024)
+
+// TMEM rings: accumulators at [0, kAcc * NTOK), A buffers from kABase. The
+// rings are as deep as 256 columns allow, so that the MMA round trip (issue,
+// completion, mbarrier) of a chunk or a group is covered by the unpacking of
+// the next ones; a group's epilogue runs kAcc - 1 groups after its last chunk.
+template <int NTOK>
+struct Ring {
+  static constexpr int kAcc = NTOK <= 32 ? 4 : 2;
+  static constexpr int kA = NTOK <= 16 ? 4 : 3;
+  static constexpr int kABase = kAcc * NTOK <= 64 ? 64 : 128;
+  static_assert(kABase + kA * kACols <= kTmemCols, "TMEM rings exceed the allocation");
+};
+// barrier slots (8 bytes each): full[kStages], empty[kStages], afull[4],
+// aempty[4], accfull[4], accfree[4], done
+constexpr int kBarFull = 0, kBarEmpty = kStages, kBarAFull = 2 * kStages, kBarAEmpty = kBarAFull + 4,
+              kBarAccFull = kBarAEmpty + 4, kBarAccFree = kBarAccFull + 4, kBarDone = kBarAccFree + 4,
+              kNumBars = kBarDone + 1;
 
 __host__ __device__ inline int code_bytes(int maxbits) { return maxbits >= 16 ? 16384 : 4096; }
 // stage: [act NTOK x 128 B][corr NTOK x 32 B][codes][scales 512 B]
@@ -96,7 +111,7 @@ __device__ __forceinline__ void group_pos(const Ctx& c, int i, bool& first, bool
 template <int NTOK, int FMT, int BITS, int GROUP>
 __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, uint8_t* sm, int stage_b, int cbytes,
                          uint32_t bars, Cnt& cnt, volatile int* abort_flag) {
-  const uint32_t full = bars, empty = bars + 8 * kStages;
+  const uint32_t full = bars + 8 * kBarFull, empty = bars + 8 * kBarEmpty;
   const int RB = a.M / kRows;
   constexpr int kBlk = (FMT == FMT_DENSE) ? 16384 : 128 * 8 * BITS;  // bytes of one code block (per plane: 1 KiB)
   for (int p = 0; p < c.npass && !*abort_flag; ++p) {
@@ -153,28 +168,29 @@ __device__ void producer_drain(const DecodeArgs& a, uint32_t bars, const Cnt& cn
 template <int NTOK, int FMT, int GROUP>
 __device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int stage_b, uint32_t bars, uint32_t tmem,
                            Cnt& cnt, volatile int* abort_flag) {
-  const uint32_t full = bars, empty = bars + 8 * kStages;
-  const uint32_t afull = bars + 16 * kStages, aempty = afull + 8 * kABufs;
-  const uint32_t accfull = aempty + 8 * kABufs, accfree = accfull + 16;
+  using RG = Ring<NTOK>;
+  const uint32_t full = bars + 8 * kBarFull, empty = bars + 8 * kBarEmpty;
+  const uint32_t afull = bars + 8 * kBarAFull, aempty = bars + 8 * kBarAEmpty;
+  const uint32_t accfull = bars + 8 * kBarAccFull, accfree = bars + 8 * kBarAccFree;
   for (int p = 0; p < c.npass; ++p) {
     const int n_pass = min(NTOK, c.n_e - p * NTOK);
     const int npad = (n_pass + 15) & ~15;
     const uint32_t idesc = idesc_f16(128, npad);
     for (int i = 0; i < c.nmain + c.next; ++i, ++cnt.it) {
-      const int slot = cnt.it % kStages, buf = cnt.it % kABufs;
+      const int slot = cnt.it % kStages, buf = cnt.it % RG::kA;
       bool first, last;
       group_pos<FMT, GROUP>(c, i, first, last);
-      const int ab = cnt.gc & 1;
+      const int ab = cnt.gc % RG::kAcc;
       if (*abort_flag || !mbar_wait(full + 8 * slot, (cnt.it / kStages) & 1, a.status) ||
-          !mbar_wait(afull + 8 * buf, (cnt.it / kABufs) & 1, a.status) ||
-          (first && !mbar_wait(accfree + 8 * ab, ((cnt.gc >> 1) & 1) ^ 1, a.status))) {
+          !mbar_wait(afull + 8 * buf, (cnt.it / RG::kA) & 1, a.status) ||
+          (first && !mbar_wait(accfree + 8 * ab, ((cnt.gc / RG::kAcc) & 1) ^ 1, a.status))) {
         *abort_flag = 1;
         return;
       }
       tc_fence_after();
       const uint32_t bt = smem_u32(sm + slot * stage_b);
       const uint32_t acc = tmem + ab * NTOK;
-      const uint32_t ta = tmem + kABase + buf * kACols;
+      const uint32_t ta = tmem + RG::kABase + buf * kACols;
       const bool corr = FMT == FMT_INT && i < c.nmain && first;
       if (corr) mma_f16_ts(acc, ta + 32, sw32_desc(bt + NTOK * 128), idesc, 0);
 #pragma unroll
@@ -194,9 +210,10 @@ __device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int s
 template <int NTOK>
 __device__ __forceinline__ bool group_epilogue(const DecodeArgs& a, uint32_t bars, uint32_t tmem, uint32_t lane_base,
                                                int h, int gq, float scale, float (&y)[NTOK / 2]) {
-  const uint32_t accfull = bars + 16 * kStages + 16 * kABufs, accfree = accfull + 16;
-  const int ab = gq & 1;
-  if (!__all_sync(0xffffffffu, mbar_wait(accfull + 8 * ab, (gq >> 1) & 1, a.status))) return false;
+  using RG = Ring<NTOK>;
+  const uint32_t accfull = bars + 8 * kBarAccFull, accfree = bars + 8 * kBarAccFree;
+  const int ab = gq % RG::kAcc;
+  if (!__all_sync(0xffffffffu, mbar_wait(accfull + 8 * ab, (gq / RG::kAcc) & 1, a.status))) return false;
   tc_fence_after();
   uint32_t v[NTOK / 2];
   tmem_ld<NTOK / 2>(tmem + lane_base + ab * NTOK + h * (NTOK / 2), v);
@@ -210,9 +227,12 @@ __device__ __forceinline__ bool group_epilogue(const DecodeArgs& a, uint32_t bar
 
 template <int NTOK, int FMT, int BITS, int GROUP>
 __device__ void dequant_epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, uint8_t* sm, int stage_b,
-                                 int cbytes, uint32_t bars, uint32_t tmem, Cnt& cnt, volatile int* abort_flag) {
-  const uint32_t full = bars, empty = bars + 8 * kStages;
-  const uint32_t afull = bars + 16 * kStages, aempty = afull + 8 * kABufs;
+                                 int cbytes, uint32_t bars, uint32_t tmem, Cnt& cnt, volatile int* abort_flag,
+                                 float* sscale) {
+  using RG = Ring<NTOK>;
+  constexpr int kDefer = RG::kAcc - 1;  // groups between a group's last chunk and its epilogue
+  const uint32_t full = bars + 8 * kBarFull, empty = bars + 8 * kBarEmpty;
+  const uint32_t afull = bars + 8 * kBarAFull, aempty = bars + 8 * kBarAEmpty;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3, h = warp >> 2;      // TMEM lane quarter, K half / token half
   const int row = q * 32 + lane;              // TMEM lane
@@ -227,21 +247,22 @@ __device__ void dequant_epilogue(const DecodeArgs& a, const BlockDesc& d, const 
     float y[NH];
 #pragma unroll
     for (int t = 0; t < NH; ++t) y[t] = 0.f;
-    int pending = -1;        // group whose epilogue is deferred by one chunk
-    float pend_scale = 1.f;
+    // groups whose epilogue is pending: cnt.gc - npend .. cnt.gc - 1; their
+    // scales wait in shared memory, one slot per accumulator
+    int npend = 0;
     float s_cur = 1.f;
     for (int i = 0; i < c.nmain + c.next; ++i, ++cnt.it) {
-      const int slot = cnt.it % kStages, buf = cnt.it % kABufs;
+      const int slot = cnt.it % kStages, buf = cnt.it % RG::kA;
       bool first, last;
       group_pos<FMT, GROUP>(c, i, first, last);
       // warp-uniform waits: every lane must reach the .sync.aligned TMEM stores
       const bool ok = !*abort_flag && mbar_wait(full + 8 * slot, (cnt.it / kStages) & 1, a.status) &&
-                      mbar_wait(aempty + 8 * buf, ((cnt.it / kABufs) & 1) ^ 1, a.status);
+                      mbar_wait(aempty + 8 * buf, ((cnt.it / RG::kA) & 1) ^ 1, a.status);
       if (!__all_sync(0xffffffffu, ok)) {
         *abort_flag = 1;
         return;
       }
-      const uint32_t ta = tmem + lane_base + kABase + buf * kACols;
+      const uint32_t ta = tmem + lane_base + RG::kABase + buf * kACols;
       uint32_t v[16];
       const bool main = i < c.nmain;
       if (main) {
@@ -279,22 +300,27 @@ __device__ void dequant_epilogue(const DecodeArgs& a, const BlockDesc& d, const 
         mbar_arrive(afull + 8 * buf);
         mbar_arrive(empty + 8 * slot);
       }
-      // the previous group's accumulator, while this chunk's MMAs queue
-      if (pending >= 0) {
-        if (!group_epilogue<NTOK>(a, bars, tmem, lane_base, h, pending, pend_scale, y)) {
+      // the oldest pending group's accumulator, kDefer groups behind the MMAs
+      if (npend == kDefer) {
+        const int gq = cnt.gc - npend;
+        if (!group_epilogue<NTOK>(a, bars, tmem, lane_base, h, gq, sscale[(h * 4 + gq % RG::kAcc) * kRows + row], y)) {
           *abort_flag = 1;
           return;
         }
-        pending = -1;
+        --npend;
       }
       if (last) {
-        pending = cnt.gc++;
-        pend_scale = (FMT == FMT_INT && main) ? s_cur : 1.f;
+        sscale[(h * 4 + cnt.gc % RG::kAcc) * kRows + row] = (FMT == FMT_INT && main) ? s_cur : 1.f;
+        ++npend;
+        ++cnt.gc;
       }
     }
-    if (pending >= 0 && !group_epilogue<NTOK>(a, bars, tmem, lane_base, h, pending, pend_scale, y)) {
-      *abort_flag = 1;
-      return;
+    for (; npend > 0; --npend) {
+      const int gq = cnt.gc - npend;
+      if (!group_epilogue<NTOK>(a, bars, tmem, lane_base, h, gq, sscale[(h * 4 + gq % RG::kAcc) * kRows + row], y)) {
+        *abort_flag = 1;
+        return;
+      }
     }
     // ---- outputs of pass p: tokens p*NTOK + h*NH + t
     const int tok0 = p * NTOK + h * NH;
@@ -324,7 +350,7 @@ __device__ void dequant_epilogue(const DecodeArgs& a, const BlockDesc& d, const 
 
 template <int NTOK, int FMT, int BITS, int GROUP>
 __device__ void decode_tile(const DecodeArgs& a, const BlockDesc& d, const Ctx& c0, uint8_t* sm, int stage_b,
-                            int cbytes, uint32_t bars, uint32_t tmem, Cnt& cnt, volatile int* ab) {
+                            int cbytes, uint32_t bars, uint32_t tmem, Cnt& cnt, volatile int* ab, float* sscale) {
   // group-aligned K range of this split
   Ctx c = c0;
   const int KC = a.K / 64;
@@ -340,7 +366,7 @@ __device__ void decode_tile(const DecodeArgs& a, const BlockDesc& d, const Ctx& 
   }
   const int warp = threadIdx.x >> 5;
   if (warp < kDqWarps) {
-    dequant_epilogue<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, tmem, cnt, ab);
+    dequant_epilogue<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, tmem, cnt, ab, sscale);
   } else if (warp == kDqWarps) {
     if ((threadIdx.x & 31) == 0) producer<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, cnt, ab);
   } else {
@@ -355,25 +381,24 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
                                                                         int stage_b, int cbytes) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // full, empty [stages]; afull, aempty [A bufs]; accfull, accfree [2]; done
-  __shared__ __align__(8) unsigned long long bars[2 * dk::kStages + 2 * dk::kABufs + 5];
+  using RG = dk::Ring<NTOK>;
+  __shared__ __align__(8) unsigned long long bars[dk::kNumBars];
+  __shared__ float sscale[2 * 4 * dk::kRows];  // [token half][accumulator][row]: scale of a pending group
   __shared__ int abort_flag;
   __shared__ uint32_t tmem_slot;
   const uint32_t b0 = smem_u32(bars);
-  const uint32_t done_bar = b0 + 8 * (2 * dk::kStages + 2 * dk::kABufs + 4);
+  const uint32_t done_bar = b0 + 8 * dk::kBarDone;
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int i = 0; i < dk::kStages; ++i) {
-      mbar_init(b0 + 8 * i, 1);                                  // full: producer arrival + tx bytes
-      mbar_init(b0 + 8 * (dk::kStages + i), dk::kDqWarps + 1);   // empty: dequant warps + MMA commit
+      mbar_init(b0 + 8 * (dk::kBarFull + i), 1);                  // producer arrival + tx bytes
+      mbar_init(b0 + 8 * (dk::kBarEmpty + i), dk::kDqWarps + 1);  // dequant warps + MMA commit
     }
-    for (int i = 0; i < dk::kABufs; ++i) {
-      mbar_init(b0 + 8 * (2 * dk::kStages + i), dk::kDqWarps);    // A buffer written
-      mbar_init(b0 + 8 * (2 * dk::kStages + dk::kABufs + i), 1);  // A buffer free (MMA commit)
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(b0 + 8 * (2 * dk::kStages + 2 * dk::kABufs + i), 1);                 // accumulator complete
-      mbar_init(b0 + 8 * (2 * dk::kStages + 2 * dk::kABufs + 2 + i), dk::kDqWarps);  // accumulator read
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(b0 + 8 * (dk::kBarAFull + i), dk::kDqWarps);    // A buffer written
+      mbar_init(b0 + 8 * (dk::kBarAEmpty + i), 1);              // A buffer free (MMA commit)
+      mbar_init(b0 + 8 * (dk::kBarAccFull + i), 1);             // accumulator complete (MMA commit)
+      mbar_init(b0 + 8 * (dk::kBarAccFree + i), dk::kDqWarps);  // accumulator read
     }
     mbar_init(done_bar, 1);
     abort_flag = 0;
@@ -388,7 +413,7 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
     // constant correction columns of both A buffers: (1024, 1024), then zeros
     const uint32_t lb = (uint32_t)(warp * 32) << 16;
     const uint32_t cz[8] = {dk::kOne1024, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-    for (int b = 0; b < dk::kABufs; ++b) tmem_st8_nw(tmem + lb + dk::kABase + b * dk::kACols + 32, cz);
+    for (int b = 0; b < RG::kA; ++b) tmem_st8_nw(tmem + lb + RG::kABase + b * dk::kACols + 32, cz);
     tmem_wait_st();
   }
   tc_fence_before();
@@ -418,23 +443,23 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
     bool ran = true;
     if (d.fmt == FMT_INT) {
       switch (d.bits * 1000 + d.group) {
-        case 2064: dk::decode_tile<NTOK, FMT_INT, 2, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
-        case 2128: dk::decode_tile<NTOK, FMT_INT, 2, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
-        case 3064: dk::decode_tile<NTOK, FMT_INT, 3, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
-        case 3128: dk::decode_tile<NTOK, FMT_INT, 3, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
-        case 4064: dk::decode_tile<NTOK, FMT_INT, 4, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
-        case 4128: dk::decode_tile<NTOK, FMT_INT, 4, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
+        case 2064: dk::decode_tile<NTOK, FMT_INT, 2, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
+        case 2128: dk::decode_tile<NTOK, FMT_INT, 2, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
+        case 3064: dk::decode_tile<NTOK, FMT_INT, 3, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
+        case 3128: dk::decode_tile<NTOK, FMT_INT, 3, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
+        case 4064: dk::decode_tile<NTOK, FMT_INT, 4, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
+        case 4128: dk::decode_tile<NTOK, FMT_INT, 4, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
         default: ran = false; break;
       }
     } else if (d.fmt == FMT_BITPLANE) {
       switch (d.bits) {
-        case 2: dk::decode_tile<NTOK, FMT_BITPLANE, 2, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
-        case 3: dk::decode_tile<NTOK, FMT_BITPLANE, 3, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
-        case 4: dk::decode_tile<NTOK, FMT_BITPLANE, 4, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab); break;
+        case 2: dk::decode_tile<NTOK, FMT_BITPLANE, 2, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
+        case 3: dk::decode_tile<NTOK, FMT_BITPLANE, 3, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
+        case 4: dk::decode_tile<NTOK, FMT_BITPLANE, 4, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
         default: ran = false; break;
       }
     } else if (d.fmt == FMT_DENSE) {
-      dk::decode_tile<NTOK, FMT_DENSE, 16, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab);
+      dk::decode_tile<NTOK, FMT_DENSE, 16, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale);
     } else {
       ran = false;
     }
