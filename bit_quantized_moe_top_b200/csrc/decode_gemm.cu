@@ -86,7 +86,8 @@ __host__ __device__ inline int stage_bytes(int ntok, int maxbits) {
 }
 
 struct Ctx {
-  int n_e, prow0, rb, ks, kc0, nmain, next, npass;
+  int n_e, prow0, rb, ks, kc0, nmain, next;
+  int tok0;  // first token (within the expert) of this tile's pass of up to NTOK tokens
 };
 struct Cnt {
   int it = 0;  // chunk (stage and A buffer) counter
@@ -114,10 +115,10 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
   const uint32_t full = bars + 8 * kBarFull, empty = bars + 8 * kBarEmpty;
   const int RB = a.M / kRows;
   constexpr int kBlk = (FMT == FMT_DENSE) ? 16384 : 128 * 8 * BITS;  // bytes of one code block (per plane: 1 KiB)
-  for (int p = 0; p < c.npass && !*abort_flag; ++p) {
-    const int n_pass = min(NTOK, c.n_e - p * NTOK);
+  {
+    const int n_pass = min(NTOK, c.n_e - c.tok0);
     const int nbox = (n_pass + kActBox - 1) / kActBox;
-    const int row0 = c.prow0 + p * NTOK;
+    const int row0 = c.prow0 + c.tok0;
     for (int i = 0; i < c.nmain + c.next; ++i, ++cnt.it) {
       const int slot = cnt.it % kStages;
       if (*abort_flag || !mbar_wait(empty + 8 * slot, ((cnt.it / kStages) & 1) ^ 1, a.status)) {
@@ -172,8 +173,8 @@ __device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int s
   const uint32_t full = bars + 8 * kBarFull, empty = bars + 8 * kBarEmpty;
   const uint32_t afull = bars + 8 * kBarAFull, aempty = bars + 8 * kBarAEmpty;
   const uint32_t accfull = bars + 8 * kBarAccFull, accfree = bars + 8 * kBarAccFree;
-  for (int p = 0; p < c.npass; ++p) {
-    const int n_pass = min(NTOK, c.n_e - p * NTOK);
+  {
+    const int n_pass = min(NTOK, c.n_e - c.tok0);
     const int npad = (n_pass + 15) & ~15;
     const uint32_t idesc = idesc_f16(128, npad);
     for (int i = 0; i < c.nmain + c.next; ++i, ++cnt.it) {
@@ -242,8 +243,8 @@ __device__ void dequant_epilogue(const DecodeArgs& a, const BlockDesc& d, const 
   if constexpr (FMT == FMT_BITPLANE) lut = load_lut(d.lut, BITS);
   const int RS2 = d.rank / 2;  // compensator column pairs
   constexpr int NH = NTOK / 2;
-  for (int p = 0; p < c.npass; ++p) {
-    const int n_pass = min(NTOK, c.n_e - p * NTOK);
+  {
+    const int n_pass = min(NTOK, c.n_e - c.tok0);
     float y[NH];
 #pragma unroll
     for (int t = 0; t < NH; ++t) y[t] = 0.f;
@@ -322,8 +323,8 @@ __device__ void dequant_epilogue(const DecodeArgs& a, const BlockDesc& d, const 
         return;
       }
     }
-    // ---- outputs of pass p: tokens p*NTOK + h*NH + t
-    const int tok0 = p * NTOK + h * NH;
+    // ---- outputs: tokens tok0 + t of this half
+    const int tok0 = c.tok0 + h * NH;
     const int nt = n_pass - h * NH;  // valid tokens of this half
     if (a.mode == MODE_SWIGLU) {
       // gate rows are lanes 16f..16f+7 of each 16-row group, up rows 8 lanes later
@@ -384,6 +385,7 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
   using RG = dk::Ring<NTOK>;
   __shared__ __align__(8) unsigned long long bars[dk::kNumBars];
   __shared__ float sscale[2 * 4 * dk::kRows];  // [token half][accumulator][row]: scale of a pending group
+  __shared__ int s_pre[kMaxExperts + 1];
   __shared__ int abort_flag;
   __shared__ uint32_t tmem_slot;
   const uint32_t b0 = smem_u32(bars);
@@ -422,23 +424,56 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
   // everything above overlaps the previous kernel's tail
   pdl_wait();
   pdl_trigger();
+  // Tiles: per active expert slot, (row block, K split, token pass) with the
+  // passes of one (row block, K split) adjacent, so that they run at about the
+  // same time and share the weight block through L2. s_pre = exclusive prefix
+  // of the token passes (ceil(n_e / NTOK)) over the slots.
   const int RB = a.M / dk::kRows;
-  const int total = *a.n_active * RB * a.KS;
+  const int per = RB * a.KS;
+  const int nact = *a.n_active;
+  if (warp == 0) {
+    const int lane = threadIdx.x & 31;
+    int loc[kMaxExperts / 32];
+    int sum = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j) {
+      const int sl = (kMaxExperts / 32) * lane + j;
+      loc[j] = sum;
+      sum += sl < nact ? (a.counts[a.active[sl]] + NTOK - 1) / NTOK : 0;
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j) s_pre[(kMaxExperts / 32) * lane + j] = incl - sum + loc[j];
+    if (lane == 31) s_pre[kMaxExperts] = incl;
+  }
+  __syncthreads();
+  const int total = s_pre[nact] * per;
   volatile int* ab = &abort_flag;
   dk::Cnt cnt;
   for (int tile = blockIdx.x; tile < total && !*ab; tile += gridDim.x) {
-    const int slot = tile / (RB * a.KS);
-    const int rem = tile % (RB * a.KS);
+    int lo = 0, hi = nact - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pre[mid] * per <= tile) lo = mid;
+      else hi = mid - 1;
+    }
+    const int slot = lo;
+    const int np = s_pre[slot + 1] - s_pre[slot];
+    const int local = tile - s_pre[slot] * per;
     const int e = a.active[slot];
     dk::Ctx c;
     c.n_e = a.counts[e];
-    if (c.n_e <= 0) continue;
     c.prow0 = a.poffsets[e];
-    c.rb = rem / a.KS;
-    c.ks = rem % a.KS;
+    c.tok0 = (local % np) * NTOK;
+    c.rb = (local / np) / a.KS;
+    c.ks = (local / np) % a.KS;
     const BlockDesc& d = a.experts[e].blk[a.block];
     c.next = (c.ks == 0 && d.rank > 0) ? 1 : 0;
-    c.npass = (c.n_e + NTOK - 1) / NTOK;
     c.kc0 = c.nmain = 0;
     bool ran = true;
     if (d.fmt == FMT_INT) {
@@ -524,7 +559,9 @@ static cudaError_t launch_ntok(const DecodeArgs& a, int maxbits, int grid_y, cud
   cudaError_t err = cudaFuncSetAttribute(decode_gemm_kernel<NTOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
   if (err != cudaSuccess) return err;
-  const long long tiles = (long long)grid_y * (a.M / dk::kRows) * a.KS;
+  // at most rows / NTOK + (one ragged pass per expert) token passes
+  const long long passes = std::min<long long>(a.rows / NTOK + grid_y, a.rows);
+  const long long tiles = passes * (a.M / dk::kRows) * a.KS;
   const int grid = (int)std::min<long long>(tiles, 2LL * num_sms());
   return launch_kernel(decode_gemm_kernel<NTOK>, dim3(grid), dim3(dk::kThreads), smem, st, true, a, stage_b,
                        dk::code_bytes(maxbits));

@@ -69,6 +69,7 @@ struct DecodeArgs {
   float* out;                 // MODE_OUT: [KS][prows][M] fp32 partials
   long long out_ks_stride;
   int KS;
+  long long rows;             // routed rows of the forward (host-side grid sizing)
   unsigned* status;
 };
 

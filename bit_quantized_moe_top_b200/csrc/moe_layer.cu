@@ -786,6 +786,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
       da.out = static_cast<float*>(L->obuf.p);
       da.out_ks_stride = prows * K;
       da.KS = KS;
+      da.rows = rows;
       da.status = ra.status;
       prof_mark(L, st, block == 0 ? "decode_gemm_w1_swiglu" : "decode_gemm_w2");
       ce = launch_decode_gemm(da, ntok, maxbits[block], grid_y, st, &launches);

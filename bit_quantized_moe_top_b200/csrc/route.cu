@@ -22,6 +22,7 @@ __device__ __forceinline__ bool better(float a, int ia, float b, int ib) {
 // The last CTA to finish (atomic ticket) scans the block histograms.
 __global__ void __launch_bounds__(kRouteThreads) route_topk_kernel(RouteArgs a) {
   __shared__ int hist[kMaxExperts];
+  __shared__ int seg[kMaxExperts > kRouteThreads ? kMaxExperts : kRouteThreads];  // per-(expert, segment) sums
   __shared__ int is_last;
   pdl_wait();
   pdl_trigger();
@@ -107,11 +108,28 @@ __global__ void __launch_bounds__(kRouteThreads) route_topk_kernel(RouteArgs a) 
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  // ---- last CTA: totals, offsets, padded offsets, per-block bases, active list
+  // ---- last CTA: totals, offsets, padded offsets, per-block bases, active list.
+  // Thread (e, s) owns a contiguous segment of the token blocks of expert e
+  // (S segments per expert), so long block lists are summed in parallel.
   const int nb = gridDim.x;
+  const int S = a.E >= kRouteThreads ? 1 : kRouteThreads / a.E;
+  const int bpseg = (nb + S - 1) / S;
+  for (int t = threadIdx.x; t < a.E * S; t += blockDim.x) {
+    const int e = t / S, sg = t % S;
+    const int b0 = min(nb, sg * bpseg), b1 = min(nb, b0 + bpseg);
+    int sum = 0;
+#pragma unroll 4
+    for (int b = b0; b < b1; ++b) sum += __ldcg(a.block_counts + (long long)b * a.E + e);
+    seg[t] = sum;
+  }
+  __syncthreads();
   for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
     int tot = 0;
-    for (int b = 0; b < nb; ++b) tot += __ldcg(a.block_counts + (long long)b * a.E + e);
+    for (int sg = 0; sg < S; ++sg) {
+      const int v = seg[e * S + sg];
+      seg[e * S + sg] = tot;  // exclusive prefix over the expert's segments
+      tot += v;
+    }
     hist[e] = tot;
   }
   __syncthreads();
@@ -132,9 +150,11 @@ __global__ void __launch_bounds__(kRouteThreads) route_topk_kernel(RouteArgs a) 
     *a.ticket = 0;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
-    int run = a.offsets[e], prun = a.poffsets[e];
-    for (int b = 0; b < nb; ++b) {
+  for (int t = threadIdx.x; t < a.E * S; t += blockDim.x) {
+    const int e = t / S, sg = t % S;
+    const int b0 = min(nb, sg * bpseg), b1 = min(nb, b0 + bpseg);
+    int run = a.offsets[e] + seg[t], prun = a.poffsets[e] + seg[t];
+    for (int b = b0; b < b1; ++b) {
       const long long i = (long long)b * a.E + e;
       const int c = __ldcg(a.block_counts + i);
       a.block_base[i] = run;
