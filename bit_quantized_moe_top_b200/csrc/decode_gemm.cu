@@ -55,7 +55,7 @@ namespace dk {
 constexpr int kDqWarps = 8;
 constexpr int kThreads = 32 * (kDqWarps + 2);
 constexpr int kRows = 128;
-constexpr int kStages = 4;
+constexpr int kMaxStages = 16;   // stage ring depth: as many as about 100 KiB of shared memory hold
 constexpr int kACols = 40;        // per A buffer: 32 code columns + 8 correction columns
 constexpr int kActBox = 16;       // rows per TMA box
 constexpr int kTmemCols = 256;
@@ -72,13 +72,14 @@ struct Ring {
   static constexpr int kABase = kAcc * NTOK <= 64 ? 64 : 128;
   static_assert(kABase + kA * kACols <= kTmemCols, "TMEM rings exceed the allocation");
 };
-// barrier slots (8 bytes each): full[kStages], empty[kStages], afull[4],
+// barrier slots (8 bytes each): full[stages], empty[stages], afull[4],
 // aempty[4], accfull[4], accfree[4], done
-constexpr int kBarFull = 0, kBarEmpty = kStages, kBarAFull = 2 * kStages, kBarAEmpty = kBarAFull + 4,
+constexpr int kBarFull = 0, kBarEmpty = kMaxStages, kBarAFull = 2 * kMaxStages, kBarAEmpty = kBarAFull + 4,
               kBarAccFull = kBarAEmpty + 4, kBarAccFree = kBarAccFull + 4, kBarDone = kBarAccFree + 4,
               kNumBars = kBarDone + 1;
 
-__host__ __device__ inline int code_bytes(int maxbits) { return maxbits >= 16 ? 16384 : 4096; }
+// code block bytes of a 128-row x 64-k chunk at the largest bitwidth of the block's experts
+__host__ __device__ inline int code_bytes(int maxbits) { return maxbits >= 16 ? 16384 : 1024 * maxbits; }
 // stage: [act NTOK x 128 B][corr NTOK x 32 B][codes][scales 512 B]
 __host__ __device__ inline int stage_bytes(int ntok, int maxbits) {
   const int b = ntok * 160 + code_bytes(maxbits) + 512;
@@ -120,8 +121,8 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
     const int nbox = (n_pass + kActBox - 1) / kActBox;
     const int row0 = c.prow0 + c.tok0;
     for (int i = 0; i < c.nmain + c.next; ++i, ++cnt.it) {
-      const int slot = cnt.it % kStages;
-      if (*abort_flag || !mbar_wait(empty + 8 * slot, ((cnt.it / kStages) & 1) ^ 1, a.status)) {
+      const int slot = cnt.it % a.nstages;
+      if (*abort_flag || !mbar_wait(empty + 8 * slot, ((cnt.it / a.nstages) & 1) ^ 1, a.status)) {
         *abort_flag = 1;
         return;
       }
@@ -162,8 +163,8 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
 
 // every issued stage must land before the CTA may exit
 __device__ void producer_drain(const DecodeArgs& a, uint32_t bars, const Cnt& cnt) {
-  for (int k = max(0, cnt.it - kStages); k < cnt.it; ++k)
-    if (!mbar_wait(bars + 8 * (k % kStages), (k / kStages) & 1, a.status)) break;
+  for (int k = max(0, cnt.it - a.nstages); k < cnt.it; ++k)
+    if (!mbar_wait(bars + 8 * (kBarFull + k % a.nstages), (k / a.nstages) & 1, a.status)) break;
 }
 
 template <int NTOK, int FMT, int GROUP>
@@ -178,11 +179,11 @@ __device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int s
     const int npad = (n_pass + 15) & ~15;
     const uint32_t idesc = idesc_f16(128, npad);
     for (int i = 0; i < c.nmain + c.next; ++i, ++cnt.it) {
-      const int slot = cnt.it % kStages, buf = cnt.it % RG::kA;
+      const int slot = cnt.it % a.nstages, buf = cnt.it % RG::kA;
       bool first, last;
       group_pos<FMT, GROUP>(c, i, first, last);
       const int ab = cnt.gc % RG::kAcc;
-      if (*abort_flag || !mbar_wait(full + 8 * slot, (cnt.it / kStages) & 1, a.status) ||
+      if (*abort_flag || !mbar_wait(full + 8 * slot, (cnt.it / a.nstages) & 1, a.status) ||
           !mbar_wait(afull + 8 * buf, (cnt.it / RG::kA) & 1, a.status) ||
           (first && !mbar_wait(accfree + 8 * ab, ((cnt.gc / RG::kAcc) & 1) ^ 1, a.status))) {
         *abort_flag = 1;
@@ -253,11 +254,11 @@ __device__ void dequant_epilogue(const DecodeArgs& a, const BlockDesc& d, const 
     int npend = 0;
     float s_cur = 1.f;
     for (int i = 0; i < c.nmain + c.next; ++i, ++cnt.it) {
-      const int slot = cnt.it % kStages, buf = cnt.it % RG::kA;
+      const int slot = cnt.it % a.nstages, buf = cnt.it % RG::kA;
       bool first, last;
       group_pos<FMT, GROUP>(c, i, first, last);
       // warp-uniform waits: every lane must reach the .sync.aligned TMEM stores
-      const bool ok = !*abort_flag && mbar_wait(full + 8 * slot, (cnt.it / kStages) & 1, a.status) &&
+      const bool ok = !*abort_flag && mbar_wait(full + 8 * slot, (cnt.it / a.nstages) & 1, a.status) &&
                       mbar_wait(aempty + 8 * buf, ((cnt.it / RG::kA) & 1) ^ 1, a.status);
       if (!__all_sync(0xffffffffu, ok)) {
         *abort_flag = 1;
@@ -392,7 +393,7 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
   const uint32_t done_bar = b0 + 8 * dk::kBarDone;
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < dk::kStages; ++i) {
+    for (int i = 0; i < a.nstages; ++i) {
       mbar_init(b0 + 8 * (dk::kBarFull + i), 1);                  // producer arrival + tx bytes
       mbar_init(b0 + 8 * (dk::kBarEmpty + i), dk::kDqWarps + 1);  // dequant warps + MMA commit
     }
@@ -554,8 +555,11 @@ static int num_sms() {
 template <int NTOK>
 static cudaError_t launch_ntok(const DecodeArgs& a, int maxbits, int grid_y, cudaStream_t st) {
   const int stage_b = dk::stage_bytes(NTOK, maxbits);
-  // at least 80 KiB so that at most two CTAs (2 x 256 TMEM columns) share an SM
-  const size_t smem = std::max<size_t>((size_t)dk::kStages * stage_b + 1024, 80 * 1024);
+  // two CTAs per SM (2 x 256 TMEM columns): each takes about 100 KiB of
+  // stages, as deep a ring as fits, to keep enough weight bytes in flight
+  DecodeArgs b = a;
+  b.nstages = std::min(dk::kMaxStages, (100 * 1024 - 1024) / stage_b);
+  const size_t smem = (size_t)b.nstages * stage_b + 1024;
   cudaError_t err = cudaFuncSetAttribute(decode_gemm_kernel<NTOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
   if (err != cudaSuccess) return err;
@@ -563,7 +567,7 @@ static cudaError_t launch_ntok(const DecodeArgs& a, int maxbits, int grid_y, cud
   const long long passes = std::min<long long>(a.rows / NTOK + grid_y, a.rows);
   const long long tiles = passes * (a.M / dk::kRows) * a.KS;
   const int grid = (int)std::min<long long>(tiles, 2LL * num_sms());
-  return launch_kernel(decode_gemm_kernel<NTOK>, dim3(grid), dim3(dk::kThreads), smem, st, true, a, stage_b,
+  return launch_kernel(decode_gemm_kernel<NTOK>, dim3(grid), dim3(dk::kThreads), smem, st, true, b, stage_b,
                        dk::code_bytes(maxbits));
 }
 

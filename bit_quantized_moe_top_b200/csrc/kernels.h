@@ -70,6 +70,7 @@ struct DecodeArgs {
   long long out_ks_stride;
   int KS;
   long long rows;             // routed rows of the forward (host-side grid sizing)
+  int nstages;                // shared-memory stages of the ring (set by the launcher)
   unsigned* status;
 };
 
