@@ -197,6 +197,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
     }
   }
 }
+// Probe of a phase without a suspend hint (a completed phase returns at once).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// The bounded wait, out of line: only taken when the phase is still open.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, unsigned* status) {
+  return mbar_wait(bar, parity, status);
+}
+// Bounded wait with an inlined fast path.
+__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, unsigned* status) {
+  return mbar_test(bar, parity) || mbar_wait_slow(bar, parity, status);
+}
+
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),

@@ -2,20 +2,26 @@
 // 5th-generation tensor cores with the unpacked weights in TMEM.
 //
 // The decode matmuls stream weights: every packed code is read once per
-// token pass, so the kernel is bound by HBM bandwidth and by the ALU work of
-// unpacking. A CTA owns 128 weight rows of one expert (one row per TMEM
-// lane) and a group-aligned range of 64-wide K chunks; CTAs are persistent
-// and walk the (expert, row block, K split) tiles round-robin.
+// token pass, so the kernel is bound by HBM bandwidth and by the instruction
+// work of unpacking. A CTA owns 128 weight rows of one expert (one row per
+// TMEM lane) and a group-aligned range of 64-wide K chunks; CTAs are
+// persistent and walk the (expert, row block, K split, token pass) tiles.
 //   warp 8     producer: per chunk, the 128 rows' packed codes (one contiguous
-//              block), at a group's first chunk its scales and zero points
-//              and the routed rows' correction columns, and the expert's
+//              block), at a group's first chunk the routed rows' correction
+//              columns and the group's scale/zero pairs, and the expert's
 //              routed activation rows (TMA 2-D boxes of 16 rows, no multicast);
-//   warps 0-7  two threads per weight row (warps w and w+4 share TMEM lane
-//              quarter w, one K half each) unpack the codes in registers and
-//              store them into a TMEM buffer (tcgen05.st), the MMA's A operand;
+//   warps 0-3  unpack: one thread per weight row turns the row's 64 codes into
+//              32 fp16 pairs in registers and stores them into a TMEM buffer
+//              (one tcgen05.st), the MMA's A operand;
 //   warp 9     allocates TMEM and issues tcgen05.mma kind::f16 with A from
 //              TMEM (M = 128 weight rows), B = activations from shared memory
-//              (N = tokens, 16..64), D in TMEM.
+//              (N = tokens, 16 or 32), D in TMEM;
+//   warps 4-7  epilogue: per quantisation group, y += s * acc in fp32
+//              registers; at the end of the tile SwiGLU or fp32 output rows.
+// Every hand-off is an mbarrier; a warp's work per chunk is kept to a few
+// dozen instructions (ring positions advance incrementally, waits have an
+// inlined fast path), since that instruction stream, not the tensor core,
+// sets the pace.
 //
 // Integer codes are not dequantised per weight. The A operand holds the raw
 // fp16 values P_k + q_k of the exponent-bias unpack (exact small integers
@@ -27,10 +33,9 @@
 // columns are (1024, 1024, z_g, z_g, 0...) and whose B columns are the
 // routed row's precomputed sums XP_g = sum (P_k/1024) x_k and X_g = sum x_k,
 // each split into fp16 value + fp16 remainder. The epilogue of a group is
-// y += s_g * acc_g in fp32 registers (two threads per row, one half of the
-// tokens each). Per pair of weights this leaves one or two logic ops and no
-// fp16 arithmetic. Bit-plane (LUT) and dense blocks store their fp16 weight
-// values as A and use one accumulator for the whole K range.
+// y += s_g * acc_g. Per pair of weights this leaves one or two logic ops and
+// no fp16 arithmetic. Bit-plane (LUT) and dense blocks store their fp16
+// weight values as A and use one accumulator for the whole K range.
 //
 // The rank-r compensator is one more 64-wide stage (its own accumulator,
 // scale 1): the B factor's row values as A against the U = A x columns stored
@@ -52,30 +57,24 @@
 namespace moeq {
 namespace dk {
 
-constexpr int kDqWarps = 8;
-constexpr int kThreads = 32 * (kDqWarps + 2);
+constexpr int kDqWarps = 4;
+constexpr int kEpWarps = 4;
+constexpr int kProdWarp = kDqWarps + kEpWarps, kMmaWarp = kProdWarp + 1;
+constexpr int kThreads = 32 * (kMmaWarp + 1);
 constexpr int kRows = 128;
-constexpr int kMaxStages = 16;   // stage ring depth: as many as about 100 KiB of shared memory hold
-constexpr int kACols = 40;        // per A buffer: 32 code columns + 8 correction columns
-constexpr int kActBox = 16;       // rows per TMA box
+constexpr int kMaxStages = 16;  // stage ring depth: as many as about 100 KiB of shared memory hold
+constexpr int kA = 3;           // TMEM A buffers
+constexpr int kAcc = 2;         // TMEM accumulators
+constexpr int kACols = 40;      // per A buffer: 32 code columns + 8 correction columns
+constexpr int kABase = 128;     // accumulators at [0, kAcc * NTOK), A buffers at [128, 248)
 constexpr int kTmemCols = 256;
+constexpr int kActBox = 16;     // rows per TMA box
 constexpr uint32_t kOne1024 = 0x64006400u;  // fp16 pair (1024, 1024)
+static_assert(kABase + kA * kACols <= kTmemCols, "TMEM rings exceed the allocation");
 
-// TMEM rings: accumulators at [0, kAcc * NTOK), A buffers from kABase. The
-// rings are as deep as 256 columns allow, so that the MMA round trip (issue,
-// completion, mbarrier) of a chunk or a group is covered by the unpacking of
-// the next ones; a group's epilogue runs kAcc - 1 groups after its last chunk.
-template <int NTOK>
-struct Ring {
-  static constexpr int kAcc = NTOK <= 32 ? 4 : 2;
-  static constexpr int kA = NTOK <= 16 ? 4 : 3;
-  static constexpr int kABase = kAcc * NTOK <= 64 ? 64 : 128;
-  static_assert(kABase + kA * kACols <= kTmemCols, "TMEM rings exceed the allocation");
-};
-// barrier slots (8 bytes each): full[stages], empty[stages], afull[4],
-// aempty[4], accfull[4], accfree[4], done
-constexpr int kBarFull = 0, kBarEmpty = kMaxStages, kBarAFull = 2 * kMaxStages, kBarAEmpty = kBarAFull + 4,
-              kBarAccFull = kBarAEmpty + 4, kBarAccFree = kBarAccFull + 4, kBarDone = kBarAccFree + 4,
+// barrier slots (8 bytes each)
+constexpr int kBarFull = 0, kBarEmpty = kMaxStages, kBarAFull = 2 * kMaxStages, kBarAEmpty = kBarAFull + kA,
+              kBarAccFull = kBarAEmpty + kA, kBarAccFree = kBarAccFull + kAcc, kBarDone = kBarAccFree + kAcc,
               kNumBars = kBarDone + 1;
 
 // code block bytes of a 128-row x 64-k chunk at the largest bitwidth of the block's experts
@@ -86,16 +85,33 @@ __host__ __device__ inline int stage_bytes(int ntok, int maxbits) {
   return (b + 1023) & ~1023;
 }
 
+// position in a ring of n slots with the phase parity of the current lap
+struct RingPos {
+  int idx = 0;
+  uint32_t ph = 0;
+  __device__ __forceinline__ void next(int n) {
+    if (++idx == n) {
+      idx = 0;
+      ph ^= 1u;
+    }
+  }
+};
+
 struct Ctx {
   int n_e, prow0, rb, ks, kc0, nmain, next;
   int tok0;  // first token (within the expert) of this tile's pass of up to NTOK tokens
 };
-struct Cnt {
-  int it = 0;  // chunk (stage and A buffer) counter
-  int gc = 0;  // accumulator group counter
+
+// per-role ring positions, kept across tiles
+struct Pos {
+  RingPos st;   // stage ring
+  RingPos rel;  // stage to release (unpack warps: kA chunks behind st)
+  RingPos ab;   // A buffer ring
+  RingPos acc;  // accumulator ring
+  int chunks = 0;
 };
 
-// group position of chunk i of a pass: first / last chunk of its accumulator group
+// group position of chunk i of a tile: first / last chunk of its accumulator group
 template <int FMT, int GROUP>
 __device__ __forceinline__ void group_pos(const Ctx& c, int i, bool& first, bool& last) {
   if (i >= c.nmain) {
@@ -112,247 +128,227 @@ __device__ __forceinline__ void group_pos(const Ctx& c, int i, bool& first, bool
 
 template <int NTOK, int FMT, int BITS, int GROUP>
 __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, uint8_t* sm, int stage_b, int cbytes,
-                         uint32_t bars, Cnt& cnt, volatile int* abort_flag) {
+                         uint32_t bars, Pos& ps, volatile int* abort_flag) {
   const uint32_t full = bars + 8 * kBarFull, empty = bars + 8 * kBarEmpty;
   const int RB = a.M / kRows;
   constexpr int kBlk = (FMT == FMT_DENSE) ? 16384 : 128 * 8 * BITS;  // bytes of one code block (per plane: 1 KiB)
-  {
-    const int n_pass = min(NTOK, c.n_e - c.tok0);
-    const int nbox = (n_pass + kActBox - 1) / kActBox;
-    const int row0 = c.prow0 + c.tok0;
-    for (int i = 0; i < c.nmain + c.next; ++i, ++cnt.it) {
-      const int slot = cnt.it % a.nstages;
-      if (*abort_flag || !mbar_wait(empty + 8 * slot, ((cnt.it / a.nstages) & 1) ^ 1, a.status)) {
-        *abort_flag = 1;
-        return;
-      }
-      bool first, last;
-      group_pos<FMT, GROUP>(c, i, first, last);
-      uint8_t* st = sm + slot * stage_b;
-      const bool main = i < c.nmain;
-      const int kc = c.kc0 + i;
-      const bool corr = FMT == FMT_INT && main && first;
-      uint32_t bytes = nbox * kActBox * 128;
-      if (main) bytes += (FMT == FMT_BITPLANE ? BITS * 1024 : kBlk);
-      if (corr) bytes += nbox * kActBox * 32 + 512;
-      mbar_expect_tx(full + 8 * slot, bytes);
-      const int kx = main ? kc * 64 : a.K;
-      for (int b = 0; b < nbox; ++b)
-        tma_load_2d(smem_u32(st + b * kActBox * 128), &a.tmap_act, kx, row0 + b * kActBox, full + 8 * slot);
-      if (main) {
-        uint8_t* cs = st + NTOK * 160;
-        const long long bidx = (long long)kc * RB + c.rb;
-        if constexpr (FMT == FMT_BITPLANE) {
+  const int n_pass = min(NTOK, c.n_e - c.tok0);
+  const int nbox = (n_pass + kActBox - 1) / kActBox;
+  const int row0 = c.prow0 + c.tok0;
+  const uint8_t* codes = (FMT == FMT_BITPLANE) ? d.plane[0] : d.codes;
+  for (int i = 0; i < c.nmain + c.next; ++i, ps.st.next(a.nstages)) {
+    if (*abort_flag || !mbar_wait_fast(empty + 8 * ps.st.idx, ps.st.ph ^ 1u, a.status)) {
+      *abort_flag = 1;
+      return;
+    }
+    bool first, last;
+    group_pos<FMT, GROUP>(c, i, first, last);
+    uint8_t* st = sm + ps.st.idx * stage_b;
+    const uint32_t fb = full + 8 * ps.st.idx;
+    const bool main = i < c.nmain;
+    const int kc = c.kc0 + i;
+    const bool corr = FMT == FMT_INT && main && first;
+    uint32_t bytes = nbox * kActBox * 128;
+    if (main) bytes += (FMT == FMT_BITPLANE ? BITS * 1024 : kBlk);
+    if (corr) bytes += nbox * kActBox * 32 + 512;
+    mbar_expect_tx(fb, bytes);
+    const int kx = main ? kc * 64 : a.K;
+    for (int b = 0; b < nbox; ++b)
+      tma_load_2d(smem_u32(st + b * kActBox * 128), &a.tmap_act, kx, row0 + b * kActBox, fb);
+    if (main) {
+      uint8_t* cs = st + NTOK * 160;
+      const long long bidx = (long long)kc * RB + c.rb;
+      if constexpr (FMT == FMT_BITPLANE) {
 #pragma unroll
-          for (int q = 0; q < BITS; ++q)
-            bulk_g2s(smem_u32(cs + q * 1024), d.plane[q] + bidx * 1024, 1024, full + 8 * slot);
-        } else {
-          bulk_g2s(smem_u32(cs), d.codes + bidx * kBlk, kBlk, full + 8 * slot);
-        }
-        if (corr) {
-          const int g = kc * 64 / GROUP;
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d(smem_u32(st + NTOK * 128 + b * kActBox * 32), &a.tmap_corr, 16 * g, row0 + b * kActBox,
-                        full + 8 * slot);
-          bulk_g2s(smem_u32(cs + cbytes), d.sz + (long long)g * a.M + c.rb * kRows, 512, full + 8 * slot);
-        }
+        for (int q = 0; q < BITS; ++q) bulk_g2s(smem_u32(cs + q * 1024), d.plane[q] + bidx * 1024, 1024, fb);
+      } else {
+        bulk_g2s(smem_u32(cs), codes + bidx * kBlk, kBlk, fb);
+      }
+      if (corr) {
+        const int g = kc * 64 / GROUP;
+        for (int b = 0; b < nbox; ++b)
+          tma_load_2d(smem_u32(st + NTOK * 128 + b * kActBox * 32), &a.tmap_corr, 16 * g, row0 + b * kActBox, fb);
+        bulk_g2s(smem_u32(cs + cbytes), d.sz + (long long)g * a.M + c.rb * kRows, 512, fb);
       }
     }
   }
-}
-
-// every issued stage must land before the CTA may exit
-__device__ void producer_drain(const DecodeArgs& a, uint32_t bars, const Cnt& cnt) {
-  for (int k = max(0, cnt.it - a.nstages); k < cnt.it; ++k)
-    if (!mbar_wait(bars + 8 * (kBarFull + k % a.nstages), (k / a.nstages) & 1, a.status)) break;
 }
 
 template <int NTOK, int FMT, int GROUP>
 __device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int stage_b, uint32_t bars, uint32_t tmem,
-                           Cnt& cnt, volatile int* abort_flag) {
-  using RG = Ring<NTOK>;
-  const uint32_t full = bars + 8 * kBarFull, empty = bars + 8 * kBarEmpty;
+                           Pos& ps, volatile int* abort_flag) {
+  const uint32_t full = bars + 8 * kBarFull;
   const uint32_t afull = bars + 8 * kBarAFull, aempty = bars + 8 * kBarAEmpty;
   const uint32_t accfull = bars + 8 * kBarAccFull, accfree = bars + 8 * kBarAccFree;
-  {
-    const int n_pass = min(NTOK, c.n_e - c.tok0);
-    const int npad = (n_pass + 15) & ~15;
-    const uint32_t idesc = idesc_f16(128, npad);
-    for (int i = 0; i < c.nmain + c.next; ++i, ++cnt.it) {
-      const int slot = cnt.it % a.nstages, buf = cnt.it % RG::kA;
-      bool first, last;
-      group_pos<FMT, GROUP>(c, i, first, last);
-      const int ab = cnt.gc % RG::kAcc;
-      if (*abort_flag || !mbar_wait(full + 8 * slot, (cnt.it / a.nstages) & 1, a.status) ||
-          !mbar_wait(afull + 8 * buf, (cnt.it / RG::kA) & 1, a.status) ||
-          (first && !mbar_wait(accfree + 8 * ab, ((cnt.gc / RG::kAcc) & 1) ^ 1, a.status))) {
-        *abort_flag = 1;
-        return;
-      }
-      tc_fence_after();
-      const uint32_t bt = smem_u32(sm + slot * stage_b);
-      const uint32_t acc = tmem + ab * NTOK;
-      const uint32_t ta = tmem + RG::kABase + buf * kACols;
-      const bool corr = FMT == FMT_INT && i < c.nmain && first;
-      if (corr) mma_f16_ts(acc, ta + 32, sw32_desc(bt + NTOK * 128), idesc, 0);
-#pragma unroll
-      for (int k16 = 0; k16 < 4; ++k16)
-        mma_f16_ts(acc, ta + k16 * 8, sw128_desc(bt + k16 * 32), idesc, (corr || !first || k16 > 0) ? 1 : 0);
-      mma_commit(empty + 8 * slot);
-      mma_commit(aempty + 8 * buf);
-      if (last) {
-        mma_commit(accfull + 8 * ab);
-        ++cnt.gc;
-      }
+  const int n_pass = min(NTOK, c.n_e - c.tok0);
+  const uint32_t idesc = idesc_f16(128, (n_pass + 15) & ~15);
+  const uint32_t sm0 = smem_u32(sm);
+  for (int i = 0; i < c.nmain + c.next; ++i) {
+    bool first, last;
+    group_pos<FMT, GROUP>(c, i, first, last);
+    if (*abort_flag || !mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status) ||
+        !mbar_wait_fast(afull + 8 * ps.ab.idx, ps.ab.ph, a.status) ||
+        (first && !mbar_wait_fast(accfree + 8 * ps.acc.idx, ps.acc.ph ^ 1u, a.status))) {
+      *abort_flag = 1;
+      return;
     }
+    tc_fence_after();
+    const uint32_t bt = sm0 + ps.st.idx * stage_b;
+    const uint32_t acc = tmem + ps.acc.idx * NTOK;
+    const uint32_t ta = tmem + kABase + ps.ab.idx * kACols;
+    const bool corr = FMT == FMT_INT && i < c.nmain && first;
+    if (corr) mma_f16_ts(acc, ta + 32, sw32_desc(bt + NTOK * 128), idesc, 0);
+#pragma unroll
+    for (int k16 = 0; k16 < 4; ++k16)
+      mma_f16_ts(acc, ta + k16 * 8, sw128_desc(bt + k16 * 32), idesc, (corr || !first || k16 > 0) ? 1 : 0);
+    mma_commit(aempty + 8 * ps.ab.idx);
+    if (last) {
+      mma_commit(accfull + 8 * ps.acc.idx);
+      ps.acc.next(kAcc);
+    }
+    ps.st.next(a.nstages);
+    ps.ab.next(kA);
   }
 }
 
-// y[t] += scale * acc[t] for this thread's half of the tokens of group gq
-template <int NTOK>
-__device__ __forceinline__ bool group_epilogue(const DecodeArgs& a, uint32_t bars, uint32_t tmem, uint32_t lane_base,
-                                               int h, int gq, float scale, float (&y)[NTOK / 2]) {
-  using RG = Ring<NTOK>;
-  const uint32_t accfull = bars + 8 * kBarAccFull, accfree = bars + 8 * kBarAccFree;
-  const int ab = gq % RG::kAcc;
-  if (!__all_sync(0xffffffffu, mbar_wait(accfull + 8 * ab, (gq / RG::kAcc) & 1, a.status))) return false;
-  tc_fence_after();
-  uint32_t v[NTOK / 2];
-  tmem_ld<NTOK / 2>(tmem + lane_base + ab * NTOK + h * (NTOK / 2), v);
-#pragma unroll
-  for (int t = 0; t < NTOK / 2; ++t) y[t] = fmaf(scale, __uint_as_float(v[t]), y[t]);
-  tc_fence_before();
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(accfree + 8 * ab);
-  return true;
-}
-
 template <int NTOK, int FMT, int BITS, int GROUP>
-__device__ void dequant_epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, uint8_t* sm, int stage_b,
-                                 int cbytes, uint32_t bars, uint32_t tmem, Cnt& cnt, volatile int* abort_flag,
-                                 float* sscale) {
-  using RG = Ring<NTOK>;
-  constexpr int kDefer = RG::kAcc - 1;  // groups between a group's last chunk and its epilogue
+__device__ void unpack(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, uint8_t* sm, int stage_b, int cbytes,
+                       uint32_t bars, uint32_t tmem, Pos& ps, volatile int* abort_flag) {
   const uint32_t full = bars + 8 * kBarFull, empty = bars + 8 * kBarEmpty;
   const uint32_t afull = bars + 8 * kBarAFull, aempty = bars + 8 * kBarAEmpty;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q = warp & 3, h = warp >> 2;      // TMEM lane quarter, K half / token half
-  const int row = q * 32 + lane;              // TMEM lane
-  const int R = c.rb * kRows + row;           // internal row of the block
-  const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+  const int lane = threadIdx.x & 31;
+  const int row = threadIdx.x;  // 0..127 = TMEM lane
+  const uint32_t lane_base = (uint32_t)(row & ~31) << 16;
   LutRegs lut;
   if constexpr (FMT == FMT_BITPLANE) lut = load_lut(d.lut, BITS);
   const int RS2 = d.rank / 2;  // compensator column pairs
-  constexpr int NH = NTOK / 2;
-  {
-    const int n_pass = min(NTOK, c.n_e - c.tok0);
-    float y[NH];
+  const int R = c.rb * kRows + row;
+  for (int i = 0; i < c.nmain + c.next; ++i) {
+    bool first, last;
+    group_pos<FMT, GROUP>(c, i, first, last);
+    // warp-uniform waits: every lane reaches the .sync.aligned TMEM stores
+    const bool ok = !*abort_flag && mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status) &&
+                    mbar_wait_fast(aempty + 8 * ps.ab.idx, ps.ab.ph ^ 1u, a.status);
+    if (!__all_sync(0xffffffffu, ok)) {
+      *abort_flag = 1;
+      return;
+    }
+    // the MMAs of chunk (this - kA) are complete: its stage (codes read by
+    // these warps, activations read by the MMAs) may be refilled
+    if (ps.chunks >= kA) {
+      if (lane == 0) mbar_arrive(empty + 8 * ps.rel.idx);
+      ps.rel.next(a.nstages);
+    }
+    const uint32_t ta = tmem + lane_base + kABase + ps.ab.idx * kACols;
+    uint32_t v[32];
+    if (i < c.nmain) {
+      const uint8_t* cs = sm + ps.st.idx * stage_b + NTOK * 160;
+      if constexpr (FMT == FMT_INT) {
+        if (first) {
+          const uint32_t sz = reinterpret_cast<const uint32_t*>(cs + cbytes)[row];
+          tmem_st1_nw(ta + 33, prmt(sz, sz, 0x3232u));  // (z, z) against (-X_hi, -X_lo)
+        }
 #pragma unroll
-    for (int t = 0; t < NH; ++t) y[t] = 0.f;
-    // groups whose epilogue is pending: cnt.gc - npend .. cnt.gc - 1; their
-    // scales wait in shared memory, one slot per accumulator
-    int npend = 0;
-    float s_cur = 1.f;
-    for (int i = 0; i < c.nmain + c.next; ++i, ++cnt.it) {
-      const int slot = cnt.it % a.nstages, buf = cnt.it % RG::kA;
-      bool first, last;
-      group_pos<FMT, GROUP>(c, i, first, last);
-      // warp-uniform waits: every lane must reach the .sync.aligned TMEM stores
-      const bool ok = !*abort_flag && mbar_wait(full + 8 * slot, (cnt.it / a.nstages) & 1, a.status) &&
-                      mbar_wait(aempty + 8 * buf, ((cnt.it / RG::kA) & 1) ^ 1, a.status);
-      if (!__all_sync(0xffffffffu, ok)) {
-        *abort_flag = 1;
-        return;
-      }
-      const uint32_t ta = tmem + lane_base + RG::kABase + buf * kACols;
-      uint32_t v[16];
-      const bool main = i < c.nmain;
-      if (main) {
-        const uint8_t* cs = sm + slot * stage_b + NTOK * 160;
-        if constexpr (FMT == FMT_INT) {
-          if (first) {
-            const uint32_t sz = reinterpret_cast<const uint32_t*>(cs + cbytes)[row];
-            s_cur = __half2float(__ushort_as_half((uint16_t)(sz & 0xFFFFu)));
-            if (h == 0) tmem_st1_nw(ta + 33, prmt(sz, sz, 0x3232u));  // (z, z) against (-X_hi, -X_lo)
-          }
-          uint32_t w[4];
+        for (int h = 0; h < 2; ++h) {
+          uint32_t w[4], r16[16];
           load_half_words_int<BITS>(cs, row, h, w);
-          int_raw_half<BITS>(w, v);
-        } else if constexpr (FMT == FMT_BITPLANE) {
-          uint32_t pw[4];
-          load_half_planes<BITS>(cs, 1024, row, h, pw);
-          lut_half<BITS>(pw, lut, v);
-        } else {
+          int_raw_half<BITS>(w, r16);
 #pragma unroll
-          for (int qd = 0; qd < 4; ++qd) {
-            const uint4 x = reinterpret_cast<const uint4*>(cs + (4 * h + qd) * 2048)[row];
-            v[4 * qd] = x.x; v[4 * qd + 1] = x.y; v[4 * qd + 2] = x.z; v[4 * qd + 3] = x.w;
-          }
+          for (int j = 0; j < 16; ++j) v[16 * h + j] = r16[j];
+        }
+      } else if constexpr (FMT == FMT_BITPLANE) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pw[4], r16[16];
+          load_half_planes<BITS>(cs, 1024, row, h, pw);
+          lut_half<BITS>(pw, lut, r16);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[16 * h + j] = r16[j];
         }
       } else {
-        // compensator stage: the row's B values (pairs), zero past the rank
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = (16 * h + j) < RS2 ? d.brow[(long long)(16 * h + j) * a.M + R] : 0u;
-      }
-      tmem_st16_nw(ta + 16 * h, v);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(afull + 8 * buf);
-        mbar_arrive(empty + 8 * slot);
-      }
-      // the oldest pending group's accumulator, kDefer groups behind the MMAs
-      if (npend == kDefer) {
-        const int gq = cnt.gc - npend;
-        if (!group_epilogue<NTOK>(a, bars, tmem, lane_base, h, gq, sscale[(h * 4 + gq % RG::kAcc) * kRows + row], y)) {
-          *abort_flag = 1;
-          return;
-        }
-        --npend;
-      }
-      if (last) {
-        sscale[(h * 4 + cnt.gc % RG::kAcc) * kRows + row] = (FMT == FMT_INT && main) ? s_cur : 1.f;
-        ++npend;
-        ++cnt.gc;
-      }
-    }
-    for (; npend > 0; --npend) {
-      const int gq = cnt.gc - npend;
-      if (!group_epilogue<NTOK>(a, bars, tmem, lane_base, h, gq, sscale[(h * 4 + gq % RG::kAcc) * kRows + row], y)) {
-        *abort_flag = 1;
-        return;
-      }
-    }
-    // ---- outputs: tokens tok0 + t of this half
-    const int tok0 = c.tok0 + h * NH;
-    const int nt = n_pass - h * NH;  // valid tokens of this half
-    if (a.mode == MODE_SWIGLU) {
-      // gate rows are lanes 16f..16f+7 of each 16-row group, up rows 8 lanes later
-      float up[NH];
-#pragma unroll
-      for (int t = 0; t < NH; ++t) up[t] = __shfl_down_sync(0xffffffffu, y[t], 8);
-      if ((R & 15) < 8) {
-        const int col = 8 * (R >> 4) + (R & 7);
-#pragma unroll
-        for (int t = 0; t < NH; ++t) {
-          if (t < nt) {
-            const float gt = y[t];
-            a.zout[(long long)(c.prow0 + tok0 + t) * a.ldz + col] = __float2half_rn(gt / (1.f + expf(-gt)) * up[t]);
-          }
+        for (int qd = 0; qd < 8; ++qd) {
+          const uint4 x = reinterpret_cast<const uint4*>(cs + qd * 2048)[row];
+          v[4 * qd] = x.x; v[4 * qd + 1] = x.y; v[4 * qd + 2] = x.z; v[4 * qd + 3] = x.w;
         }
       }
     } else {
+      // compensator stage: the row's B values (pairs), zero past the rank
 #pragma unroll
-      for (int t = 0; t < NH; ++t)
-        if (t < nt) a.out[c.ks * a.out_ks_stride + (long long)(c.prow0 + tok0 + t) * a.M + R] = y[t];
+      for (int j = 0; j < 32; ++j) v[j] = j < RS2 ? d.brow[(long long)j * a.M + R] : 0u;
     }
+    tmem_st32(ta, v);  // includes the wait for the store
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(afull + 8 * ps.ab.idx);
+    ps.st.next(a.nstages);
+    ps.ab.next(kA);
+    ++ps.chunks;
+  }
+}
+
+template <int NTOK, int FMT, int GROUP>
+__device__ void epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, uint32_t bars, uint32_t tmem,
+                         Pos& ps, volatile int* abort_flag) {
+  const uint32_t accfull = bars + 8 * kBarAccFull, accfree = bars + 8 * kBarAccFree;
+  const int lane = threadIdx.x & 31;
+  const int row = threadIdx.x - 32 * kDqWarps;  // 0..127 = TMEM lane
+  const uint32_t lane_base = (uint32_t)(row & ~31) << 16;
+  const int R = c.rb * kRows + row;
+  int nmain_groups = 0;
+  if constexpr (FMT == FMT_INT) nmain_groups = c.nmain / (GROUP / 64);
+  else nmain_groups = c.nmain > 0 ? 1 : 0;
+  const int g0 = (FMT == FMT_INT) ? c.kc0 / (GROUP / 64) : 0;
+  float y[NTOK];
+#pragma unroll
+  for (int t = 0; t < NTOK; ++t) y[t] = 0.f;
+  for (int gi = 0; gi < nmain_groups + c.next; ++gi) {
+    float s = 1.f;
+    if (FMT == FMT_INT && gi < nmain_groups) {
+      const uint32_t sz = d.sz[(long long)(g0 + gi) * a.M + R];
+      s = __half2float(__ushort_as_half((uint16_t)(sz & 0xFFFFu)));
+    }
+    if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait_fast(accfull + 8 * ps.acc.idx, ps.acc.ph, a.status))) {
+      *abort_flag = 1;
+      return;
+    }
+    tc_fence_after();
+    uint32_t v[NTOK];
+    tmem_ld<NTOK>(tmem + lane_base + ps.acc.idx * NTOK, v);
+#pragma unroll
+    for (int t = 0; t < NTOK; ++t) y[t] = fmaf(s, __uint_as_float(v[t]), y[t]);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(accfree + 8 * ps.acc.idx);
+    ps.acc.next(kAcc);
+  }
+  // ---- outputs: tokens tok0 + t
+  const int nt = min(NTOK, c.n_e - c.tok0);
+  if (a.mode == MODE_SWIGLU) {
+    // gate rows are lanes 16f..16f+7 of each 16-row group, up rows 8 lanes later
+    float up[NTOK];
+#pragma unroll
+    for (int t = 0; t < NTOK; ++t) up[t] = __shfl_down_sync(0xffffffffu, y[t], 8);
+    if ((R & 15) < 8) {
+      const int col = 8 * (R >> 4) + (R & 7);
+#pragma unroll
+      for (int t = 0; t < NTOK; ++t) {
+        if (t < nt) {
+          const float gt = y[t];
+          a.zout[(long long)(c.prow0 + c.tok0 + t) * a.ldz + col] = __float2half_rn(gt / (1.f + expf(-gt)) * up[t]);
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int t = 0; t < NTOK; ++t)
+      if (t < nt) a.out[c.ks * a.out_ks_stride + (long long)(c.prow0 + c.tok0 + t) * a.M + R] = y[t];
   }
 }
 
 template <int NTOK, int FMT, int BITS, int GROUP>
 __device__ void decode_tile(const DecodeArgs& a, const BlockDesc& d, const Ctx& c0, uint8_t* sm, int stage_b,
-                            int cbytes, uint32_t bars, uint32_t tmem, Cnt& cnt, volatile int* ab, float* sscale) {
+                            int cbytes, uint32_t bars, uint32_t tmem, Pos& ps, volatile int* ab) {
   // group-aligned K range of this split
   Ctx c = c0;
   const int KC = a.K / 64;
@@ -368,11 +364,13 @@ __device__ void decode_tile(const DecodeArgs& a, const BlockDesc& d, const Ctx& 
   }
   const int warp = threadIdx.x >> 5;
   if (warp < kDqWarps) {
-    dequant_epilogue<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, tmem, cnt, ab, sscale);
-  } else if (warp == kDqWarps) {
-    if ((threadIdx.x & 31) == 0) producer<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, cnt, ab);
+    unpack<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, tmem, ps, ab);
+  } else if (warp < kProdWarp) {
+    epilogue<NTOK, FMT, GROUP>(a, d, c, bars, tmem, ps, ab);
+  } else if (warp == kProdWarp) {
+    if ((threadIdx.x & 31) == 0) producer<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, ps, ab);
   } else {
-    if ((threadIdx.x & 31) == 0) mma_issuer<NTOK, FMT, GROUP>(a, c, sm, stage_b, bars, tmem, cnt, ab);
+    if ((threadIdx.x & 31) == 0) mma_issuer<NTOK, FMT, GROUP>(a, c, sm, stage_b, bars, tmem, ps, ab);
   }
 }
 
@@ -383,9 +381,7 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
                                                                         int stage_b, int cbytes) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  using RG = dk::Ring<NTOK>;
   __shared__ __align__(8) unsigned long long bars[dk::kNumBars];
-  __shared__ float sscale[2 * 4 * dk::kRows];  // [token half][accumulator][row]: scale of a pending group
   __shared__ int s_pre[kMaxExperts + 1];
   __shared__ int abort_flag;
   __shared__ uint32_t tmem_slot;
@@ -395,33 +391,32 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
   if (threadIdx.x == 0) {
     for (int i = 0; i < a.nstages; ++i) {
       mbar_init(b0 + 8 * (dk::kBarFull + i), 1);                  // producer arrival + tx bytes
-      mbar_init(b0 + 8 * (dk::kBarEmpty + i), dk::kDqWarps + 1);  // dequant warps + MMA commit
+      mbar_init(b0 + 8 * (dk::kBarEmpty + i), dk::kDqWarps);      // unpack warps, after the stage's MMAs
     }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(b0 + 8 * (dk::kBarAFull + i), dk::kDqWarps);    // A buffer written
-      mbar_init(b0 + 8 * (dk::kBarAEmpty + i), 1);              // A buffer free (MMA commit)
-      mbar_init(b0 + 8 * (dk::kBarAccFull + i), 1);             // accumulator complete (MMA commit)
-      mbar_init(b0 + 8 * (dk::kBarAccFree + i), dk::kDqWarps);  // accumulator read
+    for (int i = 0; i < dk::kA; ++i) {
+      mbar_init(b0 + 8 * (dk::kBarAFull + i), dk::kDqWarps);      // A buffer written
+      mbar_init(b0 + 8 * (dk::kBarAEmpty + i), 1);                // A buffer read (MMA commit)
+    }
+    for (int i = 0; i < dk::kAcc; ++i) {
+      mbar_init(b0 + 8 * (dk::kBarAccFull + i), 1);               // accumulator complete (MMA commit)
+      mbar_init(b0 + 8 * (dk::kBarAccFree + i), dk::kEpWarps);    // accumulator read
     }
     mbar_init(done_bar, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == dk::kDqWarps + 1) tmem_alloc(smem_u32(&tmem_slot), dk::kTmemCols);
+  if (warp == dk::kMmaWarp) tmem_alloc(smem_u32(&tmem_slot), dk::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   if (warp < 4) {
-    // constant correction columns of both A buffers: (1024, 1024), then zeros
+    // constant correction columns of the A buffers: (1024, 1024), then zeros
     const uint32_t lb = (uint32_t)(warp * 32) << 16;
     const uint32_t cz[8] = {dk::kOne1024, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-    for (int b = 0; b < RG::kA; ++b) tmem_st8_nw(tmem + lb + RG::kABase + b * dk::kACols + 32, cz);
+    for (int b = 0; b < dk::kA; ++b) tmem_st8_nw(tmem + lb + dk::kABase + b * dk::kACols + 32, cz);
     tmem_wait_st();
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
   // everything above overlaps the previous kernel's tail
   pdl_wait();
   pdl_trigger();
@@ -434,12 +429,11 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
   const int nact = *a.n_active;
   if (warp == 0) {
     const int lane = threadIdx.x & 31;
-    int loc[kMaxExperts / 32];
+    constexpr int kPerLane = kMaxExperts / 32;
     int sum = 0;
 #pragma unroll
-    for (int j = 0; j < kMaxExperts / 32; ++j) {
-      const int sl = (kMaxExperts / 32) * lane + j;
-      loc[j] = sum;
+    for (int j = 0; j < kPerLane; ++j) {
+      const int sl = kPerLane * lane + j;
       sum += sl < nact ? (a.counts[a.active[sl]] + NTOK - 1) / NTOK : 0;
     }
     int incl = sum;
@@ -448,14 +442,21 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
       const int t = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += t;
     }
+    int run = incl - sum;
 #pragma unroll
-    for (int j = 0; j < kMaxExperts / 32; ++j) s_pre[(kMaxExperts / 32) * lane + j] = incl - sum + loc[j];
+    for (int j = 0; j < kPerLane; ++j) {
+      const int sl = kPerLane * lane + j;
+      s_pre[sl] = run;
+      run += sl < nact ? (a.counts[a.active[sl]] + NTOK - 1) / NTOK : 0;
+    }
     if (lane == 31) s_pre[kMaxExperts] = incl;
   }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
   const int total = s_pre[nact] * per;
   volatile int* ab = &abort_flag;
-  dk::Cnt cnt;
+  dk::Pos ps;
   for (int tile = blockIdx.x; tile < total && !*ab; tile += gridDim.x) {
     int lo = 0, hi = nact - 1;
     while (lo < hi) {
@@ -479,23 +480,23 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
     bool ran = true;
     if (d.fmt == FMT_INT) {
       switch (d.bits * 1000 + d.group) {
-        case 2064: dk::decode_tile<NTOK, FMT_INT, 2, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
-        case 2128: dk::decode_tile<NTOK, FMT_INT, 2, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
-        case 3064: dk::decode_tile<NTOK, FMT_INT, 3, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
-        case 3128: dk::decode_tile<NTOK, FMT_INT, 3, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
-        case 4064: dk::decode_tile<NTOK, FMT_INT, 4, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
-        case 4128: dk::decode_tile<NTOK, FMT_INT, 4, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
+        case 2064: dk::decode_tile<NTOK, FMT_INT, 2, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, ps, ab); break;
+        case 2128: dk::decode_tile<NTOK, FMT_INT, 2, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, ps, ab); break;
+        case 3064: dk::decode_tile<NTOK, FMT_INT, 3, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, ps, ab); break;
+        case 3128: dk::decode_tile<NTOK, FMT_INT, 3, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, ps, ab); break;
+        case 4064: dk::decode_tile<NTOK, FMT_INT, 4, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, ps, ab); break;
+        case 4128: dk::decode_tile<NTOK, FMT_INT, 4, 128>(a, d, c, sm, stage_b, cbytes, b0, tmem, ps, ab); break;
         default: ran = false; break;
       }
     } else if (d.fmt == FMT_BITPLANE) {
       switch (d.bits) {
-        case 2: dk::decode_tile<NTOK, FMT_BITPLANE, 2, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
-        case 3: dk::decode_tile<NTOK, FMT_BITPLANE, 3, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
-        case 4: dk::decode_tile<NTOK, FMT_BITPLANE, 4, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale); break;
+        case 2: dk::decode_tile<NTOK, FMT_BITPLANE, 2, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, ps, ab); break;
+        case 3: dk::decode_tile<NTOK, FMT_BITPLANE, 3, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, ps, ab); break;
+        case 4: dk::decode_tile<NTOK, FMT_BITPLANE, 4, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, ps, ab); break;
         default: ran = false; break;
       }
     } else if (d.fmt == FMT_DENSE) {
-      dk::decode_tile<NTOK, FMT_DENSE, 16, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, cnt, ab, sscale);
+      dk::decode_tile<NTOK, FMT_DENSE, 16, 64>(a, d, c, sm, stage_b, cbytes, b0, tmem, ps, ab);
     } else {
       ran = false;
     }
@@ -504,15 +505,28 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
       break;
     }
   }
-  if (warp == dk::kDqWarps && (threadIdx.x & 31) == 0) dk::producer_drain(a, b0, cnt);
-  if (warp == dk::kDqWarps + 1 && (threadIdx.x & 31) == 0) {
+  if (warp == dk::kProdWarp && (threadIdx.x & 31) == 0) {
+    // every issued stage must land before the CTA may exit: walk back over
+    // the last nstages fills (a slot never filled in that lap tests complete)
+    dk::RingPos p = ps.st;
+    for (int k = 0; k < a.nstages; ++k) {
+      if (p.idx == 0) {
+        p.idx = a.nstages - 1;
+        p.ph ^= 1u;
+      } else {
+        --p.idx;
+      }
+      if (!mbar_wait_fast(b0 + 8 * (dk::kBarFull + p.idx), p.ph, a.status)) break;
+    }
+  }
+  if (warp == dk::kMmaWarp && (threadIdx.x & 31) == 0) {
     // every issued MMA must complete before TMEM is released
     mma_commit(done_bar);
     mbar_wait(done_bar, 0, a.status);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == dk::kDqWarps + 1) {
+  if (warp == dk::kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, dk::kTmemCols);
   }
@@ -557,8 +571,10 @@ static cudaError_t launch_ntok(const DecodeArgs& a, int maxbits, int grid_y, cud
   const int stage_b = dk::stage_bytes(NTOK, maxbits);
   // two CTAs per SM (2 x 256 TMEM columns): each takes about 100 KiB of
   // stages, as deep a ring as fits, to keep enough weight bytes in flight
+  // (a stage is released kA chunks after its own; kA + 2 stages keep the
+  // producer ahead, even for the large dense code blocks)
   DecodeArgs b = a;
-  b.nstages = std::min(dk::kMaxStages, (100 * 1024 - 1024) / stage_b);
+  b.nstages = std::max(dk::kA + 2, std::min(dk::kMaxStages, (100 * 1024 - 1024) / stage_b));
   const size_t smem = (size_t)b.nstages * stage_b + 1024;
   cudaError_t err = cudaFuncSetAttribute(decode_gemm_kernel<NTOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -575,8 +591,7 @@ cudaError_t launch_decode_gemm(const DecodeArgs& a, int ntok, int maxbits, int g
                                int* launches) {
   if (launches) ++*launches;
   if (ntok <= 16) return launch_ntok<16>(a, maxbits, grid_y, st);
-  if (ntok <= 32) return launch_ntok<32>(a, maxbits, grid_y, st);
-  return launch_ntok<64>(a, maxbits, grid_y, st);
+  return launch_ntok<32>(a, maxbits, grid_y, st);
 }
 
 }  // namespace moeq

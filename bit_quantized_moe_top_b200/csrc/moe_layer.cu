@@ -764,7 +764,8 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     // larger batches take more passes
     const double avg = (double)rows / E;
     const int want = (int)std::ceil(avg + 3.0 * std::sqrt(avg) + 1.0);
-    const int ntok = std::min(64, std::min(T, want) <= 16 ? 16 : std::min(T, want) <= 32 ? 32 : 64);
+    // (larger batches take more passes, run as separate tiles that share the weights through L2)
+    const int ntok = std::min(T, want) <= 16 ? 16 : 32;
     auto decode_gemm = [&](int block, const CUtensorMap& map, const CUtensorMap& cmap, int Kin, int M, int mode,
                            int KS) {
       if (ce != cudaSuccess) return;
