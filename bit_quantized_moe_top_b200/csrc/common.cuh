@@ -208,23 +208,12 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // The bounded wait, out of line: only taken when the phase is still open.
-// Gives up early once another role of the CTA has raised *abort_flag.
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, unsigned* status,
-                                                   volatile int* abort_flag) {
-  const unsigned long long t0 = globaltimer_ns();
-  for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (abort_flag && *abort_flag) return false;
-    if (globaltimer_ns() - t0 > 2000000000ull) {
-      atomicOr(status, ST_TIMEOUT);
-      return false;
-    }
-  }
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, unsigned* status) {
+  return mbar_wait(bar, parity, status);
 }
 // Bounded wait with an inlined fast path.
-__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, unsigned* status,
-                                               volatile int* abort_flag = nullptr) {
-  return mbar_test(bar, parity) || mbar_wait_slow(bar, parity, status, abort_flag);
+__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, unsigned* status) {
+  return mbar_test(bar, parity) || mbar_wait_slow(bar, parity, status);
 }
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

@@ -6,18 +6,17 @@
 // work of unpacking. A CTA owns 128 weight rows of one expert (one row per
 // TMEM lane) and a group-aligned range of 64-wide K chunks; CTAs are
 // persistent and walk the (expert, row block, K split, token pass) tiles.
-//   warp 12    producer: per chunk, the 128 rows' packed codes (one contiguous
+//   warp 8     producer: per chunk, the 128 rows' packed codes (one contiguous
 //              block), at a group's first chunk the routed rows' correction
 //              columns and the group's scale/zero pairs, and the expert's
 //              routed activation rows (TMA 2-D boxes of 16 rows, no multicast);
-//   warps 0-7  unpack, two groups of four taking alternate chunks: one thread
-//              per weight row turns the row's 64 codes into 32 fp16 pairs in
-//              registers and stores them into a TMEM buffer, the MMA's A
-//              operand;
-//   warp 13    allocates TMEM and issues tcgen05.mma kind::f16 with A from
+//   warps 0-3  unpack: one thread per weight row turns the row's 64 codes into
+//              32 fp16 pairs in registers and stores them into a TMEM buffer
+//              (one tcgen05.st), the MMA's A operand;
+//   warp 9     allocates TMEM and issues tcgen05.mma kind::f16 with A from
 //              TMEM (M = 128 weight rows), B = activations from shared memory
 //              (N = tokens, 16 or 32), D in TMEM;
-//   warps 8-11 epilogue: per quantisation group, y += s * acc in fp32
+//   warps 4-7  epilogue: per quantisation group, y += s * acc in fp32
 //              registers; at the end of the tile SwiGLU or fp32 output rows.
 // Every hand-off is an mbarrier; a warp's work per chunk is kept to a few
 // dozen instructions (ring positions advance incrementally, waits have an
@@ -58,17 +57,16 @@
 namespace moeq {
 namespace dk {
 
-constexpr int kUnpackGroups = 2;  // alternate chunks: one group's per-chunk chain is longer than the budget
-constexpr int kDqWarps = 4 * kUnpackGroups;
+constexpr int kDqWarps = 4;
 constexpr int kEpWarps = 4;
-constexpr int kEpWarp0 = kDqWarps, kProdWarp = kEpWarp0 + kEpWarps, kMmaWarp = kProdWarp + 1;
+constexpr int kProdWarp = kDqWarps + kEpWarps, kMmaWarp = kProdWarp + 1;
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 constexpr int kRows = 128;
 constexpr int kMaxStages = 16;  // stage ring depth: as many as about 100 KiB of shared memory hold
-constexpr int kA = 4;           // TMEM A buffers (two chunks per unpack group in flight)
+constexpr int kA = 3;           // TMEM A buffers
 constexpr int kAcc = 2;         // TMEM accumulators
 constexpr int kACols = 40;      // per A buffer: 32 code columns + 8 correction columns
-constexpr int kABase = 64;      // accumulators at [0, kAcc * NTOK), A buffers at [64, 224)
+constexpr int kABase = 128;     // accumulators at [0, kAcc * NTOK), A buffers at [128, 248)
 constexpr int kTmemCols = 256;
 constexpr int kActBox = 16;     // rows per TMA box
 constexpr uint32_t kOne1024 = 0x64006400u;  // fp16 pair (1024, 1024)
@@ -138,14 +136,15 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
   const int nbox = (n_pass + kActBox - 1) / kActBox;
   const int row0 = c.prow0 + c.tok0;
   const uint8_t* codes = (FMT == FMT_BITPLANE) ? d.plane[0] : d.codes;
+  // the whole warp runs the loop (warp-uniform values); one lane issues the copies
   for (int i = 0; i < c.nmain + c.next; ++i, ps.st.next(a.nstages)) {
-    if (!mbar_wait_fast(empty + 8 * ps.st.idx, ps.st.ph ^ 1u, a.status, abort_flag)) {
+    if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait_fast(empty + 8 * ps.st.idx, ps.st.ph ^ 1u, a.status))) {
       *abort_flag = 1;
       return;
     }
     bool first, last;
     group_pos<FMT, GROUP>(c, i, first, last);
-    uint8_t* st = sm + ps.st.idx * stage_b;
+    const uint32_t st = smem_u32(sm) + ps.st.idx * stage_b;
     const uint32_t fb = full + 8 * ps.st.idx;
     const bool main = i < c.nmain;
     const int kc = c.kc0 + i;
@@ -153,26 +152,28 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
     uint32_t bytes = nbox * kActBox * 128;
     if (main) bytes += (FMT == FMT_BITPLANE ? BITS * 1024 : kBlk);
     if (corr) bytes += nbox * kActBox * 32 + 512;
-    mbar_expect_tx(fb, bytes);
     const int kx = main ? kc * 64 : a.K;
-    for (int b = 0; b < nbox; ++b)
-      tma_load_2d(smem_u32(st + b * kActBox * 128), &a.tmap_act, kx, row0 + b * kActBox, fb);
-    if (main) {
-      uint8_t* cs = st + NTOK * 160;
-      const long long bidx = (long long)kc * RB + c.rb;
-      if constexpr (FMT == FMT_BITPLANE) {
+    const uint32_t cs = st + NTOK * 160;
+    const long long bidx = (long long)kc * RB + c.rb;
+    const int g = kc * 64 / GROUP;
+    if (elect_one()) {
+      mbar_expect_tx(fb, bytes);
+      for (int b = 0; b < nbox; ++b) tma_load_2d(st + b * kActBox * 128, &a.tmap_act, kx, row0 + b * kActBox, fb);
+      if (main) {
+        if constexpr (FMT == FMT_BITPLANE) {
 #pragma unroll
-        for (int q = 0; q < BITS; ++q) bulk_g2s(smem_u32(cs + q * 1024), d.plane[q] + bidx * 1024, 1024, fb);
-      } else {
-        bulk_g2s(smem_u32(cs), codes + bidx * kBlk, kBlk, fb);
-      }
-      if (corr) {
-        const int g = kc * 64 / GROUP;
-        for (int b = 0; b < nbox; ++b)
-          tma_load_2d(smem_u32(st + NTOK * 128 + b * kActBox * 32), &a.tmap_corr, 16 * g, row0 + b * kActBox, fb);
-        bulk_g2s(smem_u32(cs + cbytes), d.sz + (long long)g * a.M + c.rb * kRows, 512, fb);
+          for (int q = 0; q < BITS; ++q) bulk_g2s(cs + q * 1024, d.plane[q] + bidx * 1024, 1024, fb);
+        } else {
+          bulk_g2s(cs, codes + bidx * kBlk, kBlk, fb);
+        }
+        if (corr) {
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(st + NTOK * 128 + b * kActBox * 32, &a.tmap_corr, 16 * g, row0 + b * kActBox, fb);
+          bulk_g2s(cs + cbytes, d.sz + (long long)g * a.M + c.rb * kRows, 512, fb);
+        }
       }
     }
+    __syncwarp();
   }
 }
 
@@ -184,34 +185,34 @@ __device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int s
   const uint32_t accfull = bars + 8 * kBarAccFull, accfree = bars + 8 * kBarAccFree;
   const int n_pass = min(NTOK, c.n_e - c.tok0);
   const uint32_t idesc = idesc_f16(128, (n_pass + 15) & ~15);
-  // shared-memory descriptors of stage 0; a stage adds stage_b >> 4 to the
-  // start-address field, a K step of 16 fp16 adds 32 B >> 4 = 2
   const uint32_t sm0 = smem_u32(sm);
-  const uint64_t dact0 = sw128_desc(sm0), dcorr0 = sw32_desc(sm0 + NTOK * 128);
-  const uint64_t dstep = (uint64_t)(stage_b >> 4);
   for (int i = 0; i < c.nmain + c.next; ++i) {
     bool first, last;
     group_pos<FMT, GROUP>(c, i, first, last);
-    if (!mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status, abort_flag) ||
-        !mbar_wait_fast(afull + 8 * ps.ab.idx, ps.ab.ph, a.status, abort_flag) ||
-        (first && !mbar_wait_fast(accfree + 8 * ps.acc.idx, ps.acc.ph ^ 1u, a.status, abort_flag))) {
+    const bool ok = !*abort_flag && mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status) &&
+                    mbar_wait_fast(afull + 8 * ps.ab.idx, ps.ab.ph, a.status) &&
+                    (!first || mbar_wait_fast(accfree + 8 * ps.acc.idx, ps.acc.ph ^ 1u, a.status));
+    if (!__all_sync(0xffffffffu, ok)) {
       *abort_flag = 1;
       return;
     }
     tc_fence_after();
-    const uint64_t doff = dstep * (uint64_t)ps.st.idx;
+    const uint32_t bt = sm0 + ps.st.idx * stage_b;
     const uint32_t acc = tmem + ps.acc.idx * NTOK;
     const uint32_t ta = tmem + kABase + ps.ab.idx * kACols;
     const bool corr = FMT == FMT_INT && i < c.nmain && first;
-    if (corr) mma_f16_ts(acc, ta + 32, dcorr0 + doff, idesc, 0);
+    const uint64_t dact = sw128_desc(bt), dcorr = sw32_desc(bt + NTOK * 128);
+    // the whole warp runs the loop (warp-uniform values); one lane issues
+    if (elect_one()) {
+      if (corr) mma_f16_ts(acc, ta + 32, dcorr, idesc, 0);
 #pragma unroll
-    for (int k16 = 0; k16 < 4; ++k16)
-      mma_f16_ts(acc, ta + k16 * 8, dact0 + doff + 2 * k16, idesc, (corr || !first || k16 > 0) ? 1 : 0);
-    mma_commit(aempty + 8 * ps.ab.idx);
-    if (last) {
-      mma_commit(accfull + 8 * ps.acc.idx);
-      ps.acc.next(kAcc);
+      for (int k16 = 0; k16 < 4; ++k16)
+        mma_f16_ts(acc, ta + k16 * 8, dact + 2 * k16, idesc, (corr || !first || k16 > 0) ? 1 : 0);
+      mma_commit(aempty + 8 * ps.ab.idx);
+      if (last) mma_commit(accfull + 8 * ps.acc.idx);
     }
+    __syncwarp();
+    if (last) ps.acc.next(kAcc);
     ps.st.next(a.nstages);
     ps.ab.next(kA);
   }
@@ -223,8 +224,7 @@ __device__ void unpack(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, ui
   const uint32_t full = bars + 8 * kBarFull, empty = bars + 8 * kBarEmpty;
   const uint32_t afull = bars + 8 * kBarAFull, aempty = bars + 8 * kBarAEmpty;
   const int lane = threadIdx.x & 31;
-  const int grp = threadIdx.x >> 7;   // unpack group: the chunks with (count % kUnpackGroups) == grp
-  const int row = threadIdx.x & 127;  // TMEM lane
+  const int row = threadIdx.x;  // 0..127 = TMEM lane
   const uint32_t lane_base = (uint32_t)(row & ~31) << 16;
   LutRegs lut;
   if constexpr (FMT == FMT_BITPLANE) lut = load_lut(d.lut, BITS);
@@ -233,57 +233,61 @@ __device__ void unpack(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, ui
   for (int i = 0; i < c.nmain + c.next; ++i) {
     bool first, last;
     group_pos<FMT, GROUP>(c, i, first, last);
-    if (ps.chunks % kUnpackGroups == grp) {
-      // warp-uniform waits: every lane reaches the .sync.aligned TMEM stores
-      const bool ok = mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status, abort_flag) &&
-                      mbar_wait_fast(aempty + 8 * ps.ab.idx, ps.ab.ph ^ 1u, a.status, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) {
-        *abort_flag = 1;
-        return;
-      }
-      // the MMAs of chunk (this - kA), also this group's, are complete: its
-      // stage (codes read here, activations read by the MMAs) may be refilled
-      if (ps.chunks >= kA && lane == 0) mbar_arrive(empty + 8 * ps.rel.idx);
-      const uint32_t ta = tmem + lane_base + kABase + ps.ab.idx * kACols;
-      const uint8_t* cs = sm + ps.st.idx * stage_b + NTOK * 160;
-      if (FMT == FMT_INT && i < c.nmain && first) {
-        const uint32_t sz = reinterpret_cast<const uint32_t*>(cs + cbytes)[row];
-        tmem_st1_nw(ta + 33, prmt(sz, sz, 0x3232u));  // (z, z) against (-X_hi, -X_lo)
-      }
-      // the two K halves are stored as they are produced (16 registers live)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t v[16];
-        if (i < c.nmain) {
-          if constexpr (FMT == FMT_INT) {
-            uint32_t w[4];
-            load_half_words_int<BITS>(cs, row, h, w);
-            int_raw_half<BITS>(w, v);
-          } else if constexpr (FMT == FMT_BITPLANE) {
-            uint32_t pw[4];
-            load_half_planes<BITS>(cs, 1024, row, h, pw);
-            lut_half<BITS>(pw, lut, v);
-          } else {
-#pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-              const uint4 x = reinterpret_cast<const uint4*>(cs + (4 * h + qd) * 2048)[row];
-              v[4 * qd] = x.x; v[4 * qd + 1] = x.y; v[4 * qd + 2] = x.z; v[4 * qd + 3] = x.w;
-            }
-          }
-        } else {
-          // compensator stage: the row's B values (pairs), zero past the rank
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            v[j] = (16 * h + j) < RS2 ? d.brow[(long long)(16 * h + j) * a.M + R] : 0u;
-        }
-        tmem_st16_nw(ta + 16 * h, v);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(afull + 8 * ps.ab.idx);
+    // warp-uniform waits: every lane reaches the .sync.aligned TMEM stores
+    const bool ok = !*abort_flag && mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status) &&
+                    mbar_wait_fast(aempty + 8 * ps.ab.idx, ps.ab.ph ^ 1u, a.status);
+    if (!__all_sync(0xffffffffu, ok)) {
+      *abort_flag = 1;
+      return;
     }
-    if (ps.chunks >= kA) ps.rel.next(a.nstages);
+    // the MMAs of chunk (this - kA) are complete: its stage (codes read by
+    // these warps, activations read by the MMAs) may be refilled
+    if (ps.chunks >= kA) {
+      if (lane == 0) mbar_arrive(empty + 8 * ps.rel.idx);
+      ps.rel.next(a.nstages);
+    }
+    const uint32_t ta = tmem + lane_base + kABase + ps.ab.idx * kACols;
+    uint32_t v[32];
+    if (i < c.nmain) {
+      const uint8_t* cs = sm + ps.st.idx * stage_b + NTOK * 160;
+      if constexpr (FMT == FMT_INT) {
+        if (first) {
+          const uint32_t sz = reinterpret_cast<const uint32_t*>(cs + cbytes)[row];
+          tmem_st1_nw(ta + 33, prmt(sz, sz, 0x3232u));  // (z, z) against (-X_hi, -X_lo)
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t w[4], r16[16];
+          load_half_words_int<BITS>(cs, row, h, w);
+          int_raw_half<BITS>(w, r16);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[16 * h + j] = r16[j];
+        }
+      } else if constexpr (FMT == FMT_BITPLANE) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pw[4], r16[16];
+          load_half_planes<BITS>(cs, 1024, row, h, pw);
+          lut_half<BITS>(pw, lut, r16);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[16 * h + j] = r16[j];
+        }
+      } else {
+#pragma unroll
+        for (int qd = 0; qd < 8; ++qd) {
+          const uint4 x = reinterpret_cast<const uint4*>(cs + qd * 2048)[row];
+          v[4 * qd] = x.x; v[4 * qd + 1] = x.y; v[4 * qd + 2] = x.z; v[4 * qd + 3] = x.w;
+        }
+      }
+    } else {
+      // compensator stage: the row's B values (pairs), zero past the rank
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = j < RS2 ? d.brow[(long long)j * a.M + R] : 0u;
+    }
+    tmem_st32(ta, v);  // includes the wait for the store
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(afull + 8 * ps.ab.idx);
     ps.st.next(a.nstages);
     ps.ab.next(kA);
     ++ps.chunks;
@@ -295,7 +299,7 @@ __device__ void epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
                          Pos& ps, volatile int* abort_flag) {
   const uint32_t accfull = bars + 8 * kBarAccFull, accfree = bars + 8 * kBarAccFree;
   const int lane = threadIdx.x & 31;
-  const int row = threadIdx.x - 32 * kEpWarp0;  // 0..127 = TMEM lane
+  const int row = threadIdx.x - 32 * kDqWarps;  // 0..127 = TMEM lane
   const uint32_t lane_base = (uint32_t)(row & ~31) << 16;
   const int R = c.rb * kRows + row;
   int nmain_groups = 0;
@@ -305,25 +309,21 @@ __device__ void epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
   float y[NTOK];
 #pragma unroll
   for (int t = 0; t < NTOK; ++t) y[t] = 0.f;
-  // scale of the next group, loaded one group ahead
-  const uint32_t* szp = d.sz + (long long)g0 * a.M + R;
-  uint32_t sz_next = (FMT == FMT_INT && nmain_groups > 0) ? szp[0] : 0x3C00u;
   for (int gi = 0; gi < nmain_groups + c.next; ++gi) {
-    const uint32_t sz = sz_next;
-    if (FMT == FMT_INT) sz_next = gi + 1 < nmain_groups ? szp[(long long)(gi + 1) * a.M] : 0x3C00u;
-    const float s = (FMT == FMT_INT) ? __half2float(__ushort_as_half((uint16_t)(sz & 0xFFFFu))) : 1.f;
-    if (!__all_sync(0xffffffffu, mbar_wait_fast(accfull + 8 * ps.acc.idx, ps.acc.ph, a.status, abort_flag))) {
+    float s = 1.f;
+    if (FMT == FMT_INT && gi < nmain_groups) {
+      const uint32_t sz = d.sz[(long long)(g0 + gi) * a.M + R];
+      s = __half2float(__ushort_as_half((uint16_t)(sz & 0xFFFFu)));
+    }
+    if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait_fast(accfull + 8 * ps.acc.idx, ps.acc.ph, a.status))) {
       *abort_flag = 1;
       return;
     }
     tc_fence_after();
+    uint32_t v[NTOK];
+    tmem_ld<NTOK>(tmem + lane_base + ps.acc.idx * NTOK, v);
 #pragma unroll
-    for (int hh = 0; hh < NTOK / 8; ++hh) {
-      uint32_t v[8];
-      tmem_ld8(tmem + lane_base + ps.acc.idx * NTOK + 8 * hh, v);
-#pragma unroll
-      for (int t = 0; t < 8; ++t) y[8 * hh + t] = fmaf(s, __uint_as_float(v[t]), y[8 * hh + t]);
-    }
+    for (int t = 0; t < NTOK; ++t) y[t] = fmaf(s, __uint_as_float(v[t]), y[t]);
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(accfree + 8 * ps.acc.idx);
@@ -333,14 +333,17 @@ __device__ void epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
   const int nt = min(NTOK, c.n_e - c.tok0);
   if (a.mode == MODE_SWIGLU) {
     // gate rows are lanes 16f..16f+7 of each 16-row group, up rows 8 lanes later
-    const bool gate = (R & 15) < 8;
-    __half* zrow = a.zout + (long long)(c.prow0 + c.tok0) * a.ldz + 8 * (R >> 4) + (R & 7);
+    float up[NTOK];
 #pragma unroll
-    for (int t = 0; t < NTOK; ++t) {
-      const float up = __shfl_down_sync(0xffffffffu, y[t], 8);
-      if (gate && t < nt) {
-        const float gt = y[t];
-        zrow[(long long)t * a.ldz] = __float2half_rn(gt / (1.f + expf(-gt)) * up);
+    for (int t = 0; t < NTOK; ++t) up[t] = __shfl_down_sync(0xffffffffu, y[t], 8);
+    if ((R & 15) < 8) {
+      const int col = 8 * (R >> 4) + (R & 7);
+#pragma unroll
+      for (int t = 0; t < NTOK; ++t) {
+        if (t < nt) {
+          const float gt = y[t];
+          a.zout[(long long)(c.prow0 + c.tok0 + t) * a.ldz + col] = __float2half_rn(gt / (1.f + expf(-gt)) * up[t]);
+        }
       }
     }
   } else {
@@ -367,14 +370,14 @@ __device__ void decode_tile(const DecodeArgs& a, const BlockDesc& d, const Ctx& 
     c.nmain = (int)((long long)KC * (c.ks + 1) / a.KS) - c.kc0;
   }
   const int warp = threadIdx.x >> 5;
-  if (warp < kEpWarp0) {
+  if (warp < kDqWarps) {
     unpack<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, tmem, ps, ab);
   } else if (warp < kProdWarp) {
     epilogue<NTOK, FMT, GROUP>(a, d, c, bars, tmem, ps, ab);
   } else if (warp == kProdWarp) {
-    if ((threadIdx.x & 31) == 0) producer<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, ps, ab);
+    producer<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, ps, ab);
   } else {
-    if ((threadIdx.x & 31) == 0) mma_issuer<NTOK, FMT, GROUP>(a, c, sm, stage_b, bars, tmem, ps, ab);
+    mma_issuer<NTOK, FMT, GROUP>(a, c, sm, stage_b, bars, tmem, ps, ab);
   }
 }
 
@@ -395,10 +398,10 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
   if (threadIdx.x == 0) {
     for (int i = 0; i < a.nstages; ++i) {
       mbar_init(b0 + 8 * (dk::kBarFull + i), 1);                  // producer arrival + tx bytes
-      mbar_init(b0 + 8 * (dk::kBarEmpty + i), 4);                 // the chunk's unpack group, after its MMAs
+      mbar_init(b0 + 8 * (dk::kBarEmpty + i), dk::kDqWarps);      // unpack warps, after the stage's MMAs
     }
     for (int i = 0; i < dk::kA; ++i) {
-      mbar_init(b0 + 8 * (dk::kBarAFull + i), 4);                 // A buffer written (one unpack group)
+      mbar_init(b0 + 8 * (dk::kBarAFull + i), dk::kDqWarps);      // A buffer written
       mbar_init(b0 + 8 * (dk::kBarAEmpty + i), 1);                // A buffer read (MMA commit)
     }
     for (int i = 0; i < dk::kAcc; ++i) {
