@@ -31,9 +31,11 @@ Sources (page titles and the passage each step follows):
   Co-Design, abstract: bitwidths that differ between linear blocks and experts
   (step 1 takes each block's own bits).
 * TileQ: Efficient Low-Rank Quantization of Mixture-of-Experts with 2D Tiling,
-  abstract: low-rank expert terms evaluated with the quantized GEMM (step 4).
+  abstract: low-rank expert terms evaluated with the quantized GEMM (step 4);
+  its shared 2D-tiled factors enter step 4 as dense compensators D1, D2
+  (oracle/tileq.py).
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent:
 
 * integer format: w^ = (q - z) * s with one fp16 scale s and one fp16 zero z
   per group of g consecutive elements along K; codes packed little-endian per
@@ -192,14 +194,20 @@ def silu(a: np.ndarray) -> np.ndarray:
 
 
 def expert_ffn(x: np.ndarray, W1: np.ndarray, W2: np.ndarray, N: int,
-               A1=None, B1=None, A2=None, B2=None) -> np.ndarray:
-    """Rows x [n, K] -> o [n, K] for one expert (all fp64)."""
+               A1=None, B1=None, A2=None, B2=None, D1=None, D2=None) -> np.ndarray:
+    """Rows x [n, K] -> o [n, K] for one expert (all fp64). D1 / D2 are dense
+    compensators (the 2D-tiled shared form, oracle/tileq.py) that take the
+    place of B1 A1 / B2 A2."""
     h = x @ W1.T
-    if A1 is not None and A1.shape[0] > 0:
+    if D1 is not None:
+        h = h + x @ D1.T
+    elif A1 is not None and A1.shape[0] > 0:
         h = h + (x @ A1.T) @ B1.T
     z = silu(h[:, :N]) * h[:, N:]
     o = z @ W2.T
-    if A2 is not None and A2.shape[0] > 0:
+    if D2 is not None:
+        o = o + z @ D2.T
+    elif A2 is not None and A2.shape[0] > 0:
         o = o + (z @ A2.T) @ B2.T
     return o
 
@@ -210,8 +218,8 @@ def moe_forward(X: np.ndarray, logits: np.ndarray, top_k: int,
     """The layer's forward pass.
 
     ``expert(e)`` returns a dict with fp64 arrays W1 [2N, K], W2 [K, N] and
-    optional A1, B1, A2, B2 (it is called only for experts that receive
-    tokens). ``rows`` restricts the output to those tokens (routing and
+    optional A1, B1, A2, B2, or dense compensators D1 [2N, K], D2 [K, N] (it
+    is called only for experts that receive tokens). ``rows`` restricts the output to those tokens (routing and
     bucketing are still computed for all tokens). ``comp_top_n`` > 0 applies
     the compensators only to the first n routing slots of each token and runs
     the other slots' experts on their quantised weights alone (Bandwidth-
@@ -238,7 +246,7 @@ def moe_forward(X: np.ndarray, logits: np.ndarray, top_k: int,
         plain = [p for p in ps if not (comp_top_n <= 0 or slot[p] < comp_top_n)]
         if comp:
             o = expert_ffn(X64[perm[comp]], ex["W1"], ex["W2"], N, ex.get("A1"), ex.get("B1"), ex.get("A2"),
-                           ex.get("B2"))
+                           ex.get("B2"), ex.get("D1"), ex.get("D2"))
             for i, p in enumerate(comp):
                 O[p] = o[i]
         if plain:

@@ -13,7 +13,7 @@ multiplier and eta the exponentiated prompt residual. Figure 4: pages are
 restored before a higher bitwidth is committed (the restore plan below undoes
 reductions, the most damage removed per byte first).
 
-Readings where the pages are silent (listed in the design doc): one action drops or
+Readings where the pages are silent: one action drops or
 restores one bit-plane of one block; a block's floor bitwidth and per-plan
 depth cap bound its actions ("bitwidth floor stages", "depth caps"); equal
 damage per byte goes to the lower block index; a block's next action is a
