@@ -41,6 +41,10 @@ def parse():
     p.add_argument("--tokens", type=int, default=64)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=20.0)
+    p.add_argument("--tileq", type=int, default=0,
+                   help="rank of 2D-tiled shared compensators on both blocks (replacing the per-expert ones); 0 = off")
+    p.add_argument("--tile-m", type=int, default=1024)
+    p.add_argument("--tile-k", type=int, default=1024)
     return p.parse_args()
 
 
@@ -72,17 +76,46 @@ def layer_bytes(cfg, counts, T):
     return tot + 2 * T * cfg.K + 4 * T * cfg.E + 2 * T * cfg.K
 
 
-def gemm1_bytes(cfg, counts):
+def tileq_shape(cfg, block, tq):
+    """(M, K_in, P, Q) of a block type under tiled shared compensators tq = (r, tile_m, tile_k)."""
+    M, Kin = (2 * cfg.N, cfg.K) if block == 0 else (cfg.K, cfg.N)
+    return M, Kin, M // tq[1], Kin // tq[2]
+
+
+def gemm1_bytes(cfg, counts, tq=None):
     """Algorithmic bytes of one gate/up GEMM launch: codes + scales + B1 of the
     touched experts, the routed activation rows (K + r columns, fp16) and the
-    SwiGLU output rows (N columns, fp16)."""
+    SwiGLU output rows (N columns, fp16). With tiled shared compensators
+    (tq = (r, tile_m, tile_k)): the shared U1 once, and P*r compensator
+    columns per routed row."""
     tot = 0.0
+    if tq:
+        M, Kin, P, Q = tileq_shape(cfg, 0, tq)
+        tot += 2 * M * tq[0]
     for e, n in enumerate(counts):
         if n > 0:
             wb, bb, _ = block_bytes(cfg, cfg.experts[e], 0)
             r = cfg.experts[e].rank
-            tot += wb + bb + 2 * n * (cfg.K + r) + 2 * n * cfg.N
+            if tq:
+                tot += wb + 2 * n * (cfg.K + P * tq[0]) + 2 * n * cfg.N
+            else:
+                tot += wb + bb + 2 * n * (cfg.K + r) + 2 * n * cfg.N
     return tot
+
+
+def tileq_bytes_flops(cfg, counts, T, tq):
+    """Factor bytes (U, V once; the cores of touched experts) and flops of the
+    tiled shared compensators of both blocks: z = V x per token (W1) or per
+    routed row (W2), u = C z per routed row and row tile, U u per routed row."""
+    r = tq[0]
+    rows = sum(counts)
+    touched = sum(1 for n in counts if n > 0)
+    b = f = 0.0
+    for block in (0, 1):
+        M, Kin, P, Q = tileq_shape(cfg, block, tq)
+        b += 2 * (M * r + r * Kin) + touched * 2 * P * Q * r * r
+        f += 2.0 * (T if block == 0 else rows) * Kin * r + 2.0 * rows * (P * Q * r * r + M * r)
+    return b, f
 
 
 def gemm1_flops(cfg, counts):
@@ -261,6 +294,11 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     T = args.tokens
     cfg = ms.make_config(args.config)
+    tq = (args.tileq, args.tile_m, args.tile_k) if args.tileq else None
+    if tq:
+        # the tiled shared compensators replace every expert's own pair
+        cfg.experts = [ms.ExpertSpec(sp.fmt, sp.bits, sp.group, 0) for sp in cfg.experts]
+    workload = f"{WORKLOADS[args.config]}_T{T}" + (f"_tileq_r{tq[0]}_{tq[1]}x{tq[2]}" if tq else "")
 
     if args.impl == "reference":
         if rank != 0:
@@ -303,6 +341,10 @@ def main():
         for b in (0, 1):
             blocks[(e, b)] = ms.make_block(cfg, e, b, device=dev)
     L = build_layer(bq, cfg, blocks, max_tokens=T)
+    if tq:
+        for b in (0, 1):
+            U, V, C = ms.make_tileq(cfg, b, tq[0], tq[1], tq[2], dev)
+            L.set_tileq(b, tq[0], tq[1], tq[2], U, V, C)
     X, logits = ms.make_inputs(cfg, T, dev, key_extra=rank)
     Y = torch.empty_like(X)
     stream = torch.cuda.current_stream(dev)
@@ -350,21 +392,25 @@ def main():
     k1 = kernel_means.get(kname, float("nan"))
     layer_b = layer_bytes(cfg, counts, T)
     layer_f = layer_flops(cfg, counts)
+    if tq:
+        tb, tf = tileq_bytes_flops(cfg, counts, T, tq)
+        layer_b += tb
+        layer_f += tf
     if prefill:
         f1 = gemm1_flops(cfg, counts)
         achieved = f1 / (k1 * 1e-3) / 1e12
         roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": tc_sustained,
                     "unit": "TFLOP/s", "frac": achieved / tc_sustained,
-                    "traffic": stored_traffic(kname, f"{WORKLOADS[args.config]}_T{T}"),
+                    "traffic": stored_traffic(kname, workload),
                     "peak_source": f"{peak_src} bf16 sustained (fp16 has the same dense rate)",
                     "frac_of_burst_peak": achieved / tc_peak, "algorithmic_flops_per_launch": f1,
                     "launch_ms": k1}
     else:
-        b1 = gemm1_bytes(cfg, counts)
+        b1 = gemm1_bytes(cfg, counts, tq)
         achieved = b1 / (k1 * 1e-3) / 1e9
         roofline = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                     "frac": achieved / hbm_peak,
-                    "traffic": stored_traffic(kname, f"{WORKLOADS[args.config]}_T{T}"), "peak_source": peak_src,
+                    "traffic": stored_traffic(kname, workload), "peak_source": peak_src,
                     "algorithmic_bytes_per_launch": b1, "launch_ms": k1}
 
     # end to end: host buffers through moe_layer_forward_host (copies inside the timed region)
@@ -384,7 +430,7 @@ def main():
     line = None
     if rank == 0:
         cpu = None
-        if not args.no_cpu_baseline and world == 1:
+        if not args.no_cpu_baseline and world == 1 and not tq:
             cpu_blocks = {k: ms.BlockWeights(**{**v.__dict__, "codes": v.codes.cpu(),
                                               "scales": None if v.scales is None else v.scales.cpu(),
                                               "zeros_or_lut": None if v.zeros_or_lut is None else v.zeros_or_lut.cpu(),
@@ -400,13 +446,15 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16 operands, f32 accumulate",
             "data": "synthetic",
-            "config": {"workload": f"{WORKLOADS[args.config]}_T{T}", "T": T, "E": cfg.E, "top_k": cfg.top_k,
+            "config": {"workload": workload, "T": T, "E": cfg.E, "top_k": cfg.top_k,
                        "d_model": cfg.K, "d_ff": cfg.N,
                        "bits": sorted(set(b for sp in cfg.experts for b in sp.bits)),
                        "format": "bit-plane+LUT" if cfg.experts[0].fmt == 1 else "int asym",
                        "group": cfg.experts[0].group, "ranks": sorted(set(sp.rank for sp in cfg.experts)),
                        "parallelism": f"replicas x{world}",
-                       "l2": "flushed between steps (256 MiB write, untimed)"},
+                       "l2": "flushed between steps (256 MiB write, untimed)",
+                       **({"compensator": {"kind": "2D-tiled shared factors", "rank": tq[0], "tile_m": tq[1],
+                                           "tile_k": tq[2]}} if tq else {})},
             "layer_hbm_gbs": layer_b / (ms_per_step * 1e-3) / 1e9,
             "layer_tflops": layer_f / (ms_per_step * 1e-3) / 1e12,
             "layer_bytes_per_step": layer_b,

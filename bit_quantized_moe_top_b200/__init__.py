@@ -30,6 +30,7 @@ EXPORTS = ["moe_layer_create", "moe_layer_set_expert_weights", "moe_layer_set_bi
            "moe_layer_sync_status", "moe_layer_last_launch_count", "moe_layer_set_profiling",
            "moe_layer_kernel_times", "moe_route_topk_noalloc", "moe_plan_reduce", "moe_plan_restore",
            "moe_layer_release_planes", "moe_layer_reload_planes", "moe_layer_page_state",
+           "moe_layer_set_tileq", "moe_layer_clear_tileq",
            "moe_status_string", "moe_layer_destroy"]
 
 
@@ -66,6 +67,8 @@ def _lib() -> ctypes.CDLL:
         lib.moe_layer_set_bits.argtypes = [P, I, I, I]
         lib.moe_layer_set_path.argtypes = [P, I]
         lib.moe_layer_set_comp_top_n.argtypes = [P, I]
+        lib.moe_layer_set_tileq.argtypes = [P, I, I, I, I, P, P, P, I]
+        lib.moe_layer_clear_tileq.argtypes = [P, I]
         lib.moe_layer_forward.argtypes = [P, P, P, I, I, P, P]
         lib.moe_layer_forward_host.argtypes = [P, P, P, I, I, P, P]
         lib.moe_layer_get_routing.argtypes = [P, P, P, P, P, P, P]
@@ -130,6 +133,20 @@ def moe_layer_set_bits(layer: int, expert: int, block: int, bits: int) -> None:
 
 def moe_layer_set_comp_top_n(layer: int, n: int) -> None:
     _check(_lib().moe_layer_set_comp_top_n(layer, n), "moe_layer_set_comp_top_n")
+
+
+def moe_layer_set_tileq(layer: int, block: int, rank: int, tile_m: int, tile_k: int, U, V, cores) -> None:
+    """U [M, rank], V [rank, K_in], cores [E, P, Q, rank, rank]: bf16 torch
+    tensors, all on the host or all on the device."""
+    kind = 1 if U.is_cuda else 0
+    for t in (U, V, cores):
+        assert t.is_contiguous() and t.is_cuda == U.is_cuda
+    _check(_lib().moe_layer_set_tileq(layer, block, rank, tile_m, tile_k, _ptr(U), _ptr(V), _ptr(cores), kind),
+           "moe_layer_set_tileq")
+
+
+def moe_layer_clear_tileq(layer: int, block: int) -> None:
+    _check(_lib().moe_layer_clear_tileq(layer, block), "moe_layer_clear_tileq")
 
 
 def moe_layer_set_path(layer: int, path: int) -> None:
@@ -296,6 +313,12 @@ class MoELayer:
 
     def set_comp_top_n(self, n):
         moe_layer_set_comp_top_n(self.handle, n)
+
+    def set_tileq(self, block, rank, tile_m, tile_k, U, V, cores):
+        moe_layer_set_tileq(self.handle, block, rank, tile_m, tile_k, U, V, cores)
+
+    def clear_tileq(self, block):
+        moe_layer_clear_tileq(self.handle, block)
 
     def set_path(self, path):
         moe_layer_set_path(self.handle, path)

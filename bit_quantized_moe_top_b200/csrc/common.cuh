@@ -45,8 +45,16 @@ struct BlockDesc {
   int fmt, bits, group, rank;
   int M, K;
   int loaded;
-  int pad_;
+  // 2D-tiled shared compensator (0 = per-expert factors): the compensator
+  // activations of internal rows [128 rb, 128 rb + 128) start at column
+  // K + (128 rb / tq_span) * tq_cols of the activation rows
+  int tq_span, tq_cols;
 };
+
+// Column offset, after K, of a 128-row block's compensator activations.
+__host__ __device__ __forceinline__ int comp_col_offset(const BlockDesc& d, int rb) {
+  return d.tq_span > 0 ? (rb * 128 / d.tq_span) * d.tq_cols : 0;
+}
 
 struct ExpertDesc {
   BlockDesc blk[2];

@@ -152,7 +152,7 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
     uint32_t bytes = nbox * kActBox * 128;
     if (main) bytes += (FMT == FMT_BITPLANE ? BITS * 1024 : kBlk);
     if (corr) bytes += nbox * kActBox * 32 + 512;
-    const int kx = main ? kc * 64 : a.K;
+    const int kx = main ? kc * 64 : a.K + comp_col_offset(d, c.rb);
     const uint32_t cs = st + NTOK * 160;
     const long long bidx = (long long)kc * RB + c.rb;
     const int g = kc * 64 / GROUP;

@@ -47,6 +47,7 @@ struct RouteArgs {
   int* inv_pos;               // [T, k]
   int* pinv;                  // [T, k] padded row
   int* pslot;                 // [padded rows] routing slot of each routed row
+  int* ptok;                  // [padded rows] token of each routed row
   void* act;                  // activation buffer, fp16 row-major [rows, Kpad]
   int Kpad;
   unsigned* status;
@@ -117,6 +118,32 @@ struct LowrankArgs {
   unsigned* status;
 };
 
+// 2D-tiled shared compensator of one block type (TileQ abstract): z = V_q x
+// per source row and column tile, then u_p = sum_q C[e, p, q] z_q per routed
+// row and row tile, written as fp16 into the activation columns after Kin.
+struct TileqArgs {
+  int mode;                   // 0: W1 (sources = tokens, rows of x, bf16); 1: W2 (sources = routed pairs t*k+j, rows of act, fp16)
+  const __nv_bfloat16* x;     // mode 0: layer input [T, Kin]
+  __half* act;                // activation buffer, fp16 row-major, leading dimension lda
+  long long lda;
+  const int* pinv;            // [T, k] padded row of (t, j)
+  const int* ptok;            // [padded rows] token of each routed row
+  const int* pslot;           // [padded rows] routing slot of each routed row
+  const int* active;          // experts with rows, n_active of them
+  const int* n_active;
+  const int* counts;          // [E] routed rows per expert
+  const int* poffsets;        // [E+1] first padded row per expert
+  int T, k;
+  int Kin;                    // input features of the block
+  int r;                      // rank, 16 or 32
+  int tile_k, Q;              // column tiles
+  int P;                      // row tiles; mode 0: tiles < P/2 are gate tiles, the rest up tiles
+  const void* v;              // V [r][Kin] row-major, bf16 (mode 0) or fp16 (mode 1): the MMA's B operand
+  const __nv_bfloat16* ct;    // cores transposed, [E][P][Q][r (input j)][r (output i)]
+  float* z;                   // [sources][Q][r]
+  int comp_top_n;             // > 0: routed rows in slots >= comp_top_n get u = 0
+};
+
 struct PrefillArgs {
   CUtensorMap tmap_act;       // activations [rows, Kpad] fp16 row-major; box 64 x 128, 128-byte swizzle
   const ExpertDesc* experts;
@@ -170,6 +197,7 @@ int decode_rows_per_cta();
 cudaError_t launch_decode_gemm(const DecodeArgs& a, int ntok, int maxbits, int grid_y, cudaStream_t st,
                                int* launches);
 cudaError_t launch_lowrank(const LowrankArgs& a, int grid_y, cudaStream_t st, int* launches);
+cudaError_t launch_tileq(const TileqArgs& a, int grid_y, cudaStream_t st, int* launches);
 cudaError_t launch_prefill_gemm(const PrefillArgs& a, int grid_y, int grid_z, cudaStream_t st, int* launches);
 int prefill_smem_bytes();
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st, int* launches);

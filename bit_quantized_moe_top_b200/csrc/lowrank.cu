@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
   if (nrows <= 0) return;
   const BlockDesc& dd = a.experts[e].blk[a.block];
   const int r = dd.rank;
-  if (r <= 0) return;
+  if (r <= 0 || dd.tq_span > 0) return;  // 2D-tiled shared compensators have their own kernels
   const uint4* afrag = dd.afrag;
   const int RF = r / 16;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

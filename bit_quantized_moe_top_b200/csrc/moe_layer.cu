@@ -90,8 +90,14 @@ struct moe_layer {
   long long rows_pad_max = 0, nt8cap = 0;
   int nb_max = 0, ks2_max = 1, kslr_max = 1;
   long long sem_stride = 0;
-  DevBuf idx, w, counts, offsets, poffsets, active, n_active, ticket, perm, inv_pos, pinv, pslot;
+  DevBuf idx, w, counts, offsets, poffsets, active, n_active, ticket, perm, inv_pos, pinv, pslot, ptok;
   int comp_top_n = 0;
+  // 2D-tiled shared compensators, per block type (0 = W1, 1 = W2)
+  struct Tileq {
+    bool on = false;
+    int r = 0, tile_m = 0, tile_k = 0, P = 0, Q = 0, cols = 0, span = 0;
+    DevBuf brow, v, ct, z;  // v: V [r][Kin] in the z MMA's operand type (W1 bf16, W2 fp16)
+  } tq[2];
   DevBuf block_counts, block_base, pblock_base, sem, status;
   DevBuf xact, zact, obuf, part, corr_x, corr_z;
   int ldc_x = 0, ldc_z = 0;  // correction columns per row: 16 per group of 64 (the smallest group)
@@ -204,8 +210,14 @@ const char* moe_status_string(moe_status_t s) {
 void moe_layer_destroy(moe_layer_t* L) {
   if (!L) return;
   for (auto& s : L->store) free_block(s);
+  for (auto& t : L->tq) {
+    dfree(t.brow);
+    dfree(t.v);
+    dfree(t.ct);
+    dfree(t.z);
+  }
   DevBuf* bufs[] = {&L->d_experts, &L->idx, &L->w, &L->counts, &L->offsets, &L->poffsets, &L->active,
-                    &L->n_active, &L->ticket, &L->perm, &L->inv_pos, &L->pinv, &L->pslot, &L->block_counts,
+                    &L->n_active, &L->ticket, &L->perm, &L->inv_pos, &L->pinv, &L->pslot, &L->ptok, &L->block_counts,
                     &L->block_base, &L->pblock_base, &L->sem, &L->status, &L->xact, &L->zact, &L->obuf,
                     &L->part, &L->corr_x, &L->corr_z, &L->hx, &L->hl, &L->hy};
   for (DevBuf* b : bufs) dfree(*b);
@@ -281,6 +293,7 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   A(L->inv_pos, sizeof(int) * rows);
   A(L->pinv, sizeof(int) * rows);
   A(L->pslot, sizeof(int) * (size_t)L->rows_pad_max);
+  A(L->ptok, sizeof(int) * (size_t)L->rows_pad_max);
   A(L->block_counts, sizeof(int) * (size_t)L->nb_max * E);
   A(L->block_base, sizeof(int) * (size_t)L->nb_max * E);
   A(L->pblock_base, sizeof(int) * (size_t)L->nb_max * E);
@@ -329,9 +342,28 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   return MOE_OK;
 }
 
+// the device copy of an expert's descriptor: its own blocks, with a block
+// type's shared 2D-tiled compensator in place of the expert's factors
+static ExpertDesc device_desc(const moe_layer_t* L, int e) {
+  ExpertDesc x = L->hdesc[e];
+  for (int b = 0; b < 2; ++b) {
+    BlockDesc& d = x.blk[b];
+    const auto& t = L->tq[b];
+    d.tq_span = d.tq_cols = 0;
+    if (!t.on) continue;
+    d.rank = t.cols;
+    d.brow = static_cast<const uint32_t*>(t.brow.p);
+    d.afrag = nullptr;
+    d.tq_span = t.span;
+    d.tq_cols = t.cols;
+  }
+  return x;
+}
+
 static moe_status_t upload_desc(moe_layer_t* L, int e) {
-  return cuda_status(cudaMemcpy(static_cast<ExpertDesc*>(L->d_experts.p) + e, &L->hdesc[e], sizeof(ExpertDesc),
-                                cudaMemcpyHostToDevice));
+  const ExpertDesc x = device_desc(L, e);
+  return cuda_status(
+      cudaMemcpy(static_cast<ExpertDesc*>(L->d_experts.p) + e, &x, sizeof(ExpertDesc), cudaMemcpyHostToDevice));
 }
 
 // device copy of a caller buffer (host or device); owned by `tmp`
@@ -575,6 +607,145 @@ moe_status_t moe_layer_set_comp_top_n(moe_layer_t* L, int n) {
   return MOE_OK;
 }
 
+// Grows the activation buffers to Kin + wx / Kin + wz columns after the
+// inputs (wx, wz: compensator columns of W1 / W2), re-encoding their tensor
+// maps. Synchronous; no forward may be in flight.
+static moe_status_t grow_act(moe_layer_t* L, int wx, int wz) {
+  const int kx = std::max(L->Kpad_x, L->K + (wx + 31) / 32 * 32);
+  const int kz = std::max(L->Kpad_z, L->N + (wz + 31) / 32 * 32);
+  if (kx == L->Kpad_x && kz == L->Kpad_z) return MOE_OK;
+  DevBuf nx, nz;
+  moe_status_t st = dalloc(nx, sizeof(__half) * (size_t)L->rows_pad_max * kx);
+  if (st == MOE_OK) st = dalloc(nz, sizeof(__half) * (size_t)L->rows_pad_max * kz);
+  cudaError_t ce = cudaSuccess;
+  if (st == MOE_OK) ce = cudaMemset(nx.p, 0, nx.n);
+  if (st == MOE_OK && ce == cudaSuccess) ce = cudaMemset(nz.p, 0, nz.n);
+  if (st == MOE_OK && ce == cudaSuccess) ce = cudaDeviceSynchronize();
+  CUtensorMap mx, mz, mxd, mzd;
+  const bool maps = st == MOE_OK && ce == cudaSuccess && encode_act_map(&mx, nx.p, kx, L->rows_pad_max, 128) &&
+                    encode_act_map(&mz, nz.p, kz, L->rows_pad_max, 128) &&
+                    encode_act_map(&mxd, nx.p, kx, L->rows_pad_max, 16) &&
+                    encode_act_map(&mzd, nz.p, kz, L->rows_pad_max, 16);
+  if (!maps) {
+    dfree(nx);
+    dfree(nz);
+    return st != MOE_OK ? st : MOE_ERR_CUDA;
+  }
+  dfree(L->xact);
+  dfree(L->zact);
+  L->xact = nx;
+  L->zact = nz;
+  L->Kpad_x = kx;
+  L->Kpad_z = kz;
+  L->tmap_x = mx;
+  L->tmap_z = mz;
+  L->tmap_xd = mxd;
+  L->tmap_zd = mzd;
+  return MOE_OK;
+}
+
+static void free_tileq(moe_layer_t::Tileq& t) {
+  dfree(t.brow);
+  dfree(t.v);
+  dfree(t.ct);
+  dfree(t.z);
+  t.on = false;
+}
+
+moe_status_t moe_layer_set_tileq(moe_layer_t* L, int block, int rank, int tile_m, int tile_k, const void* U,
+                                 const void* V, const void* cores, int ptr_kind) {
+  if (!L || block < 0 || block > 1 || (rank != 16 && rank != 32) || !U || !V || !cores ||
+      (ptr_kind != 0 && ptr_kind != 1))
+    return MOE_ERR_INVALID_ARG;
+  const int K = L->K, N = L->N, E = L->E;
+  const int M = block == 0 ? 2 * N : K, Kin = block == 0 ? K : N, half = block == 0 ? N : K;
+  if (tile_m < 256 || tile_m % 256 || half % tile_m || tile_k < 256 || tile_k % 256 || Kin % tile_k)
+    return MOE_ERR_INVALID_ARG;
+  const int r = rank, P = M / tile_m, Q = Kin / tile_k, cols = block == 0 ? 2 * r : r;
+  const size_t nU = (size_t)M * r, nV = (size_t)r * Kin, nC = (size_t)E * P * Q * r * r;
+  std::vector<uint16_t> hU(nU), hV(nV), hC(nC);
+  auto fetch = [&](std::vector<uint16_t>& h, const void* src) {
+    if (ptr_kind == 0) {
+      std::memcpy(h.data(), src, h.size() * sizeof(uint16_t));
+      return cudaSuccess;
+    }
+    return cudaMemcpy(h.data(), src, h.size() * sizeof(uint16_t), cudaMemcpyDeviceToHost);
+  };
+  cudaError_t ce = fetch(hU, U);
+  if (ce == cudaSuccess) ce = fetch(hV, V);
+  if (ce == cudaSuccess) ce = fetch(hC, cores);
+  if (ce != cudaSuccess) return MOE_ERR_CUDA;
+  // B operand of the compensator stage: W1 gate rows take the first r
+  // columns (their gate tile's u), up rows the next r (their up tile's u)
+  std::vector<uint16_t> hB((size_t)M * cols, 0);
+  for (int m = 0; m < M; ++m)
+    for (int c = 0; c < r; ++c) hB[(size_t)m * cols + (block == 0 && m >= N ? r : 0) + c] = hU[(size_t)m * r + c];
+  // W2's z MMA multiplies fp16 rows of Z: V in fp16 there (bf16 -> fp16 is
+  // exact for values in fp16's normal range)
+  if (block == 1)
+    for (auto& x : hV) {
+      uint32_t f = (uint32_t)x << 16;
+      float fv;
+      std::memcpy(&fv, &f, sizeof(fv));
+      const __half h = __float2half_rn(fv);
+      std::memcpy(&x, &h, sizeof(x));
+    }
+  std::vector<uint16_t> hCt(nC);
+  for (size_t b = 0; b < (size_t)E * P * Q; ++b)
+    for (int i = 0; i < r; ++i)
+      for (int j = 0; j < r; ++j) hCt[b * r * r + (size_t)j * r + i] = hC[b * r * r + (size_t)i * r + j];
+  const long long src_rows = block == 0 ? L->max_tokens : (long long)L->max_tokens * L->max_top_k;
+  moe_layer_t::Tileq t;
+  DevBuf tmpB;
+  moe_status_t st = dalloc(t.brow, (size_t)(cols / 2) * M * sizeof(uint32_t));
+  if (st == MOE_OK) st = dalloc(tmpB, hB.size() * sizeof(uint16_t));
+  if (st == MOE_OK) st = dalloc(t.v, nV * sizeof(uint16_t));
+  if (st == MOE_OK) st = dalloc(t.ct, nC * sizeof(uint16_t));
+  if (st == MOE_OK) st = dalloc(t.z, (size_t)src_rows * Q * r * sizeof(float));
+  if (st == MOE_OK) {
+    ce = cudaMemcpy(tmpB.p, hB.data(), hB.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
+    if (ce == cudaSuccess)
+      ce = launch_relayout_brow(static_cast<const __nv_bfloat16*>(tmpB.p), static_cast<uint32_t*>(t.brow.p), M,
+                                cols, block, N, nullptr);
+    if (ce == cudaSuccess) ce = cudaMemcpy(t.v.p, hV.data(), nV * sizeof(uint16_t), cudaMemcpyHostToDevice);
+    if (ce == cudaSuccess) ce = cudaMemcpy(t.ct.p, hCt.data(), nC * sizeof(uint16_t), cudaMemcpyHostToDevice);
+    if (ce == cudaSuccess) ce = cudaDeviceSynchronize();
+    if (ce != cudaSuccess) st = MOE_ERR_CUDA;
+  }
+  dfree(tmpB);
+  if (st == MOE_OK) {
+    const auto& o = L->tq[1 - block];
+    const int w_this = P * r, w_other = o.on ? o.P * o.r : 0;
+    st = grow_act(L, block == 0 ? w_this : w_other, block == 0 ? w_other : w_this);
+  }
+  if (st != MOE_OK) {
+    free_tileq(t);
+    return st;
+  }
+  free_tileq(L->tq[block]);
+  t.on = true;
+  t.r = r;
+  t.tile_m = tile_m;
+  t.tile_k = tile_k;
+  t.P = P;
+  t.Q = Q;
+  t.cols = cols;
+  t.span = block == 0 ? 2 * tile_m : tile_m;  // internal rows per tile (W1 interleaves gate and up rows)
+  L->tq[block] = t;
+  for (int e = 0; e < E && st == MOE_OK; ++e) st = upload_desc(L, e);
+  return st;
+}
+
+moe_status_t moe_layer_clear_tileq(moe_layer_t* L, int block) {
+  if (!L || block < 0 || block > 1) return MOE_ERR_INVALID_ARG;
+  if (!L->tq[block].on) return MOE_OK;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  free_tileq(L->tq[block]);
+  moe_status_t st = MOE_OK;
+  for (int e = 0; e < L->E && st == MOE_OK; ++e) st = upload_desc(L, e);
+  return st;
+}
+
 moe_status_t moe_layer_set_path(moe_layer_t* L, int path) {
   if (!L || path < MOE_PATH_AUTO || path > MOE_PATH_PREFILL) return MOE_ERR_INVALID_ARG;
   L->path = path;
@@ -658,6 +829,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
   ra.inv_pos = static_cast<int*>(L->inv_pos.p);
   ra.pinv = static_cast<int*>(L->pinv.p);
   ra.pslot = static_cast<int*>(L->pslot.p);
+  ra.ptok = static_cast<int*>(L->ptok.p);
   ra.act = L->xact.p;
   ra.Kpad = L->Kpad_x;
   ra.status = static_cast<unsigned*>(L->status.p);
@@ -727,10 +899,41 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     prof_mark(L, st, block == 0 ? "lowrank_w1" : "lowrank_w2");
     ce = launch_lowrank(la, grid_y, st, &launches);
   };
+  // a block type's shared 2D-tiled compensator: z = V x, u = C z
+  auto tileq = [&](int block) {
+    const auto& t = L->tq[block];
+    if (ce != cudaSuccess || !t.on) return;
+    TileqArgs ta{};
+    ta.mode = block;
+    ta.x = static_cast<const __nv_bfloat16*>(X);
+    ta.act = static_cast<__half*>(block == 0 ? L->xact.p : L->zact.p);
+    ta.lda = block == 0 ? L->Kpad_x : L->Kpad_z;
+    ta.pinv = ra.pinv;
+    ta.ptok = ra.ptok;
+    ta.pslot = ra.pslot;
+    ta.active = ra.active;
+    ta.n_active = ra.n_active;
+    ta.counts = ra.counts;
+    ta.poffsets = ra.poffsets;
+    ta.T = T;
+    ta.k = top_k;
+    ta.Kin = block == 0 ? K : N;
+    ta.r = t.r;
+    ta.tile_k = t.tile_k;
+    ta.Q = t.Q;
+    ta.P = t.P;
+    ta.v = t.v.p;
+    ta.ct = static_cast<const __nv_bfloat16*>(t.ct.p);
+    ta.z = static_cast<float*>(t.z.p);
+    ta.comp_top_n = L->comp_top_n;
+    prof_mark(L, st, block == 0 ? "tileq_w1" : "tileq_w2");
+    ce = launch_tileq(ta, grid_y, st, &launches);
+  };
   // W1 side compensator U1 = X A1^T
   lowrank(0, static_cast<__half*>(L->xact.p), L->Kpad_x, K,
           make_corr(0, static_cast<const __half*>(L->xact.p), L->Kpad_x, K, static_cast<__half*>(L->corr_x.p),
                     L->ldc_x));
+  tileq(0);
   int ks2 = 1;
   if (prefill) {
     // tcgen05 path: one launch per block, CTAs over (row tile, 256-token pair, expert)
@@ -758,6 +961,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     };
     prefill_gemm(0, L->tmap_x, K, 2 * N, MODE_SWIGLU);
     lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N, CorrArgs{});
+    tileq(1);
     prefill_gemm(1, L->tmap_z, N, K, MODE_OUT);
   } else {
     // tokens per pass: cover the expected per-expert batch (mean + 3 sd);
@@ -796,6 +1000,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N,
             make_corr(1, static_cast<const __half*>(L->zact.p), L->Kpad_z, N, static_cast<__half*>(L->corr_z.p),
                       L->ldc_z));
+    tileq(1);
     // split the down projection's K while its grid is small (fixed-order sum in the combine)
     const int row_tiles = K / decode_rows_per_cta();
     ks2 = std::max(1, 600 / std::max(1, row_tiles * grid_y));

@@ -98,8 +98,10 @@ __device__ void producer(const PrefillArgs& a, const BlockDesc& d, const Ctx& c,
         break;
       }
       mbar_expect_tx(a_full + 8 * slot, c.ntile_live * kATile);
+      // the compensator stage (i == KC) reads the row tile's columns after K
+      const int kx = i < c.KC ? i * kBK : a.K + comp_col_offset(d, rb0);
       for (int t = 0; t < c.ntile_live; ++t)
-        tma_load_2d(smem_u32(sm + kSmemA + slot * kASlot + t * kATile), &a.tmap_act, i * kBK, row0 + t * kTileM,
+        tma_load_2d(smem_u32(sm + kSmemA + slot * kASlot + t * kATile), &a.tmap_act, kx, row0 + t * kTileM,
                     a_full + 8 * slot);
       ++issued_a;
     }

@@ -194,6 +194,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_permute_kernel(RouteArgs 
     prow_s[i] = ppos;
     if (blockIdx.y == 0) {
       a.pslot[ppos] = j;
+      a.ptok[ppos] = t;
       const int pos = a.block_base[bi] + rank;
       a.perm_token[pos] = t;
       a.inv_pos[(long long)t * a.k + j] = pos;

@@ -165,6 +165,40 @@ moe_status_t moe_layer_page_state(moe_layer_t* layer, int expert, int block, int
  * 0 <= n <= max_top_k, else MOE_ERR_INVALID_ARG. */
 moe_status_t moe_layer_set_comp_top_n(moe_layer_t* layer, int n);
 
+/* ---- 2D-tiled shared compensators ----
+ * TileQ: Efficient Low-Rank Quantization of Mixture-of-Experts with 2D Tiling
+ * (abstract: low-rank factors shared across the input and output dimensions
+ * of the experts through 2D tiling; the experts' low-rank terms computed in
+ * one pass). Reading (the page states no formula): one block type of all
+ * experts is cut into P x Q tiles of tile_m rows x tile_k columns; row tile p
+ * has an output factor U_p shared by all column tiles and experts, column tile
+ * q an input factor V_q shared by all row tiles and experts, and expert e an
+ * r x r core per tile; expert e's compensator on tile (p, q) is
+ * U_p * C[e][p][q] * V_q. It replaces every expert's own (A, B) pair of that
+ * block type (their rank in the descriptors is then ignored for it).
+ *
+ * moe_layer_set_tileq: block 0 = W1 (M = 2*d_ff rows [gate; up], K_in =
+ * d_model), 1 = W2 (M = d_model, K_in = d_ff). All inputs bf16, row-major:
+ *   U     [M, rank]              rows p*tile_m .. are U_p
+ *   V     [rank, K_in]           columns q*tile_k .. are V_q
+ *   cores [E][P][Q][rank][rank]  P = M / tile_m, Q = K_in / tile_k;
+ *                                core[e][p][q][i][j] multiplies (V_q x)_j
+ *                                into component i of U_p's input.
+ * rank 16 or 32; tile_m a multiple of 256 that divides d_ff for W1 (the gate
+ * and up halves are tiled separately) or d_model for W2; tile_k a multiple of
+ * 256 dividing K_in. ptr_kind 0 = host pointers, 1 = device pointers; the data
+ * are copied (the caller keeps ownership). Synchronous; must not be called
+ * while a forward is in flight (it may grow the layer's activation buffers).
+ * Errors: MOE_ERR_INVALID_ARG for a bad shape, rank or pointer, MOE_ERR_OOM,
+ * MOE_ERR_CUDA. The forward then computes z_q = V_q x once per token (W1) or
+ * per routed row (W2), u_p = sum_q core[e][p][q] z_q per routed row, and adds
+ * U_p u_p inside the quantised GEMM's compensator stage.
+ * moe_layer_clear_tileq: back to the experts' own compensators (no-op if the
+ * block type has none). Synchronous. */
+moe_status_t moe_layer_set_tileq(moe_layer_t* layer, int block, int rank, int tile_m, int tile_k, const void* U,
+                                 const void* V, const void* cores, int ptr_kind);
+moe_status_t moe_layer_clear_tileq(moe_layer_t* layer, int block);
+
 /* Choose the kernel path (MOE_PATH_*). */
 moe_status_t moe_layer_set_path(moe_layer_t* layer, int path);
 

@@ -287,6 +287,21 @@ def make_block(cfg: LayerConfig, expert: int, block: int, device="cpu", keep_den
                         dense=W if keep_dense else None, raw_codes=raw if keep_raw else None)
 
 
+def make_tileq(cfg: LayerConfig, block: int, rank: int, tile_m: int, tile_k: int, device="cpu",
+               core_std: float = 0.005):
+    """Seeded 2D-tiled shared compensator factors of one block type, bf16:
+    U [M, r] and V [r, K_in] ~ N(0, 1/r), cores [E, P, Q, r, r] ~ N(0, core_std^2)
+    (so that one tile of an expert's compensator has entries of about core_std).
+    Seeds [cid, 2000 + block, tensor_id]."""
+    M, K_in = block_shape(cfg, block)
+    P, Q = M // tile_m, K_in // tile_k
+    std = 1.0 / math.sqrt(rank)
+    U = gaussian((M, rank), std, [cfg.cid, 2000 + block, 0], device, torch.bfloat16)
+    V = gaussian((rank, K_in), std, [cfg.cid, 2000 + block, 1], device, torch.bfloat16)
+    C = gaussian((cfg.E, P, Q, rank, rank), core_std, [cfg.cid, 2000 + block, 2], device, torch.bfloat16)
+    return U, V, C
+
+
 def zipf_bias(E: int, s: float, key: Sequence[int]) -> np.ndarray:
     """bias_e = -s * ln(pi(e) + 1) for a seeded permutation pi of 0..E-1 (the
     logarithm of a Zipf(s) pmf, up to a constant)."""
