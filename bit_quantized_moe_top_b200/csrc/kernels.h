@@ -139,9 +139,11 @@ struct TileqArgs {
   int tile_k, Q;              // column tiles
   int P;                      // row tiles; mode 0: tiles < P/2 are gate tiles, the rest up tiles
   const void* v;              // V [r][Kin] row-major, bf16 (mode 0) or fp16 (mode 1): the MMA's B operand
-  const __nv_bfloat16* ct;    // cores transposed, [E][P][Q][r (input j)][r (output i)]
+  const __half* c16;          // cores [E][P][Q][r (output i)][r (input j)], fp16
   float* z;                   // [sources][Q][r]
   int comp_top_n;             // > 0: routed rows in slots >= comp_top_n get u = 0
+  CorrArgs corr;              // corr.act != nullptr: CTAs past the z grid compute the correction sums
+  int corr_ctas;
 };
 
 struct PrefillArgs {

@@ -96,7 +96,7 @@ struct moe_layer {
   struct Tileq {
     bool on = false;
     int r = 0, tile_m = 0, tile_k = 0, P = 0, Q = 0, cols = 0, span = 0;
-    DevBuf brow, v, ct, z;  // v: V [r][Kin] in the z MMA's operand type (W1 bf16, W2 fp16)
+    DevBuf brow, v, ct, z;  // v: V [r][Kin] in the z MMA's operand type (W1 bf16, W2 fp16); ct: cores, fp16
   } tq[2];
   DevBuf block_counts, block_base, pblock_base, sem, status;
   DevBuf xact, zact, obuf, part, corr_x, corr_z;
@@ -680,20 +680,20 @@ moe_status_t moe_layer_set_tileq(moe_layer_t* L, int block, int rank, int tile_m
   std::vector<uint16_t> hB((size_t)M * cols, 0);
   for (int m = 0; m < M; ++m)
     for (int c = 0; c < r; ++c) hB[(size_t)m * cols + (block == 0 && m >= N ? r : 0) + c] = hU[(size_t)m * r + c];
-  // W2's z MMA multiplies fp16 rows of Z: V in fp16 there (bf16 -> fp16 is
-  // exact for values in fp16's normal range)
-  if (block == 1)
-    for (auto& x : hV) {
-      uint32_t f = (uint32_t)x << 16;
+  // fp16 operands where the MMA's other side is fp16: V of W2 (its z MMA
+  // multiplies fp16 rows of Z) and every core (the u MMA multiplies fp16 z);
+  // bf16 -> fp16 is exact for values in fp16's normal range
+  auto to_half = [](std::vector<uint16_t>& v) {
+    for (auto& x : v) {
+      const uint32_t f = (uint32_t)x << 16;
       float fv;
       std::memcpy(&fv, &f, sizeof(fv));
       const __half h = __float2half_rn(fv);
       std::memcpy(&x, &h, sizeof(x));
     }
-  std::vector<uint16_t> hCt(nC);
-  for (size_t b = 0; b < (size_t)E * P * Q; ++b)
-    for (int i = 0; i < r; ++i)
-      for (int j = 0; j < r; ++j) hCt[b * r * r + (size_t)j * r + i] = hC[b * r * r + (size_t)i * r + j];
+  };
+  if (block == 1) to_half(hV);
+  to_half(hC);
   const long long src_rows = block == 0 ? L->max_tokens : (long long)L->max_tokens * L->max_top_k;
   moe_layer_t::Tileq t;
   DevBuf tmpB;
@@ -708,7 +708,7 @@ moe_status_t moe_layer_set_tileq(moe_layer_t* L, int block, int rank, int tile_m
       ce = launch_relayout_brow(static_cast<const __nv_bfloat16*>(tmpB.p), static_cast<uint32_t*>(t.brow.p), M,
                                 cols, block, N, nullptr);
     if (ce == cudaSuccess) ce = cudaMemcpy(t.v.p, hV.data(), nV * sizeof(uint16_t), cudaMemcpyHostToDevice);
-    if (ce == cudaSuccess) ce = cudaMemcpy(t.ct.p, hCt.data(), nC * sizeof(uint16_t), cudaMemcpyHostToDevice);
+    if (ce == cudaSuccess) ce = cudaMemcpy(t.ct.p, hC.data(), nC * sizeof(uint16_t), cudaMemcpyHostToDevice);
     if (ce == cudaSuccess) ce = cudaDeviceSynchronize();
     if (ce != cudaSuccess) st = MOE_ERR_CUDA;
   }
@@ -864,7 +864,8 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
   auto lowrank = [&](int block, __half* act, int Kpad, int Kin, const CorrArgs& corr) {
     if (ce != cudaSuccess) return;
     if (rmax == 0) {
-      if (corr.act) {
+      // a block type with tiled shared compensators computes the sums in its z launch
+      if (corr.act && !L->tq[block].on) {
         prof_mark(L, st, block == 0 ? "act_corr_w1" : "act_corr_w2");
         ce = launch_act_corr(corr, corr_rows, grid_y, st, &launches);
       }
@@ -900,10 +901,16 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     ce = launch_lowrank(la, grid_y, st, &launches);
   };
   // a block type's shared 2D-tiled compensator: z = V x, u = C z
-  auto tileq = [&](int block) {
+  auto tileq = [&](int block, const CorrArgs& corr) {
     const auto& t = L->tq[block];
     if (ce != cudaSuccess || !t.on) return;
     TileqArgs ta{};
+    if (rmax == 0 && corr.act) {
+      // no low-rank launch carries the correction sums: the z launch does
+      ta.corr = corr;
+      // twice the standalone kernel's CTAs: these CTAs have half its threads
+      ta.corr_ctas = 2 * act_corr_ctas(corr_rows, block == 0 ? K : N);
+    }
     ta.mode = block;
     ta.x = static_cast<const __nv_bfloat16*>(X);
     ta.act = static_cast<__half*>(block == 0 ? L->xact.p : L->zact.p);
@@ -923,17 +930,17 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     ta.Q = t.Q;
     ta.P = t.P;
     ta.v = t.v.p;
-    ta.ct = static_cast<const __nv_bfloat16*>(t.ct.p);
+    ta.c16 = static_cast<const __half*>(t.ct.p);
     ta.z = static_cast<float*>(t.z.p);
     ta.comp_top_n = L->comp_top_n;
     prof_mark(L, st, block == 0 ? "tileq_w1" : "tileq_w2");
     ce = launch_tileq(ta, grid_y, st, &launches);
   };
   // W1 side compensator U1 = X A1^T
-  lowrank(0, static_cast<__half*>(L->xact.p), L->Kpad_x, K,
-          make_corr(0, static_cast<const __half*>(L->xact.p), L->Kpad_x, K, static_cast<__half*>(L->corr_x.p),
-                    L->ldc_x));
-  tileq(0);
+  const CorrArgs corr1 =
+      make_corr(0, static_cast<const __half*>(L->xact.p), L->Kpad_x, K, static_cast<__half*>(L->corr_x.p), L->ldc_x);
+  lowrank(0, static_cast<__half*>(L->xact.p), L->Kpad_x, K, corr1);
+  tileq(0, corr1);
   int ks2 = 1;
   if (prefill) {
     // tcgen05 path: one launch per block, CTAs over (row tile, 256-token pair, expert)
@@ -961,7 +968,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     };
     prefill_gemm(0, L->tmap_x, K, 2 * N, MODE_SWIGLU);
     lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N, CorrArgs{});
-    tileq(1);
+    tileq(1, CorrArgs{});
     prefill_gemm(1, L->tmap_z, N, K, MODE_OUT);
   } else {
     // tokens per pass: cover the expected per-expert batch (mean + 3 sd);
@@ -997,10 +1004,10 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
       ce = launch_decode_gemm(da, ntok, maxbits[block], grid_y, st, &launches);
     };
     decode_gemm(0, L->tmap_xd, L->tmap_cx, K, 2 * N, MODE_SWIGLU, 1);
-    lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N,
-            make_corr(1, static_cast<const __half*>(L->zact.p), L->Kpad_z, N, static_cast<__half*>(L->corr_z.p),
-                      L->ldc_z));
-    tileq(1);
+    const CorrArgs corr2 =
+        make_corr(1, static_cast<const __half*>(L->zact.p), L->Kpad_z, N, static_cast<__half*>(L->corr_z.p), L->ldc_z);
+    lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N, corr2);
+    tileq(1, corr2);
     // split the down projection's K while its grid is small (fixed-order sum in the combine)
     const int row_tiles = K / decode_rows_per_cta();
     ks2 = std::max(1, 600 / std::max(1, row_tiles * grid_y));

@@ -13,18 +13,17 @@
 // multiplies those columns by U_p (its B operand, shared by all experts), so
 // U_p never runs as a separate pass.
 //
-// z: a small GEMM [sources, Kin] x [Kin, r] per column tile on the mma.sync
-// tensor path (16 source rows per CTA, the tile's K range split over four
-// warps, partial sums added in a fixed order). u: per (row tile, expert,
-// 16 routed rows) one CTA stages the expert's cores of that row tile in
-// shared memory, lanes own output components, fp32 FMA.
+// Both are small GEMMs on the mma.sync tensor path. z: [sources, Kin] x
+// [Kin, r] per column tile (the tile's K range split over four warps, partial
+// sums added in a fixed order). u: per (row tile, expert) [rows, Q r] x
+// [Q r, r], with z rounded to fp16 as the A operand and the fp16 cores as B.
+#include "corr.cuh"
 #include "kernels.h"
 
 namespace moeq {
 
 namespace {
 constexpr int kZWarps = 4;
-constexpr int kUQChunk = 8;  // column tiles of cores staged per round (8 x 32 x 32 bf16 = 16 KiB)
 
 __device__ __forceinline__ void mma_16816_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -35,70 +34,93 @@ __device__ __forceinline__ void mma_16816_bf16(float (&d)[4], const uint32_t (&a
 }
 }  // namespace
 
-// grid (Q, ceil(sources / 16)), kZWarps warps: warp w covers the w-th quarter
-// of column tile q's K range for the CTA's 16 source rows.
-template <int MODE>
+// grid (Q + corr CTAs, max(ceil(sources / (16 MT)), corr slots)), kZWarps
+// warps: warp w covers the w-th quarter of column tile q's K range for the
+// CTA's 16 MT source rows (MT m-tiles share each load of V). CTAs past Q
+// compute the decode GEMM's correction sums in the same launch.
+template <int MODE, int MT>
 __global__ void __launch_bounds__(kZWarps * 32) tileq_z_kernel(const TileqArgs a) {
-  __shared__ float red[kZWarps][16][33];
+  __shared__ float red[kZWarps][16 * MT][33];
   pdl_wait();
   pdl_trigger();
+  if ((int)blockIdx.x >= a.Q) {
+    act_corr_rows(a.corr, blockIdx.y, blockIdx.x - a.Q, a.corr_ctas);
+    return;
+  }
   const int q = blockIdx.x;
   const int nsrc = MODE == 0 ? a.T : a.T * a.k;
-  const int s0 = blockIdx.y * 16;
+  const int s0 = blockIdx.y * 16 * MT;
+  if (s0 >= nsrc) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const int NT = a.r / 8;  // n-tiles of 8 outputs
-  // the fragment rows g and g + 8 of the CTA's 16 sources (clamped: rows past
-  // the end load a valid row and are not stored)
-  const int sa = min(s0 + g, nsrc - 1), sb = min(s0 + g + 8, nsrc - 1);
-  const uint32_t* ra;
-  const uint32_t* rb;
-  if constexpr (MODE == 0) {
-    ra = reinterpret_cast<const uint32_t*>(a.x + (long long)sa * a.Kin);
-    rb = reinterpret_cast<const uint32_t*>(a.x + (long long)sb * a.Kin);
-  } else {
-    ra = reinterpret_cast<const uint32_t*>(a.act + (long long)a.pinv[sa] * a.lda);
-    rb = reinterpret_cast<const uint32_t*>(a.act + (long long)a.pinv[sb] * a.lda);
+  // fragment rows g and g + 8 of each m-tile (clamped: rows past the end
+  // load a valid row and are not stored)
+  const uint32_t* ra[MT];
+  const uint32_t* rb[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    const int sa = min(s0 + 16 * m + g, nsrc - 1), sb = min(s0 + 16 * m + g + 8, nsrc - 1);
+    if constexpr (MODE == 0) {
+      ra[m] = reinterpret_cast<const uint32_t*>(a.x + (long long)sa * a.Kin);
+      rb[m] = reinterpret_cast<const uint32_t*>(a.x + (long long)sb * a.Kin);
+    } else {
+      ra[m] = reinterpret_cast<const uint32_t*>(a.act + (long long)a.pinv[sa] * a.lda);
+      rb[m] = reinterpret_cast<const uint32_t*>(a.act + (long long)a.pinv[sb] * a.lda);
+    }
   }
   const uint32_t* v32 = reinterpret_cast<const uint32_t*>(a.v);
   const int ldv = a.Kin / 2;  // V row pitch in u32
   const int steps = a.tile_k / 16;
   const int k0 = q * a.tile_k;
   const int st0 = steps * warp / kZWarps, st1 = steps * (warp + 1) / kZWarps;
-  float acc[4][4];
+  float acc[MT][4][4];
 #pragma unroll
-  for (int t = 0; t < 4; ++t)
+  for (int m = 0; m < MT; ++m)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[t][i] = 0.f;
-#pragma unroll 2
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[m][t][i] = 0.f;
+#pragma unroll 4
   for (int sidx = st0; sidx < st1; ++sidx) {
     const int kw = (k0 + 16 * sidx) / 2 + c;  // u32 column of elements k0 + 16 sidx + 2c
-    uint32_t av[4];
-    av[0] = ra[kw];
-    av[1] = rb[kw];
-    av[2] = ra[kw + 4];
-    av[3] = rb[kw + 4];
+    uint32_t bv[4][2];
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      if (t < NT) {
-        // B[k][n] = V[n][k]: the pair (k, k+1) of output n = 8t + g is one u32 of V's row
-        const uint32_t* vr = v32 + (long long)(8 * t + g) * ldv;
-        if constexpr (MODE == 0) {
-          mma_16816_bf16(acc[t], av, vr[kw], vr[kw + 4]);
-        } else {
-          mma_16816(acc[t], av, vr[kw], vr[kw + 4]);
+      // B[k][n] = V[n][k]: the pair (k, k+1) of output n = 8t + g is one u32 of V's row
+      const uint32_t* vr = v32 + (long long)(8 * min(t, NT - 1) + g) * ldv;
+      bv[t][0] = vr[kw];
+      bv[t][1] = vr[kw + 4];
+    }
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      uint32_t av[4];
+      av[0] = ra[m][kw];
+      av[1] = rb[m][kw];
+      av[2] = ra[m][kw + 4];
+      av[3] = rb[m][kw + 4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        if (t < NT) {
+          if constexpr (MODE == 0) {
+            mma_16816_bf16(acc[m][t], av, bv[t][0], bv[t][1]);
+          } else {
+            mma_16816(acc[m][t], av, bv[t][0], bv[t][1]);
+          }
         }
       }
     }
   }
-  // acc[t][i]: row g + 8 (i >> 1), output 8t + 2c + (i & 1)
+  // acc[m][t][i]: row 16m + g + 8 (i >> 1), output 8t + 2c + (i & 1)
 #pragma unroll
-  for (int t = 0; t < 4; ++t)
-    if (t < NT)
+  for (int m = 0; m < MT; ++m)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) red[warp][g + 8 * (i >> 1)][8 * t + 2 * c + (i & 1)] = acc[t][i];
+    for (int t = 0; t < 4; ++t)
+      if (t < NT)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) red[warp][16 * m + g + 8 * (i >> 1)][8 * t + 2 * c + (i & 1)] = acc[m][t][i];
   __syncthreads();
-  for (int idx = threadIdx.x; idx < 16 * a.r; idx += blockDim.x) {
+  for (int idx = threadIdx.x; idx < 16 * MT * a.r; idx += blockDim.x) {
     const int i = idx / a.r, j = idx % a.r, s = s0 + i;
     if (s >= nsrc) continue;
     float v = 0.f;
@@ -108,10 +130,12 @@ __global__ void __launch_bounds__(kZWarps * 32) tileq_z_kernel(const TileqArgs a
   }
 }
 
-// grid (P, active experts, ceil(max rows per expert / 16)), 8 warps: warp w
-// handles routed rows 2w and 2w + 1 of the CTA's 16 rows of expert e.
-__global__ void __launch_bounds__(256) tileq_u_kernel(const TileqArgs a) {
-  __shared__ __align__(16) __nv_bfloat16 cs[kUQChunk * 32 * 32];
+// u_p = Z C_p^T per (row tile p, expert e) as a small GEMM on the mma.sync
+// path: rows = the expert's routed rows, K = Q r (z of all column tiles, fp16),
+// N = r. grid (P, active experts, ceil(max rows per expert / (64 MT))), four
+// warps, each owning MT m-tiles of 16 routed rows.
+template <int MT>
+__global__ void __launch_bounds__(128) tileq_u_kernel(const TileqArgs a) {
   pdl_wait();
   pdl_trigger();
   const int p = blockIdx.x;
@@ -119,63 +143,105 @@ __global__ void __launch_bounds__(256) tileq_u_kernel(const TileqArgs a) {
   if (slot >= *a.n_active) return;
   const int e = a.active[slot];
   const int n_e = a.counts[e];
-  const int r0 = blockIdx.z * 16;
-  if (r0 >= n_e) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int R = a.r;
-  const int i0 = r0 + 2 * warp, i1 = i0 + 1;
-  const bool v0 = i0 < n_e, v1 = i1 < n_e;
-  const long long pr0 = a.poffsets[e] + min(i0, n_e - 1), pr1 = a.poffsets[e] + min(i1, n_e - 1);
-  const int t0 = a.ptok[pr0], t1 = a.ptok[pr1];
-  const int j0 = a.pslot[pr0], j1 = a.pslot[pr1];
-  const long long src0 = a.mode == 0 ? t0 : (long long)t0 * a.k + j0;
-  const long long src1 = a.mode == 0 ? t1 : (long long)t1 * a.k + j1;
-  const float* z0 = a.z + src0 * a.Q * R;
-  const float* z1 = a.z + src1 * a.Q * R;
-  const __nv_bfloat16* cg = a.ct + ((long long)e * a.P + p) * a.Q * R * R;
-  float acc0 = 0.f, acc1 = 0.f;
-  for (int qb = 0; qb < a.Q; qb += kUQChunk) {
-    const int nq = min(kUQChunk, a.Q - qb);
-    __syncthreads();
-    const int n16 = nq * R * R / 8;  // uint4 units
-    const uint4* src = reinterpret_cast<const uint4*>(cg + (long long)qb * R * R);
-    for (int i = threadIdx.x; i < n16; i += blockDim.x) reinterpret_cast<uint4*>(cs)[i] = src[i];
-    __syncthreads();
-    if (lane < R) {
-      for (int q = 0; q < nq; ++q) {
-        const float* za = z0 + (qb + q) * R;
-        const float* zb = z1 + (qb + q) * R;
-#pragma unroll 8
-        for (int j = 0; j < R; ++j) {
-          const float cv = __bfloat162float(cs[(q * R + j) * R + lane]);
-          acc0 = fmaf(cv, za[j], acc0);
-          acc1 = fmaf(cv, zb[j], acc1);
-        }
-      }
+  const int r0 = (blockIdx.z * 4 + warp) * 16 * MT;
+  if (r0 >= n_e) return;  // no block-level synchronisation below
+  const int g = lane >> 2, c = lane & 3;
+  const int R = a.r, NT = R / 8;
+  long long prow[MT][2];
+  int jslot[MT][2];
+  const float* zr[MT][2];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = min(r0 + 16 * m + g + 8 * h, n_e - 1);
+      prow[m][h] = a.poffsets[e] + i;
+      const int t = a.ptok[prow[m][h]];
+      jslot[m][h] = a.pslot[prow[m][h]];
+      const long long src = a.mode == 0 ? t : (long long)t * a.k + jslot[m][h];
+      zr[m][h] = a.z + src * a.Q * R;
     }
-  }
-  if (lane >= R) return;
-  if (a.comp_top_n > 0) {
-    if (j0 >= a.comp_top_n) acc0 = 0.f;
-    if (j1 >= a.comp_top_n) acc1 = 0.f;
+  // B[k][n] = C[q][n][j] for k = q r + j: the pair (j, j+1) of output n is one u32 of the core's row n
+  const uint32_t* c32 = reinterpret_cast<const uint32_t*>(a.c16) + ((long long)e * a.P + p) * a.Q * R * R / 2;
+  float acc[MT][4][4];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[m][t][i] = 0.f;
+  const int ksteps = a.Q * R / 16;
+#pragma unroll 2
+  for (int kk = 0; kk < ksteps; ++kk) {
+    const int k0 = 16 * kk;
+    const int q = k0 / R, j0 = k0 % R;  // a 16-wide step never crosses a column tile (R = 16 or 32)
+    uint32_t bv[4][2];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int n = 8 * min(t, NT - 1) + g;
+      const uint32_t* cr = c32 + ((long long)q * R + n) * R / 2;
+      bv[t][0] = cr[(j0 + 2 * c) / 2];
+      bv[t][1] = cr[(j0 + 2 * c + 8) / 2];
+    }
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const float2 x0 = *reinterpret_cast<const float2*>(zr[m][0] + k0 + 2 * c);
+      const float2 x1 = *reinterpret_cast<const float2*>(zr[m][1] + k0 + 2 * c);
+      const float2 x2 = *reinterpret_cast<const float2*>(zr[m][0] + k0 + 2 * c + 8);
+      const float2 x3 = *reinterpret_cast<const float2*>(zr[m][1] + k0 + 2 * c + 8);
+      uint32_t av[4];
+      av[0] = pack_half2(x0.x, x0.y);
+      av[1] = pack_half2(x1.x, x1.y);
+      av[2] = pack_half2(x2.x, x2.y);
+      av[3] = pack_half2(x3.x, x3.y);
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        if (t < NT) mma_16816(acc[m][t], av, bv[t][0], bv[t][1]);
+    }
   }
   // W1: gate tile j and up tile P/2 + j sit side by side (2r columns per j),
   // matching the interleaved gate/up rows of one 128-row block
   const int hp = a.P / 2;
   const int col = a.mode == 0 ? (p < hp ? p * 2 * R : (p - hp) * 2 * R + R) : p * R;
-  if (v0) a.act[pr0 * a.lda + a.Kin + col + lane] = __float2half_rn(acc0);
-  if (v1) a.act[pr1 * a.lda + a.Kin + col + lane] = __float2half_rn(acc1);
+  // acc[m][t][i]: row 16m + g + 8 (i >> 1), output 8t + 2c + (i & 1)
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (r0 + 16 * m + g + 8 * h >= n_e) continue;
+      const bool off = a.comp_top_n > 0 && jslot[m][h] >= a.comp_top_n;
+      uint32_t* dst = reinterpret_cast<uint32_t*>(a.act + prow[m][h] * a.lda + a.Kin + col);
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        if (t < NT)
+          dst[(8 * t + 2 * c) / 2] = off ? 0u : pack_half2(acc[m][t][2 * h], acc[m][t][2 * h + 1]);
+    }
 }
 
 cudaError_t launch_tileq(const TileqArgs& a, int grid_y, cudaStream_t st, int* launches) {
   const int nsrc = a.mode == 0 ? a.T : a.T * a.k;
-  const dim3 zg(a.Q, (nsrc + 15) / 16);
-  cudaError_t err = a.mode == 0 ? launch_kernel(tileq_z_kernel<0>, zg, dim3(kZWarps * 32), 0, st, true, a)
-                                : launch_kernel(tileq_z_kernel<1>, zg, dim3(kZWarps * 32), 0, st, true, a);
+  const bool big = nsrc >= 512;
+  const int mt = big ? 4 : 1;
+  const int zy = std::max((nsrc + 16 * mt - 1) / (16 * mt), a.corr.act ? grid_y : 0);
+  const dim3 zg(a.Q + (a.corr.act ? a.corr_ctas : 0), zy);
+  const dim3 zb(kZWarps * 32);
+  cudaError_t err;
+  if (a.mode == 0)
+    err = big ? launch_kernel(tileq_z_kernel<0, 4>, zg, zb, 0, st, true, a)
+              : launch_kernel(tileq_z_kernel<0, 1>, zg, zb, 0, st, true, a);
+  else
+    err = big ? launch_kernel(tileq_z_kernel<1, 4>, zg, zb, 0, st, true, a)
+              : launch_kernel(tileq_z_kernel<1, 1>, zg, zb, 0, st, true, a);
   if (err != cudaSuccess) return err;
   if (launches) ++*launches;
-  // an expert has at most one routed row per token
-  err = launch_kernel(tileq_u_kernel, dim3(a.P, grid_y, (a.T + 15) / 16), dim3(256), 0, st, true, a);
+  // an expert has at most one routed row per token; large batches give each
+  // warp four m-tiles so one load of the cores serves 64 rows
+  const bool many = (long long)a.T * a.k >= 1024;
+  const int rows_cta = many ? 256 : 64;
+  const dim3 ug(a.P, grid_y, (a.T + rows_cta - 1) / rows_cta);
+  err = many ? launch_kernel(tileq_u_kernel<4>, ug, dim3(128), 0, st, true, a)
+             : launch_kernel(tileq_u_kernel<1>, ug, dim3(128), 0, st, true, a);
   if (err == cudaSuccess && launches) ++*launches;
   return err;
 }
