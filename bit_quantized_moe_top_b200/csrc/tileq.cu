@@ -132,10 +132,14 @@ __global__ void __launch_bounds__(kZWarps * 32) tileq_z_kernel(const TileqArgs a
 
 // u_p = Z C_p^T per (row tile p, expert e) as a small GEMM on the mma.sync
 // path: rows = the expert's routed rows, K = Q r (z of all column tiles, fp16),
-// N = r. grid (P, active experts, ceil(max rows per expert / (64 MT))), four
-// warps, each owning MT m-tiles of 16 routed rows.
-template <int MT>
+// N = r. Large batches (SPLITK false): grid (P, active experts,
+// ceil(max rows per expert / (64 MT))), four warps each owning MT m-tiles of
+// 16 routed rows. Small batches (SPLITK true, MT = 1): grid (P, active
+// experts, ceil(max rows per expert / 16)), the four warps split K for the
+// CTA's 16 rows and their partials are added in a fixed order.
+template <int MT, bool SPLITK>
 __global__ void __launch_bounds__(128) tileq_u_kernel(const TileqArgs a) {
+  __shared__ float red[SPLITK ? 4 : 1][16][33];
   pdl_wait();
   pdl_trigger();
   const int p = blockIdx.x;
@@ -144,8 +148,8 @@ __global__ void __launch_bounds__(128) tileq_u_kernel(const TileqArgs a) {
   const int e = a.active[slot];
   const int n_e = a.counts[e];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r0 = (blockIdx.z * 4 + warp) * 16 * MT;
-  if (r0 >= n_e) return;  // no block-level synchronisation below
+  const int r0 = SPLITK ? blockIdx.z * 16 : (blockIdx.z * 4 + warp) * 16 * MT;
+  if (r0 >= n_e) return;  // uniform over the CTA when SPLITK (its only block-level synchronisation)
   const int g = lane >> 2, c = lane & 3;
   const int R = a.r, NT = R / 8;
   long long prow[MT][2];
@@ -172,8 +176,9 @@ __global__ void __launch_bounds__(128) tileq_u_kernel(const TileqArgs a) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[m][t][i] = 0.f;
   const int ksteps = a.Q * R / 16;
+  const int kk0 = SPLITK ? ksteps * warp / 4 : 0, kk1 = SPLITK ? ksteps * (warp + 1) / 4 : ksteps;
 #pragma unroll 2
-  for (int kk = 0; kk < ksteps; ++kk) {
+  for (int kk = kk0; kk < kk1; ++kk) {
     const int k0 = 16 * kk;
     const int q = k0 / R, j0 = k0 % R;  // a 16-wide step never crosses a column tile (R = 16 or 32)
     uint32_t bv[4][2];
@@ -205,6 +210,23 @@ __global__ void __launch_bounds__(128) tileq_u_kernel(const TileqArgs a) {
   const int hp = a.P / 2;
   const int col = a.mode == 0 ? (p < hp ? p * 2 * R : (p - hp) * 2 * R + R) : p * R;
   // acc[m][t][i]: row 16m + g + 8 (i >> 1), output 8t + 2c + (i & 1)
+  if constexpr (SPLITK) {
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      if (t < NT)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) red[warp][g + 8 * (i >> 1)][8 * t + 2 * c + (i & 1)] = acc[0][t][i];
+    __syncthreads();
+    if (warp != 0) return;
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      if (t < NT)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int rr = g + 8 * (i >> 1), cc = 8 * t + 2 * c + (i & 1);
+          acc[0][t][i] = red[0][rr][cc] + red[1][rr][cc] + red[2][rr][cc] + red[3][rr][cc];
+        }
+  }
 #pragma unroll
   for (int m = 0; m < MT; ++m)
 #pragma unroll
@@ -238,10 +260,10 @@ cudaError_t launch_tileq(const TileqArgs& a, int grid_y, cudaStream_t st, int* l
   // an expert has at most one routed row per token; large batches give each
   // warp four m-tiles so one load of the cores serves 64 rows
   const bool many = (long long)a.T * a.k >= 1024;
-  const int rows_cta = many ? 256 : 64;
+  const int rows_cta = many ? 256 : 16;
   const dim3 ug(a.P, grid_y, (a.T + rows_cta - 1) / rows_cta);
-  err = many ? launch_kernel(tileq_u_kernel<4>, ug, dim3(128), 0, st, true, a)
-             : launch_kernel(tileq_u_kernel<1>, ug, dim3(128), 0, st, true, a);
+  err = many ? launch_kernel(tileq_u_kernel<4, false>, ug, dim3(128), 0, st, true, a)
+             : launch_kernel(tileq_u_kernel<1, true>, ug, dim3(128), 0, st, true, a);
   if (err == cudaSuccess && launches) ++*launches;
   return err;
 }
