@@ -44,6 +44,9 @@ def parse():
     p.add_argument("--tileq", type=int, default=0,
                    help="rank of 2D-tiled shared compensators on both blocks (replacing the per-expert ones); 0 = off")
     p.add_argument("--tile-m", type=int, default=1024)
+    p.add_argument("--redraw-bits", type=int, default=-1,
+                   help="bit-plane configs: before timing, re-draw every block's bitwidth from {2,3,4} with this "
+                        "seed and commit it with moe_layer_set_bits")
     p.add_argument("--tile-k", type=int, default=1024)
     return p.parse_args()
 
@@ -299,6 +302,10 @@ def main():
         # the tiled shared compensators replace every expert's own pair
         cfg.experts = [ms.ExpertSpec(sp.fmt, sp.bits, sp.group, 0) for sp in cfg.experts]
     workload = f"{WORKLOADS[args.config]}_T{T}" + (f"_tileq_r{tq[0]}_{tq[1]}x{tq[2]}" if tq else "")
+    if args.redraw_bits >= 0:
+        if any(sp.fmt != ms.FMT_BITPLANE_LUT for sp in cfg.experts):
+            raise SystemExit("--redraw-bits needs a bit-plane configuration")
+        workload += f"_bits_redrawn_{args.redraw_bits}"
 
     if args.impl == "reference":
         if rank != 0:
@@ -341,6 +348,16 @@ def main():
         for b in (0, 1):
             blocks[(e, b)] = ms.make_block(cfg, e, b, device=dev)
     L = build_layer(bq, cfg, blocks, max_tokens=T)
+    if args.redraw_bits >= 0:
+        # one set_bits re-draw of every (expert, block): the kernels then read the new number of planes
+        import numpy as np
+        rng = np.random.default_rng(np.random.SeedSequence([cfg.cid, 3000, args.redraw_bits]))
+        new = rng.integers(2, 5, size=(cfg.E, 2))
+        for e in range(cfg.E):
+            for b in (0, 1):
+                L.set_bits(e, b, int(new[e, b]))
+        cfg.experts = [ms.ExpertSpec(sp.fmt, (int(new[e, 0]), int(new[e, 1])), sp.group, sp.rank)
+                       for e, sp in enumerate(cfg.experts)]
     if tq:
         for b in (0, 1):
             U, V, C = ms.make_tileq(cfg, b, tq[0], tq[1], tq[2], dev)
@@ -380,6 +397,8 @@ def main():
         torch.cuda.synchronize()
     L.set_profiling(False)
     step_ms = [a.elapsed_time(b) for a, b in ev]
+    pct = {q: statistics.quantiles(step_ms, n=10)[i] if len(step_ms) >= 2 else step_ms[0]
+           for q, i in (("p10", 0), ("p50", 4), ("p90", 8))}
     total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
     value = weak_scaling_value(world, T, ms_per_step)
@@ -455,6 +474,7 @@ def main():
                        "l2": "flushed between steps (256 MiB write, untimed)",
                        **({"compensator": {"kind": "2D-tiled shared factors", "rank": tq[0], "tile_m": tq[1],
                                            "tile_k": tq[2]}} if tq else {})},
+            "ms_per_step_percentiles": pct,
             "layer_hbm_gbs": layer_b / (ms_per_step * 1e-3) / 1e9,
             "layer_tflops": layer_f / (ms_per_step * 1e-3) / 1e12,
             "layer_bytes_per_step": layer_b,

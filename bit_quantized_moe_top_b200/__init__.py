@@ -21,6 +21,7 @@ STATUS_NAMES = ["MOE_OK", "MOE_ERR_INVALID_ARG", "MOE_ERR_OOM", "MOE_ERR_NOT_LOA
                 "MOE_ERR_TOO_LARGE"]
 FMT_INT_ASYM, FMT_BITPLANE_LUT, FMT_DENSE16 = 0, 1, 2
 FLAG_NO_TOPK_RENORM = 1
+FLAG_DETERMINISTIC = 2
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 
 # every symbol the header declares

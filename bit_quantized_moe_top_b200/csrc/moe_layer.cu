@@ -231,7 +231,7 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   if (!out) return MOE_ERR_INVALID_ARG;
   *out = nullptr;
   if (!descs || E < 1 || E > kMaxExperts || K < 128 || N < 128 || K % 128 || N % 128 || max_tokens < 1 ||
-      max_top_k < 1 || max_top_k > kMaxTopK || max_top_k > E || (flags & ~MOE_FLAG_NO_TOPK_RENORM))
+      max_top_k < 1 || max_top_k > kMaxTopK || max_top_k > E || (flags & ~(MOE_FLAG_NO_TOPK_RENORM | MOE_FLAG_DETERMINISTIC)))
     return MOE_ERR_INVALID_ARG;
   int rmax = 0;
   for (int e = 0; e < E; ++e) {
@@ -860,6 +860,10 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     return ca;
   };
   const int corr_rows = (int)std::min<long long>(T, rows);
+  // correction-sum CTAs per expert slot, at most about 2048 over all slots:
+  // sized for one expert taking every token, the count grows with E while
+  // most slots hold a few rows (the CTAs loop over their items)
+  const int corr_cap = std::max(8, std::min(256, 2048 / std::max(1, grid_y)));
   // the low-rank down-projection, with the correction sums in the same launch
   auto lowrank = [&](int block, __half* act, int Kpad, int Kin, const CorrArgs& corr) {
     if (ce != cudaSuccess) return;
@@ -873,7 +877,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     }
     LowrankArgs la{};
     la.corr = corr;
-    la.corr_ctas = corr.act ? act_corr_ctas(corr_rows, Kin) : 0;
+    la.corr_ctas = corr.act ? std::min(act_corr_ctas(corr_rows, Kin), corr_cap) : 0;
     la.experts = dexp;
     la.block = block;
     la.active = ra.active;
@@ -909,7 +913,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
       // no low-rank launch carries the correction sums: the z launch does
       ta.corr = corr;
       // twice the standalone kernel's CTAs: these CTAs have half its threads
-      ta.corr_ctas = 2 * act_corr_ctas(corr_rows, block == 0 ? K : N);
+      ta.corr_ctas = 2 * std::min(act_corr_ctas(corr_rows, block == 0 ? K : N), corr_cap);
     }
     ta.mode = block;
     ta.x = static_cast<const __nv_bfloat16*>(X);

@@ -99,6 +99,9 @@ typedef struct moe_layer moe_layer_t; /* opaque */
 
 /* flags for moe_layer_create */
 #define MOE_FLAG_NO_TOPK_RENORM 1u /* w[t, j] = full-softmax probability of the selected expert */
+#define MOE_FLAG_DETERMINISTIC 2u  /* bitwise-repeatable results; always the case here (no floating-point
+                                      atomics: split sums are added in a fixed order), so the flag is
+                                      accepted and changes nothing */
 
 /* paths for moe_layer_set_path */
 #define MOE_PATH_AUTO 0    /* by T: decode kernels for small batches, prefill kernels above */
