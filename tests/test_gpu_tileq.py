@@ -190,3 +190,30 @@ def test_mixtral_tileq_full_size_sampled_rows():
     ref = _oracle(cfg, blocks, tq, X, logits, 2, rows=rows, fold=True)
     assert_parity(Y[rows], ref["Y"], "mixtral tiled full")
     L.close()
+
+
+@pytest.mark.parametrize("path,T", [("decode", 24), ("prefill", 300)])
+def test_tileq_on_bitplane_experts_and_set_bits(path, T):
+    """Tiled shared compensators on bit-plane + LUT experts (PagedWeight format),
+    then one set_bits on a block: the shared factors stay in force."""
+    base = ms.make_config("dsv3_bitplane")
+    cfg = ms.scaled_config(base, E=8, K=512, N=768, top_k=2)
+    cfg.experts = [ms.ExpertSpec(ms.FMT_BITPLANE_LUT, (3, 4), 0, 0) for _ in range(cfg.E)]
+    blocks = make_blocks(cfg, DEV)
+    L = make_layer(cfg, blocks, max_tokens=T)
+    L.set_path(PATHS[path])
+    tq = _tileq(cfg, L, (0, 1), 32, TILES)
+    X, logits = ms.make_inputs(cfg, T, DEV)
+    Y = L.forward(X, logits, 2)
+    assert L.sync_status() == 0
+    ref = _oracle(cfg, blocks, tq, X, logits, 2)
+    assert_parity(Y, ref["Y"], f"{path} bit-plane tiled")
+    L.set_bits(3, 0, 2)
+    Y2 = L.forward(X, logits, 2)
+    assert L.sync_status() == 0
+    from oracle import moe_oracle as mo
+    ex = TileqExperts(blocks, tq)
+    ex.bits_override = {(3, 0): 2}
+    ref2 = mo.moe_forward(_np(X), logits.cpu().numpy(), 2, ex, cfg.N)
+    assert_parity(Y2, ref2["Y"], f"{path} bit-plane tiled after set_bits")
+    L.close()
