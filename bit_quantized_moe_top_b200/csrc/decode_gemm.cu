@@ -63,14 +63,17 @@ constexpr int kProdWarp = kDqWarps + kEpWarps, kMmaWarp = kProdWarp + 1;
 constexpr int kThreads = 32 * (kMmaWarp + 1);
 constexpr int kRows = 128;
 constexpr int kMaxStages = 16;  // stage ring depth: as many as about 100 KiB of shared memory hold
-constexpr int kA = 3;           // TMEM A buffers
-constexpr int kAcc = 2;         // TMEM accumulators
-constexpr int kACols = 40;      // per A buffer: 32 code columns + 8 correction columns
-constexpr int kABase = 128;     // accumulators at [0, kAcc * NTOK), A buffers at [128, 248)
+constexpr int kSub = 2;         // 64-wide chunks per barrier round (step)
+constexpr int kA = 2;           // TMEM A buffers, one per step
+constexpr int kAcc = 3;         // TMEM accumulators (one per quantisation group; a step may hold two)
+constexpr int kACols = 40;      // per chunk: 32 code columns + 8 correction columns
+constexpr int kAStep = kSub * kACols;
+constexpr int kABase = 96;      // accumulators at [0, kAcc * NTOK), A buffers at [96, 256)
 constexpr int kTmemCols = 256;
 constexpr int kActBox = 16;     // rows per TMA box
 constexpr uint32_t kOne1024 = 0x64006400u;  // fp16 pair (1024, 1024)
-static_assert(kABase + kA * kACols <= kTmemCols, "TMEM rings exceed the allocation");
+static_assert(kABase + kA * kAStep <= kTmemCols, "TMEM rings exceed the allocation");
+static_assert(kAcc * 32 <= kABase, "accumulators overlap the A buffers");
 
 // barrier slots (8 bytes each)
 constexpr int kBarFull = 0, kBarEmpty = kMaxStages, kBarAFull = 2 * kMaxStages, kBarAEmpty = kBarAFull + kA,
@@ -79,11 +82,13 @@ constexpr int kBarFull = 0, kBarEmpty = kMaxStages, kBarAFull = 2 * kMaxStages, 
 
 // code block bytes of a 128-row x 64-k chunk at the largest bitwidth of the block's experts
 __host__ __device__ inline int code_bytes(int maxbits) { return maxbits >= 16 ? 16384 : 1024 * maxbits; }
-// stage: [act NTOK x 128 B][corr NTOK x 32 B][codes][scales 512 B]
-__host__ __device__ inline int stage_bytes(int ntok, int maxbits) {
+// one chunk's part of a stage: [act NTOK x 128 B][corr NTOK x 32 B][codes][scales 512 B];
+// a stage holds kSub of them (one step)
+__host__ __device__ inline int sub_stage_bytes(int ntok, int maxbits) {
   const int b = ntok * 160 + code_bytes(maxbits) + 512;
   return (b + 1023) & ~1023;
 }
+__host__ __device__ inline int stage_bytes(int ntok, int maxbits) { return kSub * sub_stage_bytes(ntok, maxbits); }
 
 // position in a ring of n slots with the phase parity of the current lap
 struct RingPos {
@@ -104,11 +109,11 @@ struct Ctx {
 
 // per-role ring positions, kept across tiles
 struct Pos {
-  RingPos st;   // stage ring
-  RingPos rel;  // stage to release (unpack warps: kA chunks behind st)
-  RingPos ab;   // A buffer ring
-  RingPos acc;  // accumulator ring
-  int chunks = 0;
+  RingPos st;   // stage ring (one stage per step of kSub chunks)
+  RingPos rel;  // stage to release (unpack warps: kA steps behind st)
+  RingPos ab;   // A buffer ring (one buffer per step)
+  RingPos acc;  // accumulator ring (one per group)
+  int steps = 0;
 };
 
 // group position of chunk i of a tile: first / last chunk of its accumulator group
@@ -136,40 +141,52 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
   const int nbox = (n_pass + kActBox - 1) / kActBox;
   const int row0 = c.prow0 + c.tok0;
   const uint8_t* codes = (FMT == FMT_BITPLANE) ? d.plane[0] : d.codes;
+  const int sub_b = stage_b / kSub;
+  const int n = c.nmain + c.next;
   // the whole warp runs the loop (warp-uniform values); one lane issues the copies
-  for (int i = 0; i < c.nmain + c.next; ++i, ps.st.next(a.nstages)) {
+  for (int i0 = 0; i0 < n; i0 += kSub, ps.st.next(a.nstages)) {
     if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait_fast(empty + 8 * ps.st.idx, ps.st.ph ^ 1u, a.status))) {
       *abort_flag = 1;
       return;
     }
-    bool first, last;
-    group_pos<FMT, GROUP>(c, i, first, last);
-    const uint32_t st = smem_u32(sm) + ps.st.idx * stage_b;
     const uint32_t fb = full + 8 * ps.st.idx;
-    const bool main = i < c.nmain;
-    const int kc = c.kc0 + i;
-    const bool corr = FMT == FMT_INT && main && first;
-    uint32_t bytes = nbox * kActBox * 128;
-    if (main) bytes += (FMT == FMT_BITPLANE ? BITS * 1024 : kBlk);
-    if (corr) bytes += nbox * kActBox * 32 + 512;
-    const int kx = main ? kc * 64 : a.K + comp_col_offset(d, c.rb);
-    const uint32_t cs = st + NTOK * 160;
-    const long long bidx = (long long)kc * RB + c.rb;
-    const int g = kc * 64 / GROUP;
+    const int nsub = min(kSub, n - i0);
+    uint32_t bytes = 0;
+    for (int u = 0; u < nsub; ++u) {
+      bool first, last;
+      group_pos<FMT, GROUP>(c, i0 + u, first, last);
+      const bool main = i0 + u < c.nmain;
+      bytes += nbox * kActBox * 128;
+      if (main) bytes += (FMT == FMT_BITPLANE ? BITS * 1024 : kBlk);
+      if (FMT == FMT_INT && main && first) bytes += nbox * kActBox * 32 + 512;
+    }
     if (elect_one()) {
       mbar_expect_tx(fb, bytes);
-      for (int b = 0; b < nbox; ++b) tma_load_2d(st + b * kActBox * 128, &a.tmap_act, kx, row0 + b * kActBox, fb);
-      if (main) {
-        if constexpr (FMT == FMT_BITPLANE) {
+      for (int u = 0; u < nsub; ++u) {
+        const int i = i0 + u;
+        bool first, last;
+        group_pos<FMT, GROUP>(c, i, first, last);
+        const uint32_t st = smem_u32(sm) + ps.st.idx * stage_b + u * sub_b;
+        const bool main = i < c.nmain;
+        const int kc = c.kc0 + i;
+        const bool corr = FMT == FMT_INT && main && first;
+        const int kx = main ? kc * 64 : a.K + comp_col_offset(d, c.rb);
+        const uint32_t cs = st + NTOK * 160;
+        const long long bidx = (long long)kc * RB + c.rb;
+        const int g = kc * 64 / GROUP;
+        for (int b = 0; b < nbox; ++b) tma_load_2d(st + b * kActBox * 128, &a.tmap_act, kx, row0 + b * kActBox, fb);
+        if (main) {
+          if constexpr (FMT == FMT_BITPLANE) {
 #pragma unroll
-          for (int q = 0; q < BITS; ++q) bulk_g2s(cs + q * 1024, d.plane[q] + bidx * 1024, 1024, fb);
-        } else {
-          bulk_g2s(cs, codes + bidx * kBlk, kBlk, fb);
-        }
-        if (corr) {
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d(st + NTOK * 128 + b * kActBox * 32, &a.tmap_corr, 16 * g, row0 + b * kActBox, fb);
-          bulk_g2s(cs + cbytes, d.sz + (long long)g * a.M + c.rb * kRows, 512, fb);
+            for (int q = 0; q < BITS; ++q) bulk_g2s(cs + q * 1024, d.plane[q] + bidx * 1024, 1024, fb);
+          } else {
+            bulk_g2s(cs, codes + bidx * kBlk, kBlk, fb);
+          }
+          if (corr) {
+            for (int b = 0; b < nbox; ++b)
+              tma_load_2d(st + NTOK * 128 + b * kActBox * 32, &a.tmap_corr, 16 * g, row0 + b * kActBox, fb);
+            bulk_g2s(cs + cbytes, d.sz + (long long)g * a.M + c.rb * kRows, 512, fb);
+          }
         }
       }
     }
@@ -186,33 +203,48 @@ __device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int s
   const int n_pass = min(NTOK, c.n_e - c.tok0);
   const uint32_t idesc = idesc_f16(128, (n_pass + 15) & ~15);
   const uint32_t sm0 = smem_u32(sm);
-  for (int i = 0; i < c.nmain + c.next; ++i) {
-    bool first, last;
-    group_pos<FMT, GROUP>(c, i, first, last);
+  const int sub_b = stage_b / kSub;
+  const int n = c.nmain + c.next;
+  for (int i0 = 0; i0 < n; i0 += kSub) {
     const bool ok = !*abort_flag && mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status) &&
-                    mbar_wait_fast(afull + 8 * ps.ab.idx, ps.ab.ph, a.status) &&
-                    (!first || mbar_wait_fast(accfree + 8 * ps.acc.idx, ps.acc.ph ^ 1u, a.status));
+                    mbar_wait_fast(afull + 8 * ps.ab.idx, ps.ab.ph, a.status);
     if (!__all_sync(0xffffffffu, ok)) {
       *abort_flag = 1;
       return;
     }
     tc_fence_after();
-    const uint32_t bt = sm0 + ps.st.idx * stage_b;
-    const uint32_t acc = tmem + ps.acc.idx * NTOK;
-    const uint32_t ta = tmem + kABase + ps.ab.idx * kACols;
-    const bool corr = FMT == FMT_INT && i < c.nmain && first;
-    const uint64_t dact = sw128_desc(bt), dcorr = sw32_desc(bt + NTOK * 128);
-    // the whole warp runs the loop (warp-uniform values); one lane issues
-    if (elect_one()) {
-      if (corr) mma_f16_ts(acc, ta + 32, dcorr, idesc, 0);
+    const int nsub = min(kSub, n - i0);
+    for (int u = 0; u < nsub; ++u) {
+      const int i = i0 + u;
+      bool first, last;
+      group_pos<FMT, GROUP>(c, i, first, last);
+      if (first) {
+        if (!__all_sync(0xffffffffu,
+                        !*abort_flag && mbar_wait_fast(accfree + 8 * ps.acc.idx, ps.acc.ph ^ 1u, a.status))) {
+          *abort_flag = 1;
+          return;
+        }
+        tc_fence_after();
+      }
+      const uint32_t bt = sm0 + ps.st.idx * stage_b + u * sub_b;
+      const uint32_t acc = tmem + ps.acc.idx * NTOK;
+      const uint32_t ta = tmem + kABase + ps.ab.idx * kAStep + u * kACols;
+      const bool corr = FMT == FMT_INT && i < c.nmain && first;
+      const uint64_t dact = sw128_desc(bt), dcorr = sw32_desc(bt + NTOK * 128);
+      // the whole warp runs the loop (warp-uniform values); one lane issues
+      if (elect_one()) {
+        if (corr) mma_f16_ts(acc, ta + 32, dcorr, idesc, 0);
 #pragma unroll
-      for (int k16 = 0; k16 < 4; ++k16)
-        mma_f16_ts(acc, ta + k16 * 8, dact + 2 * k16, idesc, (corr || !first || k16 > 0) ? 1 : 0);
-      mma_commit(aempty + 8 * ps.ab.idx);
-      if (last) mma_commit(accfull + 8 * ps.acc.idx);
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_f16_ts(acc, ta + k16 * 8, dact + 2 * k16, idesc, (corr || !first || k16 > 0) ? 1 : 0);
+        if (last) mma_commit(accfull + 8 * ps.acc.idx);
+      }
+      __syncwarp();
+      if (last) ps.acc.next(kAcc);
     }
+    // the step's A buffer and stage are read once all its MMAs complete
+    if (elect_one()) mma_commit(aempty + 8 * ps.ab.idx);
     __syncwarp();
-    if (last) ps.acc.next(kAcc);
     ps.st.next(a.nstages);
     ps.ab.next(kA);
   }
@@ -230,9 +262,9 @@ __device__ void unpack(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, ui
   if constexpr (FMT == FMT_BITPLANE) lut = load_lut(d.lut, BITS);
   const int RS2 = d.rank / 2;  // compensator column pairs
   const int R = c.rb * kRows + row;
-  for (int i = 0; i < c.nmain + c.next; ++i) {
-    bool first, last;
-    group_pos<FMT, GROUP>(c, i, first, last);
+  const int sub_b = stage_b / kSub;
+  const int n = c.nmain + c.next;
+  for (int i0 = 0; i0 < n; i0 += kSub) {
     // warp-uniform waits: every lane reaches the .sync.aligned TMEM stores
     const bool ok = !*abort_flag && mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status) &&
                     mbar_wait_fast(aempty + 8 * ps.ab.idx, ps.ab.ph ^ 1u, a.status);
@@ -240,57 +272,63 @@ __device__ void unpack(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, ui
       *abort_flag = 1;
       return;
     }
-    // the MMAs of chunk (this - kA) are complete: its stage (codes read by
+    // the MMAs of step (this - kA) are complete: its stage (codes read by
     // these warps, activations read by the MMAs) may be refilled
-    if (ps.chunks >= kA) {
+    if (ps.steps >= kA) {
       if (lane == 0) mbar_arrive(empty + 8 * ps.rel.idx);
       ps.rel.next(a.nstages);
     }
-    const uint32_t ta = tmem + lane_base + kABase + ps.ab.idx * kACols;
-    uint32_t v[32];
-    if (i < c.nmain) {
-      const uint8_t* cs = sm + ps.st.idx * stage_b + NTOK * 160;
-      if constexpr (FMT == FMT_INT) {
-        if (first) {
-          const uint32_t sz = reinterpret_cast<const uint32_t*>(cs + cbytes)[row];
-          tmem_st1_nw(ta + 33, prmt(sz, sz, 0x3232u));  // (z, z) against (-X_hi, -X_lo)
-        }
+    const int nsub = min(kSub, n - i0);
+    for (int u = 0; u < nsub; ++u) {
+      const int i = i0 + u;
+      bool first, last;
+      group_pos<FMT, GROUP>(c, i, first, last);
+      const uint32_t ta = tmem + lane_base + kABase + ps.ab.idx * kAStep + u * kACols;
+      uint32_t v[32];
+      if (i < c.nmain) {
+        const uint8_t* cs = sm + ps.st.idx * stage_b + u * sub_b + NTOK * 160;
+        if constexpr (FMT == FMT_INT) {
+          if (first) {
+            const uint32_t sz = reinterpret_cast<const uint32_t*>(cs + cbytes)[row];
+            tmem_st1_nw(ta + 33, prmt(sz, sz, 0x3232u));  // (z, z) against (-X_hi, -X_lo)
+          }
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t w[4], r16[16];
-          load_half_words_int<BITS>(cs, row, h, w);
-          int_raw_half<BITS>(w, r16);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t w[4], r16[16];
+            load_half_words_int<BITS>(cs, row, h, w);
+            int_raw_half<BITS>(w, r16);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[16 * h + j] = r16[j];
-        }
-      } else if constexpr (FMT == FMT_BITPLANE) {
+            for (int j = 0; j < 16; ++j) v[16 * h + j] = r16[j];
+          }
+        } else if constexpr (FMT == FMT_BITPLANE) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pw[4], r16[16];
-          load_half_planes<BITS>(cs, 1024, row, h, pw);
-          lut_half<BITS>(pw, lut, r16);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pw[4], r16[16];
+            load_half_planes<BITS>(cs, 1024, row, h, pw);
+            lut_half<BITS>(pw, lut, r16);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[16 * h + j] = r16[j];
+            for (int j = 0; j < 16; ++j) v[16 * h + j] = r16[j];
+          }
+        } else {
+#pragma unroll
+          for (int qd = 0; qd < 8; ++qd) {
+            const uint4 x = reinterpret_cast<const uint4*>(cs + qd * 2048)[row];
+            v[4 * qd] = x.x; v[4 * qd + 1] = x.y; v[4 * qd + 2] = x.z; v[4 * qd + 3] = x.w;
+          }
         }
       } else {
+        // compensator stage: the row's B values (pairs), zero past the rank
 #pragma unroll
-        for (int qd = 0; qd < 8; ++qd) {
-          const uint4 x = reinterpret_cast<const uint4*>(cs + qd * 2048)[row];
-          v[4 * qd] = x.x; v[4 * qd + 1] = x.y; v[4 * qd + 2] = x.z; v[4 * qd + 3] = x.w;
-        }
+        for (int j = 0; j < 32; ++j) v[j] = j < RS2 ? d.brow[(long long)j * a.M + R] : 0u;
       }
-    } else {
-      // compensator stage: the row's B values (pairs), zero past the rank
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = j < RS2 ? d.brow[(long long)j * a.M + R] : 0u;
+      tmem_st32(ta, v);  // includes the wait for the store
     }
-    tmem_st32(ta, v);  // includes the wait for the store
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(afull + 8 * ps.ab.idx);
     ps.st.next(a.nstages);
     ps.ab.next(kA);
-    ++ps.chunks;
+    ++ps.steps;
   }
 }
 
@@ -421,7 +459,7 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
     // constant correction columns of the A buffers: (1024, 1024), then zeros
     const uint32_t lb = (uint32_t)(warp * 32) << 16;
     const uint32_t cz[8] = {dk::kOne1024, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-    for (int b = 0; b < dk::kA; ++b) tmem_st8_nw(tmem + lb + dk::kABase + b * dk::kACols + 32, cz);
+    for (int b = 0; b < dk::kA * dk::kSub; ++b) tmem_st8_nw(tmem + lb + dk::kABase + b * dk::kACols + 32, cz);
     tmem_wait_st();
   }
   // everything above overlaps the previous kernel's tail
@@ -577,9 +615,10 @@ template <int NTOK>
 static cudaError_t launch_ntok(const DecodeArgs& a, int maxbits, int grid_y, cudaStream_t st) {
   const int stage_b = dk::stage_bytes(NTOK, maxbits);
   // two CTAs per SM (2 x 256 TMEM columns): each takes about 100 KiB of
-  // stages, as deep a ring as fits, to keep enough weight bytes in flight
-  // (a stage is released kA chunks after its own; kA + 2 stages keep the
-  // producer ahead, even for the large dense code blocks)
+  // stages (a stage holds one step of kSub chunks), as deep a ring as fits,
+  // to keep enough weight bytes in flight (a stage is released kA steps
+  // after its own; kA + 2 stages keep the producer ahead, even for the large
+  // dense code blocks, which then leave room for one CTA per SM)
   DecodeArgs b = a;
   b.nstages = std::max(dk::kA + 2, std::min(dk::kMaxStages, (100 * 1024 - 1024) / stage_b));
   const size_t smem = (size_t)b.nstages * stage_b + 1024;
