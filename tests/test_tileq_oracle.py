@@ -115,3 +115,32 @@ def test_factor_count_closed_form():
     assert n == 2 * 14336 * 32 + 32 * 4096 + 8 * 28 * 4 * 32 * 32
     per_expert = 8 * (2 * 14336 + 4096) * 32
     assert per_expert / n > 4.0
+
+
+def test_top_n_with_tiled_compensators_matches_factored_path():
+    # top-n compensation (only the first n routing slots compensated) must
+    # treat the dense tiled form exactly as the factored (A, B) form
+    rng = np.random.default_rng(7)
+    E, K, N, T, k, r = 4, 8, 8, 6, 3, 2
+    W1 = rng.standard_normal((E, 2 * N, K)) * 0.3
+    W2 = rng.standard_normal((E, K, N)) * 0.3
+    U1, V1 = rng.standard_normal((2 * N, r)), rng.standard_normal((r, K))
+    U2, V2 = rng.standard_normal((K, r)), rng.standard_normal((r, N))
+    I1 = np.broadcast_to(np.eye(r), (2 * N // 4, K // 4, r, r))
+    I2 = np.broadcast_to(np.eye(r), (K // 4, N // 4, r, r))
+    X = rng.standard_normal((T, K))
+    logits = rng.standard_normal((T, E))
+
+    def tiled(e):
+        return {"W1": W1[e], "W2": W2[e], "D1": tq.tileq_delta(U1, V1, I1, 4, 4),
+                "D2": tq.tileq_delta(U2, V2, I2, 4, 4)}
+
+    def factored(e):
+        return {"W1": W1[e], "W2": W2[e], "A1": V1, "B1": U1, "A2": V2, "B2": U2}
+
+    for n in (1, 2):
+        a = mo.moe_forward(X, logits, k, tiled, N, comp_top_n=n)["Y"]
+        b = mo.moe_forward(X, logits, k, factored, N, comp_top_n=n)["Y"]
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
+    full = mo.moe_forward(X, logits, k, tiled, N)["Y"]
+    assert np.max(np.abs(full - mo.moe_forward(X, logits, k, tiled, N, comp_top_n=1)["Y"])) > 1e-3
