@@ -40,7 +40,17 @@
  *   MOE_FMT_DENSE16      codes: bf16 [M, K] row-major (bits = 16).
  *
  * Compensator factors per block: A bf16 [r, K_in], B bf16 [M_out, r], r = the
- * expert's rank (0 disables the term).
+ * expert's rank (0 disables the term). A block type may instead carry 2D-tiled
+ * factors shared by all experts (moe_layer_set_tileq below).
+ *
+ * Calls: moe_layer_create / _destroy; moe_layer_set_expert_weights;
+ * moe_layer_set_bits; the weight-page calls moe_layer_release_planes /
+ * _reload_planes / _page_state; moe_layer_set_tileq / _clear_tileq;
+ * moe_layer_set_comp_top_n; moe_layer_set_path; moe_layer_forward /
+ * _forward_host; test and timing hooks (moe_layer_get_routing,
+ * moe_layer_debug_unpack, moe_layer_sync_status, moe_layer_last_launch_count,
+ * moe_layer_set_profiling, moe_layer_kernel_times); moe_route_topk_noalloc;
+ * the host-only planner moe_plan_reduce / moe_plan_restore; moe_status_string.
  *
  * Conventions.
  *   - Every call returns a moe_status_t; nothing aborts or throws across the ABI.
@@ -50,7 +60,8 @@
  *     errors surface at moe_layer_sync_status or at the next call.
  *   - One layer is used from one stream at a time.
  *   - Arithmetic: fp16 tensor-core operands (X, the SwiGLU output and the
- *     compensator terms are rounded to fp16; dequantised weights too on the
+ *     compensator terms are rounded to fp16, the tiled compensators' inner
+ *     projections and cores too; dequantised weights too on the
  *     prefill path, while the decode path multiplies the exact integer codes
  *     and applies scale and zero per group in fp32), fp32 accumulation, bf16
  *     output. |X| and |z| must stay below 65504, and on the decode path of an
