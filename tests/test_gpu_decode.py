@@ -194,17 +194,19 @@ def test_forward_host_matches_device():
 
 # ---------------------------------------------------------------------------- full size
 
-def test_mixtral_decode_full_size_sampled_rows():
-    """Mixtral-8x7B decode layer (E=8, top-2, 4096 x 14336, INT3 g128, rank 32),
-    T=64 on the benchmark's launch configuration; a sample of rows checked
+@pytest.mark.parametrize("T", [1, 8, 32, 64])
+def test_mixtral_decode_full_size_sampled_rows(T):
+    """Mixtral-8x7B decode layer (E=8, top-2, 4096 x 14336, INT3 g128, rank 32)
+    at each token count of the workload, on the benchmark's launch
+    configuration (a layer sized for T tokens); a sample of rows checked
     against the oracle."""
     cfg = ms.make_config("mixtral_decode")
     blocks = make_blocks(cfg, DEV)
-    L = make_layer(cfg, blocks, max_tokens=64)
-    X, logits = ms.make_inputs(cfg, 64, DEV)
+    L = make_layer(cfg, blocks, max_tokens=T)
+    X, logits = ms.make_inputs(cfg, T, DEV)
     Y = L.forward(X, logits, 2)
     assert L.sync_status() == 0
-    rows = [0, 17, 63]
+    rows = sorted(set([0, T // 2, T - 1]))
     ref = oracle_forward(cfg, blocks, X, logits, 2, rows=rows)
     assert_parity(Y[rows], ref["Y"], "mixtral full")
     L.close()
