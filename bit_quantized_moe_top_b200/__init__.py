@@ -26,7 +26,7 @@ PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 
 # every symbol the header declares
 EXPORTS = ["moe_layer_create", "moe_layer_set_expert_weights", "moe_layer_set_bits", "moe_layer_set_comp_top_n",
-           "moe_layer_set_path",
+           "moe_layer_set_path", "moe_layer_set_wait_limit",
            "moe_layer_forward", "moe_layer_forward_host", "moe_layer_get_routing", "moe_layer_debug_unpack",
            "moe_layer_sync_status", "moe_layer_last_launch_count", "moe_layer_set_profiling",
            "moe_layer_kernel_times", "moe_route_topk_noalloc", "moe_plan_reduce", "moe_plan_restore",
@@ -67,6 +67,7 @@ def _lib() -> ctypes.CDLL:
         lib.moe_layer_set_expert_weights.argtypes = [P, I, I, P, P, P, P, P, I]
         lib.moe_layer_set_bits.argtypes = [P, I, I, I]
         lib.moe_layer_set_path.argtypes = [P, I]
+        lib.moe_layer_set_wait_limit.argtypes = [P, ctypes.c_ulonglong]
         lib.moe_layer_set_comp_top_n.argtypes = [P, I]
         lib.moe_layer_set_tileq.argtypes = [P, I, I, I, I, P, P, P, I]
         lib.moe_layer_clear_tileq.argtypes = [P, I]
@@ -152,6 +153,10 @@ def moe_layer_clear_tileq(layer: int, block: int) -> None:
 
 def moe_layer_set_path(layer: int, path: int) -> None:
     _check(_lib().moe_layer_set_path(layer, path), "moe_layer_set_path")
+
+
+def moe_layer_set_wait_limit(layer: int, limit_ns: int) -> None:
+    _check(_lib().moe_layer_set_wait_limit(layer, limit_ns), "moe_layer_set_wait_limit")
 
 
 def moe_layer_forward(layer: int, X, logits, top_k: int, Y, stream: Optional[int] = None) -> None:
@@ -323,6 +328,9 @@ class MoELayer:
 
     def set_path(self, path):
         moe_layer_set_path(self.handle, path)
+
+    def set_wait_limit(self, limit_ns):
+        moe_layer_set_wait_limit(self.handle, limit_ns)
 
     def forward(self, X, logits, top_k, Y=None, stream=None):
         import torch

@@ -192,19 +192,12 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
   return t;
 }
-// Bounded wait: gives up after ~limit_ns, sets ST_TIMEOUT and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* status,
-                                          unsigned long long limit_ns = 2000000000ull) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
-  for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      atomicOr(status, ST_TIMEOUT);
-      return false;
-    }
-  }
-}
+// Limit of the waits that drain a CTA's own copies and MMAs before it exits
+// (they always complete; the limit only guards against a broken invariant).
+constexpr unsigned long long kDrainLimitNs = 2000000000ull;
+// Default limit of the hand-off waits between a kernel's roles.
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+
 // Probe of a phase without a suspend hint (a completed phase returns at once).
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -215,13 +208,31 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Bounded wait: gives up once limit_ns have passed, sets ST_TIMEOUT and
+// returns false. Limits far above the suspend hint sleep in try_wait; shorter
+// ones poll, so that the limit is honoured.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* status,
+                                          unsigned long long limit_ns = kDefaultWaitNs) {
+  const bool sleep = limit_ns >= 2000000ull;
+  if (sleep ? mbar_try_wait(bar, parity) : mbar_test(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (;;) {
+    if (sleep ? mbar_try_wait(bar, parity) : mbar_test(bar, parity)) return true;
+    if (globaltimer_ns() - t0 >= limit_ns) {
+      atomicOr(status, ST_TIMEOUT);
+      return false;
+    }
+  }
+}
 // The bounded wait, out of line: only taken when the phase is still open.
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, unsigned* status) {
-  return mbar_wait(bar, parity, status);
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, unsigned* status,
+                                                   unsigned long long limit_ns) {
+  return mbar_wait(bar, parity, status, limit_ns);
 }
 // Bounded wait with an inlined fast path.
-__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, unsigned* status) {
-  return mbar_test(bar, parity) || mbar_wait_slow(bar, parity, status);
+__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, unsigned* status,
+                                               unsigned long long limit_ns = kDefaultWaitNs) {
+  return mbar_test(bar, parity) || mbar_wait_slow(bar, parity, status, limit_ns);
 }
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

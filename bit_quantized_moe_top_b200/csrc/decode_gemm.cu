@@ -145,7 +145,7 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
   const int n = c.nmain + c.next;
   // the whole warp runs the loop (warp-uniform values); one lane issues the copies
   for (int i0 = 0; i0 < n; i0 += kSub, ps.st.next(a.nstages)) {
-    if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait_fast(empty + 8 * ps.st.idx, ps.st.ph ^ 1u, a.status))) {
+    if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait_fast(empty + 8 * ps.st.idx, ps.st.ph ^ 1u, a.status, a.wait_ns))) {
       *abort_flag = 1;
       return;
     }
@@ -206,8 +206,8 @@ __device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int s
   const int sub_b = stage_b / kSub;
   const int n = c.nmain + c.next;
   for (int i0 = 0; i0 < n; i0 += kSub) {
-    const bool ok = !*abort_flag && mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status) &&
-                    mbar_wait_fast(afull + 8 * ps.ab.idx, ps.ab.ph, a.status);
+    const bool ok = !*abort_flag && mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status, a.wait_ns) &&
+                    mbar_wait_fast(afull + 8 * ps.ab.idx, ps.ab.ph, a.status, a.wait_ns);
     if (!__all_sync(0xffffffffu, ok)) {
       *abort_flag = 1;
       return;
@@ -220,7 +220,7 @@ __device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int s
       group_pos<FMT, GROUP>(c, i, first, last);
       if (first) {
         if (!__all_sync(0xffffffffu,
-                        !*abort_flag && mbar_wait_fast(accfree + 8 * ps.acc.idx, ps.acc.ph ^ 1u, a.status))) {
+                        !*abort_flag && mbar_wait_fast(accfree + 8 * ps.acc.idx, ps.acc.ph ^ 1u, a.status, a.wait_ns))) {
           *abort_flag = 1;
           return;
         }
@@ -266,8 +266,8 @@ __device__ void unpack(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, ui
   const int n = c.nmain + c.next;
   for (int i0 = 0; i0 < n; i0 += kSub) {
     // warp-uniform waits: every lane reaches the .sync.aligned TMEM stores
-    const bool ok = !*abort_flag && mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status) &&
-                    mbar_wait_fast(aempty + 8 * ps.ab.idx, ps.ab.ph ^ 1u, a.status);
+    const bool ok = !*abort_flag && mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status, a.wait_ns) &&
+                    mbar_wait_fast(aempty + 8 * ps.ab.idx, ps.ab.ph ^ 1u, a.status, a.wait_ns);
     if (!__all_sync(0xffffffffu, ok)) {
       *abort_flag = 1;
       return;
@@ -353,7 +353,7 @@ __device__ void epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
       const uint32_t sz = d.sz[(long long)(g0 + gi) * a.M + R];
       s = __half2float(__ushort_as_half((uint16_t)(sz & 0xFFFFu)));
     }
-    if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait_fast(accfull + 8 * ps.acc.idx, ps.acc.ph, a.status))) {
+    if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait_fast(accfull + 8 * ps.acc.idx, ps.acc.ph, a.status, a.wait_ns))) {
       *abort_flag = 1;
       return;
     }
@@ -561,13 +561,13 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
       } else {
         --p.idx;
       }
-      if (!mbar_wait_fast(b0 + 8 * (dk::kBarFull + p.idx), p.ph, a.status)) break;
+      if (!mbar_wait_fast(b0 + 8 * (dk::kBarFull + p.idx), p.ph, a.status, kDrainLimitNs)) break;
     }
   }
   if (warp == dk::kMmaWarp && (threadIdx.x & 31) == 0) {
     // every issued MMA must complete before TMEM is released
     mma_commit(done_bar);
-    mbar_wait(done_bar, 0, a.status);
+    mbar_wait(done_bar, 0, a.status, kDrainLimitNs);
   }
   tc_fence_before();
   __syncthreads();

@@ -72,6 +72,7 @@ struct DecodeArgs {
   int KS;
   long long rows;             // routed rows of the forward (host-side grid sizing)
   int nstages;                // shared-memory stages of the ring (set by the launcher)
+  unsigned long long wait_ns; // limit of the hand-off waits between roles
   unsigned* status;
 };
 
@@ -160,6 +161,7 @@ struct PrefillArgs {
   __half* zout;               // MODE_SWIGLU: output rows (fp16), leading dimension ldz
   long long ldz;
   float* out;                 // MODE_OUT: [prows][M] fp32
+  unsigned long long wait_ns; // limit of the hand-off waits between roles
   unsigned* status;
 };
 

@@ -92,6 +92,7 @@ struct moe_layer {
   long long sem_stride = 0;
   DevBuf idx, w, counts, offsets, poffsets, active, n_active, ticket, perm, inv_pos, pinv, pslot, ptok;
   int comp_top_n = 0;
+  unsigned long long wait_ns = kDefaultWaitNs;  // hand-off wait limit of the GEMM kernels
   // 2D-tiled shared compensators, per block type (0 = W1, 1 = W2)
   struct Tileq {
     bool on = false;
@@ -391,6 +392,7 @@ moe_status_t moe_layer_set_expert_weights(moe_layer_t* L, int e, int block, cons
   BlockStore& S = L->store[2 * e + block];
   free_block(S);
   d.loaded = 0;
+  g_alloc_count = 0;  // allocation-failure injection counts this call's allocations
   moe_status_t st = MOE_OK;
   DevBuf t1, t2, t3, t4, t5;
   const int RB = M / 128, KC = Kin / 64;
@@ -598,6 +600,12 @@ moe_status_t moe_layer_page_state(moe_layer_t* L, int e, int block, int* committ
   if (committed_bits) *committed_bits = d.bits;
   if (resident_planes) *resident_planes = d.fmt == FMT_BITPLANE ? ps.resident : (d.loaded ? d.bits : 0);
   if (host_planes) *host_planes = nh;
+  return MOE_OK;
+}
+
+moe_status_t moe_layer_set_wait_limit(moe_layer_t* L, unsigned long long limit_ns) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  L->wait_ns = limit_ns == 0 ? kDefaultWaitNs : limit_ns;
   return MOE_OK;
 }
 
@@ -966,6 +974,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
       pa.zout = static_cast<__half*>(L->zact.p);
       pa.ldz = L->Kpad_z;
       pa.out = static_cast<float*>(L->obuf.p);
+      pa.wait_ns = L->wait_ns;
       pa.status = ra.status;
       prof_mark(L, st, block == 0 ? "prefill_gemm_w1_swiglu" : "prefill_gemm_w2");
       ce = launch_prefill_gemm(pa, pairs, grid_y, st, &launches);
@@ -1003,6 +1012,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
       da.out_ks_stride = prows * K;
       da.KS = KS;
       da.rows = rows;
+      da.wait_ns = L->wait_ns;
       da.status = ra.status;
       prof_mark(L, st, block == 0 ? "decode_gemm_w1_swiglu" : "decode_gemm_w2");
       ce = launch_decode_gemm(da, ntok, maxbits[block], grid_y, st, &launches);
@@ -1014,8 +1024,9 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     tileq(1, corr2);
     // split the down projection's K while its grid is small (fixed-order sum in the combine)
     const int row_tiles = K / decode_rows_per_cta();
-    ks2 = std::max(1, 600 / std::max(1, row_tiles * grid_y));
-    ks2 = std::min(ks2, std::min(L->ks2_max, N / 256));
+    // (each split at least 256 columns wide, and at least one split: N = 128 gives one)
+    ks2 = std::min(600 / std::max(1, row_tiles * grid_y), std::min(L->ks2_max, N / 256));
+    ks2 = std::max(1, ks2);
     if (rows > 1024) ks2 = 1;
     decode_gemm(1, L->tmap_zd, L->tmap_cz, N, K, MODE_OUT, ks2);
   }

@@ -59,7 +59,8 @@ extern "C" moe_status_t moe_route_topk_noalloc(const float* logits, int T, int E
   if (!logits || !idx || !w || !counts || !offsets || T < 1 || E < 1 || E > kMaxExperts || top_k < 1 ||
       top_k > kMaxTopK || top_k > E || (flags & ~MOE_FLAG_NO_TOPK_RENORM))
     return MOE_ERR_INVALID_ARG;
-  if ((long long)route_num_blocks(T) * E > kNoAllocBlockEntries) return MOE_ERR_TOO_LARGE;
+  // token blocks of 16, counted in 64-bit so that no T overflows the check
+  if (((long long)T + 15) / 16 * E > kNoAllocBlockEntries) return MOE_ERR_TOO_LARGE;
   int* s = nullptr;
   if (scratch_for_current_device(&s) != cudaSuccess) return MOE_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);

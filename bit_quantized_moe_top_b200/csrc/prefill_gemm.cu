@@ -70,7 +70,7 @@ __device__ void producer(const PrefillArgs& a, const BlockDesc& d, const Ctx& c,
     // code blocks + scales of stage i (main K only)
     if (i < c.KC) {
       const int slot = i % kSC;
-      if (i >= kSC && !mbar_wait(c_empty + 8 * slot, ((i / kSC) & 1) ^ 1, a.status)) {
+      if (i >= kSC && !mbar_wait(c_empty + 8 * slot, ((i / kSC) & 1) ^ 1, a.status, a.wait_ns)) {
         *abort_flag = 1;
         break;
       }
@@ -93,7 +93,7 @@ __device__ void producer(const PrefillArgs& a, const BlockDesc& d, const Ctx& c,
     // activation tiles of stage i
     {
       const int slot = i % kSA;
-      if (i >= kSA && !mbar_wait(a_empty + 8 * slot, ((i / kSA) & 1) ^ 1, a.status)) {
+      if (i >= kSA && !mbar_wait(a_empty + 8 * slot, ((i / kSA) & 1) ^ 1, a.status, a.wait_ns)) {
         *abort_flag = 1;
         break;
       }
@@ -108,20 +108,20 @@ __device__ void producer(const PrefillArgs& a, const BlockDesc& d, const Ctx& c,
   }
   // drain: every issued copy must land before the CTA may exit
   for (int k = max(0, issued_a - kSA); k < issued_a; ++k)
-    if (!mbar_wait(a_full + 8 * (k % kSA), (k / kSA) & 1, a.status)) break;
+    if (!mbar_wait(a_full + 8 * (k % kSA), (k / kSA) & 1, a.status, kDrainLimitNs)) break;
   for (int k = max(0, issued_c - kSC); k < issued_c; ++k)
-    if (!mbar_wait(c_full + 8 * (k % kSC), (k / kSC) & 1, a.status)) break;
+    if (!mbar_wait(c_full + 8 * (k % kSC), (k / kSC) & 1, a.status, kDrainLimitNs)) break;
 }
 
 __device__ void mma_issuer(const Ctx& c, uint8_t* sm, uint32_t bars, uint32_t tmem, unsigned* status,
-                           volatile int* abort_flag) {
+                           unsigned long long wait_ns, volatile int* abort_flag) {
   const uint32_t a_full = bars, a_empty = bars + 8 * kSA;
   const uint32_t b_full = bars + 8 * 2 * kSA, b_empty = b_full + 8 * kSB;
   const uint32_t acc_full = bars + 8 * (2 * kSA + 2 * kSB + 2 * kSC);
   for (int i = 0; i < c.nk; ++i) {
     const int sa = i % kSA, sb = i % kSB;
-    if (*abort_flag || !mbar_wait(a_full + 8 * sa, (i / kSA) & 1, status) ||
-        !mbar_wait(b_full + 8 * sb, (i / kSB) & 1, status)) {
+    if (*abort_flag || !mbar_wait(a_full + 8 * sa, (i / kSA) & 1, status, wait_ns) ||
+        !mbar_wait(b_full + 8 * sb, (i / kSB) & 1, status, wait_ns)) {
       *abort_flag = 1;
       break;
     }
@@ -138,6 +138,9 @@ __device__ void mma_issuer(const Ctx& c, uint8_t* sm, uint32_t bars, uint32_t tm
     mma_commit(b_empty + 8 * sb);
   }
   mma_commit(acc_full);
+  // every issued MMA completes before the CTA frees its TMEM, also when the
+  // epilogue gave up and will not wait for the accumulators
+  mbar_wait(acc_full, 0, status, kDrainLimitNs);
 }
 
 template <int FMT, int BITS, int GROUP>
@@ -161,7 +164,7 @@ __device__ void dequant_and_epilogue(const PrefillArgs& a, const BlockDesc& d, c
   bool ok = true;
   for (int i = 0; i < c.nk && ok; ++i) {
     const int sb = i % kSB;
-    if (*abort_flag || !mbar_wait(b_empty + 8 * sb, ((i / kSB) & 1) ^ 1, a.status)) {
+    if (*abort_flag || !mbar_wait(b_empty + 8 * sb, ((i / kSB) & 1) ^ 1, a.status, a.wait_ns)) {
       ok = false;
       break;
     }
@@ -169,7 +172,7 @@ __device__ void dequant_and_epilogue(const PrefillArgs& a, const BlockDesc& d, c
     uint32_t v[32];
     if (i < c.KC) {
       const int cs_slot = i % kSC;
-      if (!mbar_wait(c_full + 8 * cs_slot, (i / kSC) & 1, a.status)) {
+      if (!mbar_wait(c_full + 8 * cs_slot, (i / kSC) & 1, a.status, a.wait_ns)) {
         ok = false;
         break;
       }
@@ -205,7 +208,7 @@ __device__ void dequant_and_epilogue(const PrefillArgs& a, const BlockDesc& d, c
   }
   const int rf0 = c.rt * kFr;
   // ---- epilogue
-  if (!mbar_wait(acc_full, 0, a.status)) {
+  if (!mbar_wait(acc_full, 0, a.status, a.wait_ns)) {
     *abort_flag = 1;
     return;
   }
@@ -252,7 +255,7 @@ __device__ void prefill_tile(const PrefillArgs& a, const BlockDesc& d, const pf:
   if (warp == 0) {
     if ((threadIdx.x & 31) == 0) pf::producer<FMT, BITS, GROUP>(a, d, c, sm, bars, ab);
   } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) pf::mma_issuer(c, sm, bars, tmem, a.status, ab);
+    if ((threadIdx.x & 31) == 0) pf::mma_issuer(c, sm, bars, tmem, a.status, a.wait_ns, ab);
   } else {
     pf::dequant_and_epilogue<FMT, BITS, GROUP>(a, d, c, sm, bars, tmem, ab);
   }

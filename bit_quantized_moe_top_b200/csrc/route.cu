@@ -7,6 +7,8 @@
 // k routed experts, of which the Top-n get compensation). Selection compares
 // the fp32 logits exactly, ties to the lower expert index; the weights are the
 // softmax over the selected logits (or the full softmax, by flag).
+#include <algorithm>
+
 #include "kernels.h"
 
 namespace moeq {
@@ -235,8 +237,9 @@ cudaError_t launch_route_topk(const RouteArgs& a, cudaStream_t st, int* launches
 
 cudaError_t launch_route_permute(const RouteArgs& a, cudaStream_t st, int* launches) {
   const int nb = (a.T + kRouteTokensPerCta - 1) / kRouteTokensPerCta;
-  int gs = 296 / nb;
-  gs = gs < 1 ? 1 : gs > a.K / 256 ? a.K / 256 : gs;
+  // K slices of the gather: enough CTAs to fill the GPU, each slice at least
+  // 256 columns wide, and always at least one (K = 128 gives one slice)
+  const int gs = std::max(1, std::min(296 / nb, a.K / 256));
   const cudaError_t err = launch_kernel(route_permute_kernel, dim3(nb, gs), dim3(kRouteThreads), 0, st, true, a);
   if (launches) ++*launches;
   return err;

@@ -46,7 +46,8 @@
  * Calls: moe_layer_create / _destroy; moe_layer_set_expert_weights;
  * moe_layer_set_bits; the weight-page calls moe_layer_release_planes /
  * _reload_planes / _page_state; moe_layer_set_tileq / _clear_tileq;
- * moe_layer_set_comp_top_n; moe_layer_set_path; moe_layer_forward /
+ * moe_layer_set_comp_top_n; moe_layer_set_path; moe_layer_set_wait_limit;
+ * moe_layer_forward /
  * _forward_host; test and timing hooks (moe_layer_get_routing,
  * moe_layer_debug_unpack, moe_layer_sync_status, moe_layer_last_launch_count,
  * moe_layer_set_profiling, moe_layer_kernel_times); moe_route_topk_noalloc;
@@ -119,7 +120,12 @@ typedef struct moe_layer moe_layer_t; /* opaque */
 #define MOE_PATH_DECODE 1  /* weight-streaming tcgen05 grouped GEMM, unpacked codes in TMEM */
 #define MOE_PATH_PREFILL 2 /* TMA + shared-memory dequant + tcgen05/TMEM grouped GEMM */
 
-/* Create a layer on the current CUDA device.
+/* Create a layer on the current CUDA device from per-expert descriptors: each
+ * expert's linear blocks carry their own bitwidth (MxMoE abstract: bitwidths
+ * chosen per linear block and per expert, mixed-precision) and each expert its
+ * own compensator rank (MiLo abstract: per-expert low-rank compensators of the
+ * quantisation residual, the rank adapted per expert; a rank of 0 leaves the
+ * expert uncompensated).
  * d_model and d_ff: multiples of 128. num_experts <= 256, max_top_k <= 8 and
  * <= num_experts, max_tokens >= 1. descs: [num_experts], copied.
  * Weights start unset (forward returns MOE_ERR_NOT_LOADED until every expert's
@@ -127,8 +133,11 @@ typedef struct moe_layer moe_layer_t; /* opaque */
 moe_status_t moe_layer_create(int num_experts, int d_model, int d_ff, int max_tokens, int max_top_k,
                               const moe_expert_desc_t* descs, unsigned flags, moe_layer_t** out);
 
-/* Load one block (0 = W1 gate||up [2*d_ff, d_model], 1 = W2 down [d_model, d_ff])
- * of one expert from the canonical layouts above. ptr_kind 0 = host pointers,
+/* Load one weight page of one expert (PagedWeight, "What carries the
+ * argument": the unit of weight storage and movement is one linear block of
+ * one expert, identified by layer, expert and block type): block 0 = W1
+ * gate||up [2*d_ff, d_model], 1 = W2 down [d_model, d_ff], from the canonical
+ * layouts above, together with the block's compensator factors (MiLo abstract). ptr_kind 0 = host pointers,
  * 1 = device pointers. The data are copied and re-laid out on the device (the
  * caller keeps ownership). scales is used by INT_ASYM only; zeros_or_lut holds
  * the zeros (INT_ASYM) or the 28-entry LUT (BITPLANE_LUT). A and B may be NULL
@@ -213,10 +222,28 @@ moe_status_t moe_layer_set_tileq(moe_layer_t* layer, int block, int rank, int ti
                                  const void* V, const void* cores, int ptr_kind);
 moe_status_t moe_layer_clear_tileq(moe_layer_t* layer, int block);
 
+/* Limit, in nanoseconds, of the bounded waits by which the roles of one GEMM
+ * kernel (copy engine, unpack, MMA, epilogue) hand work to each other; 0
+ * restores the default of 2 s. A wait that runs out sets the device status
+ * word (moe_layer_sync_status then returns MOE_ERR_TIMEOUT), and the CTA
+ * drains its own copies and tensor-core operations, frees its tensor memory
+ * and returns; the forward's output is then undefined, and the layer stays
+ * usable. A limit shorter than a hand-off takes (a few ns) makes every
+ * forward give up: that is how the timeout path is tested without any fault.
+ * Drains are bounded separately (2 s). Takes effect at the next forward. */
+moe_status_t moe_layer_set_wait_limit(moe_layer_t* layer, unsigned long long limit_ns);
+
 /* Choose the kernel path (MOE_PATH_*). */
 moe_status_t moe_layer_set_path(moe_layer_t* layer, int path);
 
-/* Forward pass. X: bf16 [T, d_model] device; router_logits: fp32 [T, E] device;
+/* Forward pass of the quantised MoE expert layer, the computation stated at
+ * the top of this header: top-k routing and per-expert bucketing
+ * (Bandwidth-Efficient Adaptive Mixture-of-Experts via Low-Rank Compensation,
+ * abstract), each routed token through its expert's dequantised SwiGLU FFN
+ * plus the low-rank compensator of both linear blocks (MiLo abstract; the
+ * fused mixed-precision expert kernel of PagedWeight, "What carries the
+ * argument"), outputs combined by router weight.
+ * X: bf16 [T, d_model] device; router_logits: fp32 [T, E] device;
  * Y: bf16 [T, d_model] device, caller-allocated. 1 <= T <= max_tokens,
  * 1 <= top_k <= max_top_k. cuda_stream: a cudaStream_t (NULL = legacy stream).
  * Asynchronous. */
@@ -275,7 +302,11 @@ int moe_layer_kernel_times(moe_layer_t* layer, const char** names, float* ms, in
  * device current); make that first call before any stream capture. Every call
  * shares the one array and clears the words that must start at zero, so calls
  * whose kernels overlap on the GPU (concurrent streams or threads) race and
- * must be serialised by the caller. Calls no allocating routine. */
+ * must be serialised by the caller. Calls no allocating routine. The routing
+ * kernel's own device-side check (an out-of-range selection, which only a NaN
+ * logit row can cause) writes a status word inside the shared array that no
+ * call reads back: this call does not report device-side checks, only launch
+ * errors (MOE_ERR_CUDA) and argument errors. */
 moe_status_t moe_route_topk_noalloc(const float* router_logits, int T, int E, int top_k, unsigned flags, int* idx,
                                     float* w, int* counts, int* offsets, void* cuda_stream);
 
