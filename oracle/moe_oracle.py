@@ -212,53 +212,82 @@ def expert_ffn(x: np.ndarray, W1: np.ndarray, W2: np.ndarray, N: int,
     return o
 
 
-def moe_forward(X: np.ndarray, logits: np.ndarray, top_k: int,
-                expert: Callable[[int], Dict], N: int, renorm: bool = True,
+def routed_jobs(X: np.ndarray, logits: np.ndarray, top_k: int, E: int, renorm: bool = True,
                 rows: Optional[Sequence[int]] = None, comp_top_n: int = 0) -> Dict:
-    """The layer's forward pass.
-
-    ``expert(e)`` returns a dict with fp64 arrays W1 [2N, K], W2 [K, N] and
-    optional A1, B1, A2, B2, or dense compensators D1 [2N, K], D2 [K, N] (it
-    is called only for experts that receive tokens). ``rows`` restricts the output to those tokens (routing and
-    bucketing are still computed for all tokens). ``comp_top_n`` > 0 applies
-    the compensators only to the first n routing slots of each token and runs
-    the other slots' experts on their quantised weights alone (Bandwidth-
-    Efficient Adaptive Mixture-of-Experts via Low-Rank Compensation, abstract:
-    compensation for the Top-n (n < k) experts of each token). Returns a dict
-    with Y fp64 ([T, K] or [len(rows), K]) and the routing arrays.
-    """
-    X64 = np.asarray(X, np.float64)
-    T, K = X64.shape
-    E = np.asarray(logits).shape[1]
+    """Steps 2-3 and the work list of step 4: routing, bucketing, and per
+    expert the bucket rows p whose token is wanted, split into those that get
+    the compensator and those that do not (``comp_top_n`` > 0 compensates only
+    the first n routing slots of each token: Bandwidth-Efficient Adaptive
+    Mixture-of-Experts via Low-Rank Compensation, abstract, Top-n (n < k)
+    compensation)."""
+    T = np.asarray(X).shape[0]
     idx, w = route(logits, top_k, renorm)
     counts, offsets, perm, inv = bucket(idx, E)
     want = np.arange(T) if rows is None else np.asarray(rows, np.int64)
     wanted = set(int(t) for t in want)
     slot = {int(inv[t, j]): j for t in range(T) for j in range(top_k)}
-    O = {}
+    jobs = []
     for e in range(E):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         ps = [p for p in range(lo, hi) if int(perm[p]) in wanted]
         if not ps:
             continue
-        ex = expert(e)
         comp = [p for p in ps if comp_top_n <= 0 or slot[p] < comp_top_n]
         plain = [p for p in ps if not (comp_top_n <= 0 or slot[p] < comp_top_n)]
-        if comp:
-            o = expert_ffn(X64[perm[comp]], ex["W1"], ex["W2"], N, ex.get("A1"), ex.get("B1"), ex.get("A2"),
-                           ex.get("B2"), ex.get("D1"), ex.get("D2"))
-            for i, p in enumerate(comp):
-                O[p] = o[i]
-        if plain:
-            o = expert_ffn(X64[perm[plain]], ex["W1"], ex["W2"], N)
-            for i, p in enumerate(plain):
-                O[p] = o[i]
+        jobs.append((e, comp, plain))
+    return {"idx": idx, "w": w, "counts": counts, "offsets": offsets, "perm_token": perm, "inv_pos": inv,
+            "want": want, "jobs": jobs}
+
+
+def expert_job(X: np.ndarray, perm: np.ndarray, ex: Dict, N: int, comp: Sequence[int],
+               plain: Sequence[int]) -> Dict[int, np.ndarray]:
+    """Step 4 for one expert: the outputs o of its bucket rows p (rows in
+    ``comp`` with the compensators, rows in ``plain`` without)."""
+    X64 = np.asarray(X, np.float64)
+    O = {}
+    if comp:
+        o = expert_ffn(X64[perm[list(comp)]], ex["W1"], ex["W2"], N, ex.get("A1"), ex.get("B1"), ex.get("A2"),
+                       ex.get("B2"), ex.get("D1"), ex.get("D2"))
+        for i, p in enumerate(comp):
+            O[p] = o[i]
+    if plain:
+        o = expert_ffn(X64[perm[list(plain)]], ex["W1"], ex["W2"], N)
+        for i, p in enumerate(plain):
+            O[p] = o[i]
+    return O
+
+
+def combine(want: Sequence[int], w: np.ndarray, inv: np.ndarray, O: Dict[int, np.ndarray], K: int) -> np.ndarray:
+    """Step 5: y_t = sum_j w[t, j] * o_(t, j), slots in order."""
     Y = np.zeros((len(want), K), np.float64)
     for i, t in enumerate(want):
-        for j in range(top_k):
+        for j in range(w.shape[1]):
             Y[i] += w[t, j] * O[int(inv[t, j])]
-    return {"Y": Y, "idx": idx, "w": w, "counts": counts, "offsets": offsets,
-            "perm_token": perm, "inv_pos": inv}
+    return Y
+
+
+def moe_forward(X: np.ndarray, logits: np.ndarray, top_k: int,
+                expert: Callable[[int], Dict], N: int, renorm: bool = True,
+                rows: Optional[Sequence[int]] = None, comp_top_n: int = 0) -> Dict:
+    """The layer's forward pass: routed_jobs, then expert_job for every expert
+    that holds a wanted row, then combine.
+
+    ``expert(e)`` returns a dict with fp64 arrays W1 [2N, K], W2 [K, N] and
+    optional A1, B1, A2, B2, or dense compensators D1 [2N, K], D2 [K, N] (it
+    is called only for experts that receive wanted rows). ``rows`` restricts
+    the output to those tokens (routing and bucketing are still computed for
+    all tokens). Returns a dict with Y fp64 ([T, K] or [len(rows), K]) and the
+    routing arrays.
+    """
+    X64 = np.asarray(X, np.float64)
+    E = np.asarray(logits).shape[1]
+    r = routed_jobs(X64, logits, top_k, E, renorm, rows, comp_top_n)
+    O = {}
+    for e, comp, plain in r["jobs"]:
+        O.update(expert_job(X64, r["perm_token"], expert(e), N, comp, plain))
+    Y = combine(r["want"], r["w"], r["inv_pos"], O, X64.shape[1])
+    return {"Y": Y, "idx": r["idx"], "w": r["w"], "counts": r["counts"], "offsets": r["offsets"],
+            "perm_token": r["perm_token"], "inv_pos": r["inv_pos"]}
 
 
 # ----------------------------------------------------------------------------

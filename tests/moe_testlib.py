@@ -102,6 +102,54 @@ def oracle_forward(cfg, blocks, X, logits, top_k, rows=None, renorm=True, bits_o
                            comp_top_n=comp_top_n)
 
 
+def _block_job_dict(blk: ms.BlockWeights, bits=None) -> dict:
+    d = {"fmt": blk.fmt, "bits": bits or blk.bits, "group": blk.group, "K_in": blk.K_in,
+         "codes": blk.codes.cpu().numpy() if blk.fmt != ms.FMT_DENSE16 else blk.codes.float().cpu().numpy(),
+         "scales": None if blk.scales is None else blk.scales.cpu().numpy(),
+         "zeros_or_lut": None if blk.zeros_or_lut is None else blk.zeros_or_lut.cpu().numpy()}
+    out = {"blk": d, "A": None, "B": None}
+    if blk.rank > 0:
+        out["A"] = blk.A.float().cpu().numpy().astype(np.float64)
+        out["B"] = blk.B.float().cpu().numpy().astype(np.float64)
+    return out
+
+
+def oracle_forward_pool(cfg, blocks, X, logits, top_k, rows=None, renorm=True, bits_override=None, comp_top_n=0):
+    """``oracle_forward`` with the experts dequantised and run in a pool of
+    spawned processes (for full-size layers)."""
+    import oracle_pool
+    bo = bits_override or {}
+
+    def block_of(e):
+        return {b: _block_job_dict(blocks[(e, b)], bo.get((e, b))) for b in (0, 1)}
+
+    return oracle_pool.forward(X.float().cpu().numpy().astype(np.float64), logits.cpu().numpy(), top_k, block_of,
+                               cfg.N, renorm=renorm, rows=rows, comp_top_n=comp_top_n)
+
+
+def prefill_sample_rows(logits, top_k, tile=128, extra=8, seed=0):
+    """Tokens whose outputs a full-size prefill test compares: for every
+    expert bucket (the oracle's routing and bucketing), its first and last
+    rows, the rows on both sides of each 128-row token-tile boundary within
+    the first pair of tiles (positions 127, 128, 255, 256), and the first row
+    of its last, partially filled pair of tiles; plus a few random tokens."""
+    L = logits.cpu().numpy()
+    idx, _ = orc.route(L, top_k)
+    E = L.shape[1]
+    counts, offsets, perm, _ = orc.bucket(idx, E)
+    rows = set()
+    for e in range(E):
+        n, lo = int(counts[e]), int(offsets[e])
+        if n == 0:
+            continue
+        for pos in (0, n - 1, tile - 1, tile, 2 * tile - 1, 2 * tile, (n - 1) // (2 * tile) * (2 * tile)):
+            if 0 <= pos < n:
+                rows.add(int(perm[lo + pos]))
+    rng = np.random.default_rng(seed)
+    rows.update(int(t) for t in rng.integers(0, L.shape[0], size=extra))
+    return sorted(rows)
+
+
 def row_errors(Y: torch.Tensor, Yref: np.ndarray):
     Yg = Y.float().cpu().numpy().astype(np.float64)
     num = np.linalg.norm(Yg - Yref, axis=1)

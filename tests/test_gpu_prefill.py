@@ -6,7 +6,8 @@ import torch
 
 import moe_synth as ms
 import oracle as orc
-from moe_testlib import assert_parity, make_blocks, make_layer, oracle_forward
+from moe_testlib import (assert_parity, make_blocks, make_layer, oracle_forward, oracle_forward_pool,
+                         prefill_sample_rows)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -127,54 +128,73 @@ def test_set_bits_errors():
 
 # ---------------------------------------------------------------------------- full-size configurations
 
-def test_dsv2lite_decode_full_size_sampled_rows():
+def test_dsv2lite_decode_full_size_all_rows():
     """64 experts, top-6, 2048 x 1408, per-expert bits {2,3,4} g64, ranks
-    {0,16,32,64}, Zipf(1.1)-skewed routing, T = 256."""
+    {0,16,32,64}, Zipf(1.1)-skewed routing, T = 256; every row."""
     cfg = ms.make_config("dsv2lite_decode")
     L, blocks, X, logits, Y = _run(cfg, 256, 0)
-    rows = [0, 101, 255]
-    ref = oracle_forward(cfg, blocks, X, logits, cfg.top_k, rows=rows)
-    assert_parity(Y[rows], ref["Y"], "dsv2lite")
+    ref = oracle_forward_pool(cfg, blocks, X, logits, cfg.top_k)
+    assert_parity(Y, ref["Y"], "dsv2lite")
     L.close()
 
 
 def test_mixtral_prefill_full_size_sampled_rows():
-    """Mixtral-8x7B prefill layer: INT4 g128, rank 16, T = 8192 (tcgen05 path)."""
+    """Mixtral-8x7B prefill layer: INT4 g128, rank 16, T = 8192 (tcgen05
+    path). Rows: the first and last of every expert bucket, both sides of the
+    128-token tile boundaries, the last partial pair of tiles, random rows."""
     cfg = ms.make_config("mixtral_prefill")
     L, blocks, X, logits, Y = _run(cfg, 8192, 0)
-    rows = [0, 4097, 8191]
-    ref = oracle_forward(cfg, blocks, X, logits, cfg.top_k, rows=rows)
+    rows = prefill_sample_rows(logits, cfg.top_k)
+    assert len(rows) >= 32
+    ref = oracle_forward_pool(cfg, blocks, X, logits, cfg.top_k, rows=rows)
     assert_parity(Y[rows], ref["Y"], "mixtral prefill")
     L.close()
 
 
-def test_dsv3_bitplane_decode_full_size_sampled_rows():
-    """256 bit-plane experts, top-8, 7168 x 2048, bits {2,3,4} per block,
-    rank 32, Zipf(1.2) routing, T = 128; then one set_bits re-draw."""
-    cfg = ms.make_config("dsv3_bitplane")
-    T = 128
-    X, logits = ms.make_inputs(cfg, T, DEV)
-    idx, _ = orc.route(logits.cpu().numpy(), cfg.top_k)
-    rows = [0, 77]
-    need = sorted(set(int(e) for e in idx[rows].reshape(-1)))
-    blocks = make_blocks(cfg, DEV)
-    L = make_layer(cfg, blocks, max_tokens=T)
-    Y = L.forward(X, logits, cfg.top_k)
-    assert L.sync_status() == 0
-    ref = oracle_forward(cfg, {k: v for k, v in blocks.items() if k[0] in need}, X, logits, cfg.top_k, rows=rows)
-    assert_parity(Y[rows], ref["Y"], "dsv3 decode")
-    rng = np.random.default_rng(11)
+def _redraw_bits(L, cfg, seed=11):
+    rng = np.random.default_rng(seed)
     newbits = {}
-    for e in need:
+    for e in range(cfg.E):
         for b in (0, 1):
             nb = int(rng.choice([2, 3, 4]))
             L.set_bits(e, b, nb)
             newbits[(e, b)] = nb
+    return newbits
+
+
+def test_dsv3_bitplane_decode_full_size_all_rows():
+    """256 bit-plane experts, top-8, 7168 x 2048, bits {2,3,4} per block,
+    rank 32, Zipf(1.2) routing, T = 128, every row; then one set_bits
+    re-draw of every block."""
+    cfg = ms.make_config("dsv3_bitplane")
+    T = 128
+    L, blocks, X, logits, Y = _run(cfg, T, 0)
+    ref = oracle_forward_pool(cfg, blocks, X, logits, cfg.top_k)
+    assert_parity(Y, ref["Y"], "dsv3 decode")
+    newbits = _redraw_bits(L, cfg)
     Y2 = L.forward(X, logits, cfg.top_k)
     assert L.sync_status() == 0
-    ref2 = oracle_forward(cfg, {k: v for k, v in blocks.items() if k[0] in need}, X, logits, cfg.top_k, rows=rows,
-                          bits_override=newbits)
-    assert_parity(Y2[rows], ref2["Y"], "dsv3 decode after set_bits")
+    ref2 = oracle_forward_pool(cfg, blocks, X, logits, cfg.top_k, bits_override=newbits)
+    assert_parity(Y2, ref2["Y"], "dsv3 decode after set_bits")
+    L.close()
+
+
+def test_dsv3_bitplane_prefill_full_size_sampled_rows():
+    """The DeepSeek-V3-shaped bit-plane layer at T = 4096 on the prefill path,
+    rows by the prefill sampling rule, before and after one set_bits re-draw
+    of every block."""
+    cfg = ms.make_config("dsv3_bitplane")
+    T = 4096
+    L, blocks, X, logits, Y = _run(cfg, T, 0)
+    rows = prefill_sample_rows(logits, cfg.top_k, extra=16)
+    assert len(rows) >= 32
+    ref = oracle_forward_pool(cfg, blocks, X, logits, cfg.top_k, rows=rows)
+    assert_parity(Y[rows], ref["Y"], "dsv3 prefill")
+    newbits = _redraw_bits(L, cfg)
+    Y2 = L.forward(X, logits, cfg.top_k)
+    assert L.sync_status() == 0
+    ref2 = oracle_forward_pool(cfg, blocks, X, logits, cfg.top_k, rows=rows, bits_override=newbits)
+    assert_parity(Y2[rows], ref2["Y"], "dsv3 prefill after set_bits")
     L.close()
 
 
