@@ -48,7 +48,15 @@ def parse():
                    help="bit-plane configs: before timing, re-draw every block's bitwidth from {2,3,4} with this "
                         "seed and commit it with moe_layer_set_bits")
     p.add_argument("--tile-k", type=int, default=1024)
+    p.add_argument("--no-extras", action="store_true",
+                   help="skip the other workloads that the default single-GPU run also times")
+    p.add_argument("--extra-steps", type=int, default=20)
     return p.parse_args()
+
+
+# the other workloads a default single-GPU run times after the headline one:
+# (config, tokens), each on its own layer, reported under "extra_workloads"
+EXTRAS = [("mixtral_prefill", 8192), ("dsv3_bitplane", 4096), ("dsv3_bitplane", 128), ("dsv2lite_decode", 256)]
 
 
 # ---------------------------------------------------------------------------
@@ -221,8 +229,18 @@ def cpu_oracle_rate(cfg, blocks_cpu, X, logits, top_k, budget_s):
         if time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
-    threads = torch.get_num_threads()
-    return done / dt, done, dt, threads
+    return done / dt, done, dt, host_threads()
+
+
+def host_threads():
+    """Cores of the host and the threads the oracle's numpy BLAS may use."""
+    blas = None
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"), default=None)
+    except Exception:
+        pass
+    return {"host_cores": os.cpu_count(), "blas_threads": blas}
 
 
 KERNEL_SOURCES = {
@@ -286,72 +304,50 @@ def build_layer(bq, cfg, blocks, max_tokens):
 
 # ---------------------------------------------------------------------------
 
-def main():
-    args = parse()
-    import torch
-    import torch.distributed as dist
-    import moe_synth as ms
+def config_dict(cfg, T, workload, world, tq=None):
+    return {"workload": workload, "T": T, "E": cfg.E, "top_k": cfg.top_k, "d_model": cfg.K, "d_ff": cfg.N,
+            "bits": sorted(set(b for sp in cfg.experts for b in sp.bits)),
+            "format": "bit-plane+LUT" if cfg.experts[0].fmt == 1 else "int asym",
+            "group": cfg.experts[0].group, "ranks": sorted(set(sp.rank for sp in cfg.experts)),
+            "parallelism": f"replicas x{world}",
+            "l2": "flushed between steps (256 MiB write, untimed)",
+            **({"compensator": {"kind": "2D-tiled shared factors", "rank": tq[0], "tile_m": tq[1],
+                                "tile_k": tq[2]}} if tq else {})}
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    T = args.tokens
-    cfg = ms.make_config(args.config)
-    tq = (args.tileq, args.tile_m, args.tile_k) if args.tileq else None
+
+def make_cfg(ms, name, tq=None):
+    cfg = ms.make_config(name)
     if tq:
         # the tiled shared compensators replace every expert's own pair
         cfg.experts = [ms.ExpertSpec(sp.fmt, sp.bits, sp.group, 0) for sp in cfg.experts]
-    workload = f"{WORKLOADS[args.config]}_T{T}" + (f"_tileq_r{tq[0]}_{tq[1]}x{tq[2]}" if tq else "")
-    if args.redraw_bits >= 0:
-        if any(sp.fmt != ms.FMT_BITPLANE_LUT for sp in cfg.experts):
-            raise SystemExit("--redraw-bits needs a bit-plane configuration")
-        workload += f"_bits_redrawn_{args.redraw_bits}"
+    return cfg
 
-    if args.impl == "reference":
-        if rank != 0:
-            return
-        blocks = {}
-        for e in range(cfg.E):
-            for b in (0, 1):
-                blocks[(e, b)] = ms.make_block(cfg, e, b, device="cpu")
-        X, logits = ms.make_inputs(cfg, T, "cpu")
-        budget = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup))
-        rates = []
-        for i in range(args.warmup + args.steps):
-            r, n, dt, thr = cpu_oracle_rate(cfg, blocks, X, logits, cfg.top_k, budget)
-            if i >= args.warmup:
-                rates.append((r, n, dt, thr))
-        val = statistics.median([r[0] for r in rates])
-        ms_step = 1000.0 * T / val
-        line = {"impl": "reference", "metric": "MoE-layer tokens/s", "value": val, "unit": "tokens/s",
-                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "config": {"workload": f"{WORKLOADS[args.config]}_T{T}", "T": T},
-                "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": rates[0][3], "kind": "oracle",
-                                 "sample": f"first {rates[0][1]} token(s) of the T={T} batch per step, one token "
-                                           f"at a time (its experts dequantised in fp64)"},
-                "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-        print(json.dumps(line), flush=True)
-        return
 
-    from bit_quantized_moe_top_b200 import build
-    build.build()
-    import bit_quantized_moe_top_b200 as bq
+def workload_name(name, T, tq=None, redraw=-1):
+    w = f"{WORKLOADS[name]}_T{T}" + (f"_tileq_r{tq[0]}_{tq[1]}x{tq[2]}" if tq else "")
+    if redraw >= 0:
+        w += f"_bits_redrawn_{redraw}"
+    return w
 
-    if world > 1:
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
-    torch.cuda.set_device(local)
-    dev = f"cuda:{local}"
 
+def measure(bq, ms, name, T, dev, steps, warmup, rank=0, world=1, tq=None, redraw=-1, e2e=True):
+    """Builds the layer of one workload on ``dev`` and times ``steps`` forward
+    passes with CUDA events (L2 flushed between them, untimed). Returns the
+    figures of the bench line (without cpu_baseline)."""
+    import torch
+    cfg = make_cfg(ms, name, tq)
+    workload = workload_name(name, T, tq, redraw)
+    if redraw >= 0 and any(sp.fmt != ms.FMT_BITPLANE_LUT for sp in cfg.experts):
+        raise SystemExit("--redraw-bits needs a bit-plane configuration")
     blocks = {}
     for e in range(cfg.E):
         for b in (0, 1):
             blocks[(e, b)] = ms.make_block(cfg, e, b, device=dev)
     L = build_layer(bq, cfg, blocks, max_tokens=T)
-    if args.redraw_bits >= 0:
+    if redraw >= 0:
         # one set_bits re-draw of every (expert, block): the kernels then read the new number of planes
         import numpy as np
-        rng = np.random.default_rng(np.random.SeedSequence([cfg.cid, 3000, args.redraw_bits]))
+        rng = np.random.default_rng(np.random.SeedSequence([cfg.cid, 3000, redraw]))
         new = rng.integers(2, 5, size=(cfg.E, 2))
         for e in range(cfg.E):
             for b in (0, 1):
@@ -370,37 +366,40 @@ def main():
     def step():
         L.forward(X, logits, cfg.top_k, Y)
 
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         step()
     torch.cuda.synchronize()
-    assert L.sync_status() == 0
+    st = L.sync_status()
+    assert st == 0, f"device status {st} ({bq.moe_status_string(st)})"
     routing = L.routing(T, cfg.top_k)
     counts = routing["counts"].cpu().tolist()
     launches_per_step = L.last_launch_count()
 
     # timed region: per-step events, L2 flushed (untimed) between steps
     L.set_profiling(True)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     kt = {}
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
-        for i in range(args.steps):
+    with ClockSampler(int(str(dev).split(":")[-1])) as clocks:
+        for i in range(steps):
             flush.fill_(i & 0xFF)
             ev[i][0].record(stream)
             step()
             ev[i][1].record(stream)
-            if i % 16 == 0 or i == args.steps - 1:
-                for name, t in L.kernel_times():
-                    kt.setdefault(name, []).append(t)
+            if i % 16 == 0 or i == steps - 1:
+                for kn, t in L.kernel_times():
+                    kt.setdefault(kn, []).append(t)
         torch.cuda.synchronize()
     L.set_profiling(False)
+    assert L.sync_status() == 0
     step_ms = [a.elapsed_time(b) for a, b in ev]
     pct = {q: statistics.quantiles(step_ms, n=10)[i] if len(step_ms) >= 2 else step_ms[0]
            for q, i in (("p10", 0), ("p50", 4), ("p90", 8))}
     total_ms = max_over_ranks(sum(step_ms), world, dev)
-    ms_per_step = total_ms / args.steps
+    ms_per_step = total_ms / steps
     value = weak_scaling_value(world, T, ms_per_step)
 
     # dominant kernel: the gate/up GEMM (2/3 of the weight bytes and flops)
@@ -416,13 +415,15 @@ def main():
         layer_b += tb
         layer_f += tf
     if prefill:
+        # a kernel of a few ms timed inside a step, not a seconds-long loop:
+        # the burst peak is its denominator
         f1 = gemm1_flops(cfg, counts)
         achieved = f1 / (k1 * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": tc_sustained,
-                    "unit": "TFLOP/s", "frac": achieved / tc_sustained,
+        roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": tc_peak,
+                    "unit": "TFLOP/s", "frac": achieved / tc_peak,
                     "traffic": stored_traffic(kname, workload),
-                    "peak_source": f"{peak_src} bf16 sustained (fp16 has the same dense rate)",
-                    "frac_of_burst_peak": achieved / tc_peak, "algorithmic_flops_per_launch": f1,
+                    "peak_source": f"{peak_src} bf16 burst (fp16 has the same dense rate)",
+                    "frac_of_sustained_peak": achieved / tc_sustained, "algorithmic_flops_per_launch": f1,
                     "launch_ms": k1}
     else:
         b1 = gemm1_bytes(cfg, counts, tq)
@@ -431,64 +432,140 @@ def main():
                     "frac": achieved / hbm_peak,
                     "traffic": stored_traffic(kname, workload), "peak_source": peak_src,
                     "algorithmic_bytes_per_launch": b1, "launch_ms": k1}
+    out = {"value": value, "ms_per_step": ms_per_step, "ms_per_step_percentiles": pct,
+           "config": config_dict(cfg, T, workload, world, tq),
+           "layer_hbm_gbs": layer_b / (ms_per_step * 1e-3) / 1e9,
+           "layer_hbm_frac": layer_b / (ms_per_step * 1e-3) / 1e9 / hbm_peak,
+           "layer_tflops": layer_f / (ms_per_step * 1e-3) / 1e12,
+           "layer_bytes_per_step": layer_b, "layer_flops_per_step": layer_f,
+           "roofline": roofline, "kernels_ms": kernel_means,
+           "gpu_launches": launches_per_step * steps, "clocks": clocks.summary(),
+           "_cfg": cfg, "_blocks": blocks, "_X": X, "_logits": logits}
 
-    # end to end: host buffers through moe_layer_forward_host (copies inside the timed region)
-    Xh = X.cpu().pin_memory()
-    Lh = logits.cpu().pin_memory()
-    Yh = torch.empty_like(Xh).pin_memory()
-    for _ in range(3):
-        L.forward_host(Xh, Lh, cfg.top_k, Yh)
-    e2e_steps = max(10, args.steps // 4)
-    torch.cuda.synchronize()
-    t0 = time.perf_counter()
-    for _ in range(e2e_steps):
-        L.forward_host(Xh, Lh, cfg.top_k, Yh)
-    e2e_s = (time.perf_counter() - t0) / e2e_steps
-    e2e_val = world * T / e2e_s
+    if e2e:
+        # end to end: host buffers through moe_layer_forward_host (copies inside the timed region)
+        Xh = X.cpu().pin_memory()
+        Lh = logits.cpu().pin_memory()
+        Yh = torch.empty_like(Xh).pin_memory()
+        for _ in range(3):
+            L.forward_host(Xh, Lh, cfg.top_k, Yh)
+        e2e_steps = max(10, steps // 4)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(e2e_steps):
+            L.forward_host(Xh, Lh, cfg.top_k, Yh)
+        e2e_s = (time.perf_counter() - t0) / e2e_steps
+        out["e2e"] = {"value": world * T / e2e_s, "unit": "tokens/s",
+                      "h2d_bytes_per_step": T * cfg.K * 2 + T * cfg.E * 4, "d2h_bytes_per_step": T * cfg.K * 2}
+    L.close()
+    del flush
+    return out
 
+
+def public(d):
+    return {k: v for k, v in d.items() if not k.startswith("_")}
+
+
+def reference_arm(args, ms):
+    """The fp64 CPU oracle timed on the host cores: each step is the oracle on
+    a bounded sample of the batch (its first tokens, one at a time)."""
+    cfg = make_cfg(ms, args.config)
+    T = args.tokens
+    blocks = {}
+    for e in range(cfg.E):
+        for b in (0, 1):
+            blocks[(e, b)] = ms.make_block(cfg, e, b, device="cpu")
+    X, logits = ms.make_inputs(cfg, T, "cpu")
+    budget = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+    rates = []
+    for i in range(args.warmup + args.steps):
+        r, n, dt, thr = cpu_oracle_rate(cfg, blocks, X, logits, cfg.top_k, budget)
+        if i >= args.warmup:
+            rates.append((r, n, dt, thr))
+    val = statistics.median([r[0] for r in rates])
+    thr = rates[0][3]
+    cores = thr["blas_threads"] or thr["host_cores"]
+    return {"impl": "reference", "metric": "MoE-layer tokens/s", "value": val, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * statistics.mean([r[2] for r in rates]),
+            "ms_per_step_note": "measured: one step = the oracle on the bounded sample below",
+            "ms_per_step_extrapolated_full_batch": 1000.0 * T / val,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(cfg, T, workload_name(args.config, T), args.gpus),
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "host_cores": thr["host_cores"],
+                             "blas_threads": thr["blas_threads"], "kind": "oracle",
+                             "sample": f"first {rates[0][1]} token(s) of the T={T} batch per step, one token "
+                                       f"at a time (its experts dequantised in fp64)"},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    import torch
+    import torch.distributed as dist
+    import moe_synth as ms
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    T = args.tokens
+    tq = (args.tileq, args.tile_m, args.tile_k) if args.tileq else None
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(reference_arm(args, ms)), flush=True)
+        return
+
+    from bit_quantized_moe_top_b200 import build
+    build.build()
+    import bit_quantized_moe_top_b200 as bq
+
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+
+    head = measure(bq, ms, args.config, T, dev, args.steps, args.warmup, rank, world, tq, args.redraw_bits)
     line = None
     if rank == 0:
         cpu = None
         if not args.no_cpu_baseline and world == 1 and not tq:
+            cfg, blocks = head["_cfg"], head["_blocks"]
             cpu_blocks = {k: ms.BlockWeights(**{**v.__dict__, "codes": v.codes.cpu(),
                                               "scales": None if v.scales is None else v.scales.cpu(),
                                               "zeros_or_lut": None if v.zeros_or_lut is None else v.zeros_or_lut.cpu(),
                                               "A": None if v.A is None else v.A.cpu(),
                                               "B": None if v.B is None else v.B.cpu()})
                           for k, v in blocks.items()}
-            r, n, dt, thr = cpu_oracle_rate(cfg, cpu_blocks, X.cpu(), logits.cpu(), cfg.top_k, args.cpu_seconds)
-            cpu = {"value": r, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+            r, n, dt, thr = cpu_oracle_rate(cfg, cpu_blocks, head["_X"].cpu(), head["_logits"].cpu(), cfg.top_k,
+                                            args.cpu_seconds)
+            cpu = {"value": r, "unit": "tokens/s", "cores": thr["blas_threads"] or thr["host_cores"],
+                   "host_cores": thr["host_cores"], "blas_threads": thr["blas_threads"], "kind": "oracle",
                    "sample": f"first {n} token(s) of the T={T} batch, one token at a time (its two experts "
                              f"dequantised in fp64), {dt:.1f} s"}
-        line = {
-            "metric": "MoE-layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f16 operands, f32 accumulate",
-            "data": "synthetic",
-            "config": {"workload": workload, "T": T, "E": cfg.E, "top_k": cfg.top_k,
-                       "d_model": cfg.K, "d_ff": cfg.N,
-                       "bits": sorted(set(b for sp in cfg.experts for b in sp.bits)),
-                       "format": "bit-plane+LUT" if cfg.experts[0].fmt == 1 else "int asym",
-                       "group": cfg.experts[0].group, "ranks": sorted(set(sp.rank for sp in cfg.experts)),
-                       "parallelism": f"replicas x{world}",
-                       "l2": "flushed between steps (256 MiB write, untimed)",
-                       **({"compensator": {"kind": "2D-tiled shared factors", "rank": tq[0], "tile_m": tq[1],
-                                           "tile_k": tq[2]}} if tq else {})},
-            "ms_per_step_percentiles": pct,
-            "layer_hbm_gbs": layer_b / (ms_per_step * 1e-3) / 1e9,
-            "layer_tflops": layer_f / (ms_per_step * 1e-3) / 1e12,
-            "layer_bytes_per_step": layer_b,
-            "layer_flops_per_step": layer_f,
-            "roofline": roofline,
-            "kernels_ms": kernel_means,
-            "cpu_baseline": cpu,
-            "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": T * cfg.K * 2 + T * cfg.E * 4,
-                    "d2h_bytes_per_step": T * cfg.K * 2},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks.summary(),
-        }
+        line = {"metric": "MoE-layer tokens/s", "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f16 operands, f32 accumulate", "data": "synthetic"}
+        line.update({k: v for k, v in public(head).items() if k not in ("value", "ms_per_step")})
+        line["cpu_baseline"] = cpu
+    for k in [k for k in head if k.startswith("_")]:
+        del head[k]
+    torch.cuda.empty_cache()
+    # the other workloads, on one GPU only (the scaling runs time the headline workload alone)
+    if world == 1 and not args.no_extras and not tq and args.redraw_bits < 0:
+        extras = {}
+        for name, t in EXTRAS:
+            if name == args.config and t == T:
+                continue
+            r = measure(bq, ms, name, t, dev, args.extra_steps, 3, e2e=False)
+            extras[r["config"]["workload"]] = {k: v for k, v in public(r).items() if k != "config"}
+            del r
+            torch.cuda.empty_cache()
+        line["extra_workloads"] = extras
+        line["gpu_launches"] += sum(x["gpu_launches"] for x in extras.values())
+    if rank == 0:
         print(json.dumps(line), flush=True)
-    L.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

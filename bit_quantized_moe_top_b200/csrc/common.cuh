@@ -198,7 +198,18 @@ constexpr unsigned long long kDrainLimitNs = 2000000000ull;
 // Default limit of the hand-off waits between a kernel's roles.
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
 
-// Probe of a phase without a suspend hint (a completed phase returns at once).
+// Non-blocking probe of a phase.
+__device__ __forceinline__ bool mbar_probe(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Probe of a phase without a suspend hint: a completed phase returns at once,
+// an open one may suspend the thread for a short system-dependent time.
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -208,17 +219,28 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+__device__ __forceinline__ unsigned long long clock_cycles() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%clock64;\n" : "=l"(t));
+  return t;
+}
+// Limits at least this long may sleep in try_wait; shorter ones poll.
+constexpr unsigned long long kSleepLimitNs = 2000000ull;
 // Bounded wait: gives up once limit_ns have passed, sets ST_TIMEOUT and
-// returns false. Limits far above the suspend hint sleep in try_wait; shorter
-// ones poll, so that the limit is honoured.
+// returns false. Limits far above the suspend hint sleep in try_wait and are
+// timed with the global nanosecond timer; shorter ones poll with the
+// non-blocking test_wait and are timed in SM clock cycles (two per ns, so at
+// most twice the limit at lower clocks), whose resolution, unlike the global
+// timer's, also honours limits of a few ns.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* status,
                                           unsigned long long limit_ns = kDefaultWaitNs) {
-  const bool sleep = limit_ns >= 2000000ull;
-  if (sleep ? mbar_try_wait(bar, parity) : mbar_test(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
+  const bool sleep = limit_ns >= kSleepLimitNs;
+  if (sleep ? mbar_try_wait(bar, parity) : mbar_probe(bar, parity)) return true;
+  const unsigned long long t0 = sleep ? globaltimer_ns() : clock_cycles();
   for (;;) {
-    if (sleep ? mbar_try_wait(bar, parity) : mbar_test(bar, parity)) return true;
-    if (globaltimer_ns() - t0 >= limit_ns) {
+    if (sleep ? mbar_try_wait(bar, parity) : mbar_probe(bar, parity)) return true;
+    const unsigned long long dt = sleep ? globaltimer_ns() - t0 : (clock_cycles() - t0) / 2;
+    if (dt >= limit_ns) {
       atomicOr(status, ST_TIMEOUT);
       return false;
     }
@@ -229,10 +251,11 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity
                                                    unsigned long long limit_ns) {
   return mbar_wait(bar, parity, status, limit_ns);
 }
-// Bounded wait with an inlined fast path.
+// Bounded wait with an inlined fast path (a short limit skips it: the probe
+// without a suspend hint could outlast the limit).
 __device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, unsigned* status,
                                                unsigned long long limit_ns = kDefaultWaitNs) {
-  return mbar_test(bar, parity) || mbar_wait_slow(bar, parity, status, limit_ns);
+  return (limit_ns >= kSleepLimitNs && mbar_test(bar, parity)) || mbar_wait_slow(bar, parity, status, limit_ns);
 }
 
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

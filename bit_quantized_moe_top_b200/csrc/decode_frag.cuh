@@ -217,6 +217,47 @@ __device__ __forceinline__ void load_half_planes(const uint8_t* blk, int plane_b
     pw[p] = p < BITS ? reinterpret_cast<const uint32_t*>(blk + p * plane_bytes)[2 * row + h] : 0u;
 }
 
+// ---- the same loads from shared memory, by 32-bit shared address -------------
+// (explicit ld.shared, so the hot loops never take the generic-address path)
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 lds_v2(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint4 lds_v4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+
+template <int BITS>
+__device__ __forceinline__ void lds_half_words_int(uint32_t blk, int row, int h, uint32_t (&w)[4]) {
+  if constexpr (BITS == 4) {
+    const uint4 v = lds_v4(blk + 2048 * h + 16 * row);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (BITS == 2) {
+    const uint2 v = lds_v2(blk + 16 * row + 8 * h);
+    w[0] = v.x; w[1] = v.y; w[2] = w[3] = 0u;
+  } else {
+    w[0] = lds_u32(blk + 4 * ((3 * h + 0) * 128 + row));
+    w[1] = lds_u32(blk + 4 * ((3 * h + 1) * 128 + row));
+    w[2] = lds_u32(blk + 4 * ((3 * h + 2) * 128 + row));
+    w[3] = 0u;
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ void lds_half_planes(uint32_t blk, int plane_bytes, int row, int h, uint32_t (&pw)[4]) {
+#pragma unroll
+  for (int p = 0; p < 4; ++p) pw[p] = p < BITS ? lds_u32(blk + p * plane_bytes + 4 * (2 * row + h)) : 0u;
+}
+
 // 32 dequantised fp16 pairs (k = 0..63) of one row chunk: out[16h + i] = pair i of half h
 // INT: (q - z) * s with sz = half2(s, z); bit-plane: LUT_b[code].
 template <int FMT, int BITS>

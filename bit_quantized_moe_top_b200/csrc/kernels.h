@@ -51,6 +51,14 @@ struct RouteArgs {
   void* act;                  // activation buffer, fp16 row-major [rows, Kpad]
   int Kpad;
   unsigned* status;
+  // fused kernel only
+  int* flag;                  // [1] set to epoch once the scan is done
+  unsigned epoch;             // nonzero, different for every forward of the layer
+  int nb, gs;                 // token blocks of 16, K slices of the gather
+  const ExpertDesc* experts;  // W1 descriptors (bits, group, format) for the correction sums
+  __half* corr;               // per-chunk correction sums of the gathered rows, or null
+  long long ldc;
+  unsigned long long wait_ns; // limit of the wait for the scan
 };
 
 struct DecodeArgs {
@@ -76,11 +84,11 @@ struct DecodeArgs {
   unsigned* status;
 };
 
-// Per-group correction columns of the activations for the integer-code
-// decode GEMM: for routed row p and group g of an INT block,
-// corr[p][16g .. 16g+15] = (-XP_hi, -XP_lo, -X_hi, -X_lo, 0 x 12) in fp16, with
-// XP = sum_k (P_k / 1024) x_pk and X = sum_k x_pk over the group, each split
-// into an fp16 value and its fp16 remainder.
+// Per-chunk correction columns of the activations for the integer-code
+// decode GEMM: for routed row p and 64-column chunk c of group g (cpg chunks
+// per group), corr[p][16g + 4(c % cpg) .. +3] = (-XP_hi, -XP_lo, -X_hi, -X_lo)
+// in fp16, with XP = sum_k (P_k / 1024) x_pk and X = sum_k x_pk over the
+// chunk, each split into an fp16 value and its fp16 remainder.
 struct CorrArgs {
   const ExpertDesc* experts;
   int block;
@@ -192,12 +200,15 @@ cudaError_t launch_relayout_planes(const uint32_t* canon, PlaneOut out, int M, i
 cudaError_t launch_debug_unpack(const BlockDesc& d, uint8_t* out, int block, int N, cudaStream_t st);
 
 cudaError_t launch_route_topk(const RouteArgs& a, cudaStream_t st, int* launches);
-cudaError_t launch_route_permute(const RouteArgs& a, cudaStream_t st, int* launches);
+cudaError_t launch_route_fused(const RouteArgs& a, int num_sms, cudaStream_t st, int* launches);
 int route_num_blocks(int T);
+int route_gather_slices(int T, int K);
+int device_sms();
 
 cudaError_t launch_act_corr(const CorrArgs& a, int rows_per_expert, int grid_y, cudaStream_t st, int* launches);
 int act_corr_ctas(int rows_per_expert, int K);
 int decode_rows_per_cta();
+int decode_ctas();
 cudaError_t launch_decode_gemm(const DecodeArgs& a, int ntok, int maxbits, int grid_y, cudaStream_t st,
                                int* launches);
 cudaError_t launch_lowrank(const LowrankArgs& a, int grid_y, cudaStream_t st, int* launches);

@@ -90,7 +90,8 @@ struct moe_layer {
   long long rows_pad_max = 0, nt8cap = 0;
   int nb_max = 0, ks2_max = 1, kslr_max = 1;
   long long sem_stride = 0;
-  DevBuf idx, w, counts, offsets, poffsets, active, n_active, ticket, perm, inv_pos, pinv, pslot, ptok;
+  DevBuf idx, w, counts, offsets, poffsets, active, n_active, ticket, perm, inv_pos, pinv, pslot, ptok, flag;
+  unsigned route_epoch = 0;  // value the routing kernel's scan publishes in `flag` (never 0)
   int comp_top_n = 0;
   unsigned long long wait_ns = kDefaultWaitNs;  // hand-off wait limit of the GEMM kernels
   // 2D-tiled shared compensators, per block type (0 = W1, 1 = W2)
@@ -218,7 +219,7 @@ void moe_layer_destroy(moe_layer_t* L) {
     dfree(t.z);
   }
   DevBuf* bufs[] = {&L->d_experts, &L->idx, &L->w, &L->counts, &L->offsets, &L->poffsets, &L->active,
-                    &L->n_active, &L->ticket, &L->perm, &L->inv_pos, &L->pinv, &L->pslot, &L->ptok, &L->block_counts,
+                    &L->n_active, &L->ticket, &L->flag, &L->perm, &L->inv_pos, &L->pinv, &L->pslot, &L->ptok, &L->block_counts,
                     &L->block_base, &L->pblock_base, &L->sem, &L->status, &L->xact, &L->zact, &L->obuf,
                     &L->part, &L->corr_x, &L->corr_z, &L->hx, &L->hl, &L->hy};
   for (DevBuf* b : bufs) dfree(*b);
@@ -290,6 +291,7 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   A(L->active, sizeof(int) * E);
   A(L->n_active, sizeof(int));
   A(L->ticket, sizeof(int));
+  A(L->flag, sizeof(int));
   A(L->perm, sizeof(int) * rows);
   A(L->inv_pos, sizeof(int) * rows);
   A(L->pinv, sizeof(int) * rows);
@@ -317,7 +319,7 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
     return st;
   }
   cudaError_t ce = cudaSuccess;
-  DevBuf* zero[] = {&L->ticket, &L->sem, &L->status, &L->xact, &L->zact, &L->n_active, &L->counts, &L->corr_x,
+  DevBuf* zero[] = {&L->ticket, &L->flag, &L->sem, &L->status, &L->xact, &L->zact, &L->n_active, &L->counts, &L->corr_x,
                     &L->corr_z};
   for (DevBuf* b : zero)
     if (ce == cudaSuccess) ce = cudaMemset(b->p, 0, b->n);
@@ -841,13 +843,21 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
   ra.act = L->xact.p;
   ra.Kpad = L->Kpad_x;
   ra.status = static_cast<unsigned*>(L->status.p);
-  L->prof_names.clear();
-  prof_mark(L, st, "route_topk");
-  ce = launch_route_topk(ra, st, &launches);
-  prof_mark(L, st, "route_permute");
-  if (ce == cudaSuccess) ce = launch_route_permute(ra, st, &launches);
-
   const ExpertDesc* dexp = static_cast<const ExpertDesc*>(L->d_experts.p);
+  if (++L->route_epoch == 0) L->route_epoch = 1;
+  ra.flag = static_cast<int*>(L->flag.p);
+  ra.epoch = L->route_epoch;
+  ra.nb = route_num_blocks(T);
+  ra.gs = route_gather_slices(T, K);
+  ra.experts = dexp;
+  // the decode GEMM's correction sums of the gathered rows (integer-code W1 blocks)
+  ra.corr = (!prefill && any_int[0]) ? static_cast<__half*>(L->corr_x.p) : nullptr;
+  ra.ldc = L->ldc_x;
+  ra.wait_ns = L->wait_ns;
+  L->prof_names.clear();
+  prof_mark(L, st, "route");
+  ce = launch_route_fused(ra, device_sms(), st, &launches);
+
   const long long prows = (rows + 7LL * E + 7) / 8 * 8;
   // per-group correction sums of a block's input rows (decode path, integer-code blocks)
   auto make_corr = [&](int block, const __half* act, long long lda, int Kin, __half* corr, long long ldc) {
@@ -948,11 +958,9 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     prof_mark(L, st, block == 0 ? "tileq_w1" : "tileq_w2");
     ce = launch_tileq(ta, grid_y, st, &launches);
   };
-  // W1 side compensator U1 = X A1^T
-  const CorrArgs corr1 =
-      make_corr(0, static_cast<const __half*>(L->xact.p), L->Kpad_x, K, static_cast<__half*>(L->corr_x.p), L->ldc_x);
-  lowrank(0, static_cast<__half*>(L->xact.p), L->Kpad_x, K, corr1);
-  tileq(0, corr1);
+  // W1 side compensator U1 = X A1^T (the routing kernel computed X's correction sums)
+  lowrank(0, static_cast<__half*>(L->xact.p), L->Kpad_x, K, CorrArgs{});
+  tileq(0, CorrArgs{});
   int ks2 = 1;
   if (prefill) {
     // tcgen05 path: one launch per block, CTAs over (row tile, 256-token pair, expert)
@@ -1022,11 +1030,21 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
         make_corr(1, static_cast<const __half*>(L->zact.p), L->Kpad_z, N, static_cast<__half*>(L->corr_z.p), L->ldc_z);
     lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N, corr2);
     tileq(1, corr2);
-    // split the down projection's K while its grid is small (fixed-order sum in the combine)
-    const int row_tiles = K / decode_rows_per_cta();
-    // (each split at least 256 columns wide, and at least one split: N = 128 gives one)
-    ks2 = std::min(600 / std::max(1, row_tiles * grid_y), std::min(L->ks2_max, N / 256));
-    ks2 = std::max(1, ks2);
+    // split the down projection's K (fixed-order sum of the partials in the
+    // combine) where that shortens the busiest CTA's share: each CTA takes
+    // ceil(units / CTAs) units of 128 rows x (N / 64 / KS) chunks, plus
+    // about 3 chunks of pipeline fill per unit; splits at least 256 columns
+    // wide, and at least one split (N = 128 gives one)
+    const long long units1 = (long long)(K / decode_rows_per_cta()) * grid_y;
+    const int ctas = decode_ctas(), kmax = std::max(1, std::min(L->ks2_max, N / 256));
+    double best = 0.0;
+    for (int ks = 1; ks <= kmax; ++ks) {
+      const double t = (double)((units1 * ks + ctas - 1) / ctas) * ((double)N / 64.0 / ks + 3.0);
+      if (ks == 1 || t < best * 0.98) {
+        best = t;
+        ks2 = ks;
+      }
+    }
     if (rows > 1024) ks2 = 1;
     decode_gemm(1, L->tmap_zd, L->tmap_cz, N, K, MODE_OUT, ks2);
   }

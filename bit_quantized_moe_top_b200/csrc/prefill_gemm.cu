@@ -263,7 +263,9 @@ __device__ void prefill_tile(const PrefillArgs& a, const BlockDesc& d, const pf:
 
 __global__ void __launch_bounds__(pf::kThreads, 1) prefill_gemm_kernel(const __grid_constant__ PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, as an offset into the shared array (the compiler
+  // then keeps the shared address space and emits shared-memory loads)
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ int abort_flag;
   __shared__ uint32_t tmem_slot;
   pdl_wait();
