@@ -2,31 +2,26 @@
 // 5th-generation tensor cores with the unpacked weights in TMEM.
 //
 // The decode matmuls stream weights: every packed code is read once per
-// token pass, so the kernel is bound by HBM bandwidth as long as the work of
-// unpacking and the hand-offs between roles keep up. One CTA per SM owns all
-// 512 TMEM columns and, per tile, a pair of 128-row blocks of one expert (one
-// weight row per TMEM lane, the two blocks in different columns) over a
-// group-aligned range of 64-wide K chunks and one pass of up to NTOK routed
-// tokens. CTAs are persistent and walk the (expert, row-block pair, K split,
-// token pass) tiles. Roles:
-//   warp 8     producer: per chunk, the expert's routed activation rows (TMA
-//              2-D boxes of 16 rows, shared by both row blocks), the two
-//              blocks' packed codes (one contiguous bulk copy) and, at a
-//              group's first chunk, the routed rows' correction columns and
-//              the group's scale/zero pairs; a ring of ~16 chunk stages;
-//   warps 0-7  unpack + epilogue: warp w owns row block w / 4 and TMEM lanes
-//              32 (w % 4) .. +31; per chunk a thread turns its row's 64 codes
-//              into 32 fp16 pairs and stores them into a TMEM A buffer (one
-//              tcgen05.st); after finishing group g it reads the accumulators
-//              of group g - 2 (long complete by then) and adds s * acc into
-//              fp32 registers, the scale s having come from the stage with
-//              the codes; at the end of the tile it writes SwiGLU or fp32
-//              output rows;
+// token pass, so the kernel is bound by HBM bandwidth and by the instruction
+// work of unpacking. A CTA owns 128 weight rows of one expert (one row per
+// TMEM lane) and a group-aligned range of 64-wide K chunks; CTAs are
+// persistent and walk the (expert, row block, K split, token pass) tiles.
+//   warp 8     producer: per chunk, the 128 rows' packed codes (one contiguous
+//              block), at a group's first chunk the routed rows' correction
+//              columns and the group's scale/zero pairs, and the expert's
+//              routed activation rows (TMA 2-D boxes of 16 rows, no multicast);
+//   warps 0-3  unpack: one thread per weight row turns the row's 64 codes into
+//              32 fp16 pairs in registers and stores them into a TMEM buffer
+//              (one tcgen05.st), the MMA's A operand;
 //   warp 9     allocates TMEM and issues tcgen05.mma kind::f16 with A from
-//              TMEM (M = 128 weight rows per block), B = activations from
-//              shared memory (N = tokens, rounded to 16), D in TMEM.
-// Every hand-off is an mbarrier; rings: ~16 stages (smem), 4 A buffers and 3
-// accumulator sets (TMEM).
+//              TMEM (M = 128 weight rows), B = activations from shared memory
+//              (N = tokens, 16 or 32), D in TMEM;
+//   warps 4-7  epilogue: per quantisation group, y += s * acc in fp32
+//              registers; at the end of the tile SwiGLU or fp32 output rows.
+// Every hand-off is an mbarrier; a warp's work per chunk is kept to a few
+// dozen instructions (ring positions advance incrementally, waits have an
+// inlined fast path), since that instruction stream, not the tensor core,
+// sets the pace.
 //
 // Integer codes are not dequantised per weight. The A operand holds the raw
 // fp16 values P_k + q_k of the exponent-bias unpack (exact small integers
@@ -52,8 +47,7 @@
 // Outputs: SwiGLU of the gate/up rows 8 lanes apart (W1, fp16 rows of the
 // down projection's input), or fp32 partial outputs per K split (W2, summed
 // by the combine kernel in a fixed order). Every wait is bounded; a timeout
-// sets the status word and the CTA unwinds after draining its own copies and
-// MMAs.
+// sets the status word and the CTA unwinds.
 #include <algorithm>
 
 #include "kernels.h"
@@ -64,44 +58,38 @@
 namespace moeq {
 namespace dk {
 
-#ifndef MOE_DECODE_RB
-#define MOE_DECODE_RB 2
-#endif
-constexpr int kRB = MOE_DECODE_RB;            // 128-row blocks per tile (1: two CTAs per SM; 2: one)
-constexpr int kCtasPerSm = 2 / kRB;
-constexpr int kDqWarps = 4 * kRB;             // unpack + epilogue warps
-constexpr int kMmaWarps = kRB;                // one issuing warp per row block: an issuer sustains one
-                                              // small-N MMA per ~58 cycles, whatever its N up to 64
-constexpr int kProdWarp = kDqWarps, kMmaWarp = kDqWarps + 1;
-constexpr int kThreads = 32 * (kMmaWarp + kMmaWarps);
+constexpr int kDqWarps = 4;
+constexpr int kEpWarps = 4;
+constexpr int kProdWarp = kDqWarps + kEpWarps, kMmaWarp = kProdWarp + 1;
+constexpr int kThreads = 32 * (kMmaWarp + 1);
 constexpr int kRows = 128;
-constexpr int kMaxStages = 24;
-constexpr int kA = 4;                         // TMEM A buffers, one per step (chunk)
-constexpr int kAcc = 3;                       // accumulator sets (one per group; a set holds both row blocks)
-constexpr int kLag = 2;                       // group g's accumulators are read after group g + kLag is unpacked
-constexpr int kACols = 40;                    // per row block and chunk: 32 code columns + 8 correction columns
-constexpr int kAStep = kRB * kACols;
-constexpr int kAccBase = kA * kAStep;         // accumulators after the A buffers
-constexpr int kTmemCols = 256 * kRB;
-constexpr int kActBox = 16;                   // rows per TMA box
-constexpr int kSmemBudget = 200 * 1024 / kCtasPerSm;  // stage ring
-constexpr uint32_t kOne1024 = 0x64006400u;    // fp16 pair (1024, 1024)
-static_assert(kLag < kAcc, "the accumulator ring must outrun the epilogue lag");
-static_assert(kAccBase + kAcc * kRB * 32 <= kTmemCols, "TMEM rings exceed the allocation");
+constexpr int kMaxStages = 16;  // stage ring depth: as many as about 100 KiB of shared memory hold
+constexpr int kSub = 2;         // 64-wide chunks per barrier round (step)
+constexpr int kA = 2;           // TMEM A buffers, one per step
+constexpr int kAcc = 3;         // TMEM accumulators (one per quantisation group; a step may hold two)
+constexpr int kACols = 40;      // per chunk: 32 code columns + 8 correction columns
+constexpr int kAStep = kSub * kACols;
+constexpr int kABase = 96;      // accumulators at [0, kAcc * NTOK), A buffers at [96, 256)
+constexpr int kTmemCols = 256;
+constexpr int kActBox = 16;     // rows per TMA box
+constexpr uint32_t kOne1024 = 0x64006400u;  // fp16 pair (1024, 1024)
+static_assert(kABase + kA * kAStep <= kTmemCols, "TMEM rings exceed the allocation");
+static_assert(kAcc * 32 <= kABase, "accumulators overlap the A buffers");
 
 // barrier slots (8 bytes each)
 constexpr int kBarFull = 0, kBarEmpty = kMaxStages, kBarAFull = 2 * kMaxStages, kBarAEmpty = kBarAFull + kA,
               kBarAccFull = kBarAEmpty + kA, kBarAccFree = kBarAccFull + kAcc, kBarDone = kBarAccFree + kAcc,
               kNumBars = kBarDone + 1;
 
-// code bytes of one 128-row x 64-k block at the largest bitwidth of the block's experts
+// code block bytes of a 128-row x 64-k chunk at the largest bitwidth of the block's experts
 __host__ __device__ inline int code_bytes(int maxbits) { return maxbits >= 16 ? 16384 : 1024 * maxbits; }
-// one stage (one chunk of both row blocks):
-// [act NTOK x 128 B][corr NTOK x 32 B][codes kRB x cbytes][scales kRB x 512 B]
-__host__ __device__ inline int stage_bytes(int ntok, int maxbits) {
-  const int b = ntok * 160 + kRB * code_bytes(maxbits) + kRB * 512;
+// one chunk's part of a stage: [act NTOK x 128 B][corr NTOK x 32 B][codes][scales 512 B];
+// a stage holds kSub of them (one step)
+__host__ __device__ inline int sub_stage_bytes(int ntok, int maxbits) {
+  const int b = ntok * 160 + code_bytes(maxbits) + 512;
   return (b + 1023) & ~1023;
 }
+__host__ __device__ inline int stage_bytes(int ntok, int maxbits) { return kSub * sub_stage_bytes(ntok, maxbits); }
 
 // position in a ring of n slots with the phase parity of the current lap
 struct RingPos {
@@ -116,16 +104,16 @@ struct RingPos {
 };
 
 struct Ctx {
-  int n_e, prow0, rb0, nrb, ks, kc0, nmain, next;  // row blocks rb0 .. rb0 + nrb - 1
+  int n_e, prow0, rb, ks, kc0, nmain, next;
   int tok0;  // first token (within the expert) of this tile's pass of up to NTOK tokens
 };
 
 // per-role ring positions, kept across tiles
 struct Pos {
-  RingPos st;   // stage ring (one stage per chunk)
+  RingPos st;   // stage ring (one stage per step of kSub chunks)
   RingPos rel;  // stage to release (unpack warps: kA steps behind st)
-  RingPos ab;   // A buffer ring
-  RingPos acc;  // accumulator ring (one set per group)
+  RingPos ab;   // A buffer ring (one buffer per step)
+  RingPos acc;  // accumulator ring (one per group)
   int steps = 0;
 };
 
@@ -153,44 +141,53 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
   const int n_pass = min(NTOK, c.n_e - c.tok0);
   const int nbox = (n_pass + kActBox - 1) / kActBox;
   const int row0 = c.prow0 + c.tok0;
-  const int rb0 = c.rb0;
+  const uint8_t* codes = (FMT == FMT_BITPLANE) ? d.plane[0] : d.codes;
+  const int sub_b = stage_b / kSub;
   const int n = c.nmain + c.next;
   // the whole warp runs the loop (warp-uniform values); one lane issues the copies
-  for (int i = 0; i < n; ++i, ps.st.next(a.nstages)) {
-    if (!__all_sync(0xffffffffu,
-                    !*abort_flag && mbar_wait_fast(empty + 8 * ps.st.idx, ps.st.ph ^ 1u, a.status, a.wait_ns))) {
+  for (int i0 = 0; i0 < n; i0 += kSub, ps.st.next(a.nstages)) {
+    if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait_fast(empty + 8 * ps.st.idx, ps.st.ph ^ 1u, a.status, a.wait_ns))) {
       *abort_flag = 1;
       return;
     }
-    bool first, last;
-    group_pos<FMT, GROUP>(c, i, first, last);
-    const bool main = i < c.nmain;
-    const bool corr = FMT == FMT_INT && main && first;
-    uint32_t bytes = nbox * kActBox * 128;
-    if (main) bytes += (FMT == FMT_BITPLANE ? BITS * 1024 : kBlk) * c.nrb;
-    if (corr) bytes += nbox * kActBox * 32 + 512 * c.nrb;
+    const uint32_t fb = full + 8 * ps.st.idx;
+    const int nsub = min(kSub, n - i0);
+    uint32_t bytes = 0;
+    for (int u = 0; u < nsub; ++u) {
+      bool first, last;
+      group_pos<FMT, GROUP>(c, i0 + u, first, last);
+      const bool main = i0 + u < c.nmain;
+      bytes += nbox * kActBox * 128;
+      if (main) bytes += (FMT == FMT_BITPLANE ? BITS * 1024 : kBlk);
+      if (FMT == FMT_INT && main && first) bytes += nbox * kActBox * 32 + 512;
+    }
     if (elect_one()) {
-      const uint32_t fb = full + 8 * ps.st.idx;
-      const uint32_t st = smem_u32(sm) + ps.st.idx * stage_b;
-      const uint32_t cs = st + NTOK * 160;
-      const int kc = c.kc0 + i;
-      const int kx = main ? kc * 64 : a.K + comp_col_offset(d, rb0);
-      const long long bidx = (long long)kc * RB + rb0;
       mbar_expect_tx(fb, bytes);
-      for (int b = 0; b < nbox; ++b) tma_load_2d(st + b * kActBox * 128, &a.tmap_act, kx, row0 + b * kActBox, fb);
-      if (main) {
-        if constexpr (FMT == FMT_BITPLANE) {
-          // plane p of both blocks: 2 KiB at cs + p * 2 KiB (block rb at + rb KiB)
+      for (int u = 0; u < nsub; ++u) {
+        const int i = i0 + u;
+        bool first, last;
+        group_pos<FMT, GROUP>(c, i, first, last);
+        const uint32_t st = smem_u32(sm) + ps.st.idx * stage_b + u * sub_b;
+        const bool main = i < c.nmain;
+        const int kc = c.kc0 + i;
+        const bool corr = FMT == FMT_INT && main && first;
+        const int kx = main ? kc * 64 : a.K + comp_col_offset(d, c.rb);
+        const uint32_t cs = st + NTOK * 160;
+        const long long bidx = (long long)kc * RB + c.rb;
+        const int g = kc * 64 / GROUP;
+        for (int b = 0; b < nbox; ++b) tma_load_2d(st + b * kActBox * 128, &a.tmap_act, kx, row0 + b * kActBox, fb);
+        if (main) {
+          if constexpr (FMT == FMT_BITPLANE) {
 #pragma unroll
-          for (int q = 0; q < BITS; ++q) bulk_g2s(cs + q * kRB * 1024, d.plane[q] + bidx * 1024, 1024 * c.nrb, fb);
-        } else {
-          bulk_g2s(cs, d.codes + bidx * kBlk, kBlk * c.nrb, fb);
-        }
-        if (corr) {
-          const int g = kc * 64 / GROUP;
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d(st + NTOK * 128 + b * kActBox * 32, &a.tmap_corr, 16 * g, row0 + b * kActBox, fb);
-          bulk_g2s(cs + kRB * cbytes, d.sz + (long long)g * a.M + rb0 * kRows, 512 * c.nrb, fb);
+            for (int q = 0; q < BITS; ++q) bulk_g2s(cs + q * 1024, d.plane[q] + bidx * 1024, 1024, fb);
+          } else {
+            bulk_g2s(cs, codes + bidx * kBlk, kBlk, fb);
+          }
+          if (corr) {
+            for (int b = 0; b < nbox; ++b)
+              tma_load_2d(st + NTOK * 128 + b * kActBox * 32, &a.tmap_corr, 16 * g, row0 + b * kActBox, fb);
+            bulk_g2s(cs + cbytes, d.sz + (long long)g * a.M + c.rb * kRows, 512, fb);
+          }
         }
       }
     }
@@ -207,96 +204,68 @@ __device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int s
   const int n_pass = min(NTOK, c.n_e - c.tok0);
   const uint32_t idesc = idesc_f16(128, (n_pass + 15) & ~15);
   const uint32_t sm0 = smem_u32(sm);
+  const int sub_b = stage_b / kSub;
   const int n = c.nmain + c.next;
-  for (int i = 0; i < n; ++i) {
+  for (int i0 = 0; i0 < n; i0 += kSub) {
     const bool ok = !*abort_flag && mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status, a.wait_ns) &&
                     mbar_wait_fast(afull + 8 * ps.ab.idx, ps.ab.ph, a.status, a.wait_ns);
     if (!__all_sync(0xffffffffu, ok)) {
       *abort_flag = 1;
       return;
     }
-    bool first, last;
-    group_pos<FMT, GROUP>(c, i, first, last);
-    if (first && !__all_sync(0xffffffffu, !*abort_flag && mbar_wait_fast(accfree + 8 * ps.acc.idx, ps.acc.ph ^ 1u,
-                                                                          a.status, a.wait_ns))) {
-      *abort_flag = 1;
-      return;
-    }
     tc_fence_after();
-    const uint32_t bt = sm0 + ps.st.idx * stage_b;
-    const bool corr = FMT == FMT_INT && i < c.nmain && first;
-    const uint64_t dact = sw128_desc(bt), dcorr = sw32_desc(bt + NTOK * 128);
-    // the whole warp runs the loop (warp-uniform values); one lane issues,
-    // for this warp's row block (a warp whose block is absent only commits)
-    const int rb = (threadIdx.x >> 5) - kMmaWarp;
-    if (elect_one()) {
-      if (rb < c.nrb) {
-        const uint32_t acc = tmem + kAccBase + (ps.acc.idx * kRB + rb) * NTOK;
-        const uint32_t ta = tmem + ps.ab.idx * kAStep + rb * kACols;
+    const int nsub = min(kSub, n - i0);
+    for (int u = 0; u < nsub; ++u) {
+      const int i = i0 + u;
+      bool first, last;
+      group_pos<FMT, GROUP>(c, i, first, last);
+      if (first) {
+        if (!__all_sync(0xffffffffu,
+                        !*abort_flag && mbar_wait_fast(accfree + 8 * ps.acc.idx, ps.acc.ph ^ 1u, a.status, a.wait_ns))) {
+          *abort_flag = 1;
+          return;
+        }
+        tc_fence_after();
+      }
+      const uint32_t bt = sm0 + ps.st.idx * stage_b + u * sub_b;
+      const uint32_t acc = tmem + ps.acc.idx * NTOK;
+      const uint32_t ta = tmem + kABase + ps.ab.idx * kAStep + u * kACols;
+      const bool corr = FMT == FMT_INT && i < c.nmain && first;
+      const uint64_t dact = sw128_desc(bt), dcorr = sw32_desc(bt + NTOK * 128);
+      // the whole warp runs the loop (warp-uniform values); one lane issues
+      if (elect_one()) {
         if (corr) mma_f16_ts(acc, ta + 32, dcorr, idesc, 0);
 #pragma unroll
         for (int k16 = 0; k16 < 4; ++k16)
           mma_f16_ts(acc, ta + k16 * 8, dact + 2 * k16, idesc, (corr || !first || k16 > 0) ? 1 : 0);
+        if (last) mma_commit(accfull + 8 * ps.acc.idx);
       }
-      // the chunk's A buffer and stage are read once its MMAs complete
-      mma_commit(aempty + 8 * ps.ab.idx);
-      if (last) mma_commit(accfull + 8 * ps.acc.idx);
+      __syncwarp();
+      if (last) ps.acc.next(kAcc);
     }
+    // the step's A buffer and stage are read once all its MMAs complete
+    if (elect_one()) mma_commit(aempty + 8 * ps.ab.idx);
     __syncwarp();
-    if (last) ps.acc.next(kAcc);
     ps.st.next(a.nstages);
     ps.ab.next(kA);
   }
 }
 
-// One group's accumulators into y: wait until its MMAs completed, read the
-// row's NTOK columns, y += scale * acc, hand the accumulator set back.
-template <int NTOK>
-__device__ __forceinline__ bool epilogue_group(const DecodeArgs& a, uint32_t bars, uint32_t tmem_row, float scale,
-                                               float (&y)[NTOK], Pos& ps, volatile int* abort_flag) {
-  const uint32_t accfull = bars + 8 * kBarAccFull, accfree = bars + 8 * kBarAccFree;
-  if (!__all_sync(0xffffffffu,
-                  !*abort_flag && mbar_wait_fast(accfull + 8 * ps.acc.idx, ps.acc.ph, a.status, a.wait_ns))) {
-    *abort_flag = 1;
-    return false;
-  }
-  tc_fence_after();
-  uint32_t v[NTOK];
-  tmem_ld<NTOK>(tmem_row + ps.acc.idx * kRB * NTOK, v);
-#pragma unroll
-  for (int t = 0; t < NTOK; ++t) y[t] = fmaf(scale, __uint_as_float(v[t]), y[t]);
-  tc_fence_before();
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(accfree + 8 * ps.acc.idx);
-  ps.acc.next(kAcc);
-  return true;
-}
-
 template <int NTOK, int FMT, int BITS, int GROUP>
-__device__ void unpack_epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, uint8_t* sm, int stage_b,
-                                int cbytes, uint32_t bars, uint32_t tmem, Pos& ps, volatile int* abort_flag) {
+__device__ void unpack(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, uint8_t* sm, int stage_b, int cbytes,
+                       uint32_t bars, uint32_t tmem, Pos& ps, volatile int* abort_flag) {
   const uint32_t full = bars + 8 * kBarFull, empty = bars + 8 * kBarEmpty;
   const uint32_t afull = bars + 8 * kBarAFull, aempty = bars + 8 * kBarAEmpty;
-  constexpr int kBlk = (FMT == FMT_DENSE) ? 16384 : 128 * 8 * BITS;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rb = warp >> 2;                           // row block of the pair
-  const int row = ((warp & 3) << 5) + lane;           // TMEM lane = row within the block
-  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-  const bool rvalid = rb < c.nrb;
-  const int R = (c.rb0 + rb) * kRows + row;          // internal row of the block
+  const int lane = threadIdx.x & 31;
+  const int row = threadIdx.x;  // 0..127 = TMEM lane
+  const uint32_t lane_base = (uint32_t)(row & ~31) << 16;
   LutRegs lut;
   if constexpr (FMT == FMT_BITPLANE) lut = load_lut(d.lut, BITS);
   const int RS2 = d.rank / 2;  // compensator column pairs
+  const int R = c.rb * kRows + row;
+  const int sub_b = stage_b / kSub;
   const int n = c.nmain + c.next;
-  const uint32_t tmem_acc_row = tmem + lane_base + kAccBase + rb * NTOK;
-  const uint32_t sm0 = smem_u32(sm);
-  float y[NTOK];
-#pragma unroll
-  for (int t = 0; t < NTOK; ++t) y[t] = 0.f;
-  // scales of the last groups unpacked: sh0 = newest
-  float s_cur = 1.f, sh0 = 1.f, sh1 = 1.f, sh2 = 1.f;
-  int gdone = 0, gepi = 0;
-  for (int i = 0; i < n; ++i) {
+  for (int i0 = 0; i0 < n; i0 += kSub) {
     // warp-uniform waits: every lane reaches the .sync.aligned TMEM stores
     const bool ok = !*abort_flag && mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status, a.wait_ns) &&
                     mbar_wait_fast(aempty + 8 * ps.ab.idx, ps.ab.ph ^ 1u, a.status, a.wait_ns);
@@ -310,89 +279,109 @@ __device__ void unpack_epilogue(const DecodeArgs& a, const BlockDesc& d, const C
       if (lane == 0) mbar_arrive(empty + 8 * ps.rel.idx);
       ps.rel.next(a.nstages);
     }
-    bool first, last;
-    group_pos<FMT, GROUP>(c, i, first, last);
-    const uint32_t ta = tmem + lane_base + ps.ab.idx * kAStep + rb * kACols;
-    const uint32_t stg = sm0 + ps.st.idx * stage_b;
-    uint32_t v[32];
-    if (i < c.nmain) {
-      const uint32_t cs = stg + NTOK * 160;
-      if constexpr (FMT == FMT_INT) {
-        if (first) {
-          const uint32_t sz = lds_u32(cs + kRB * cbytes + 4 * (rb * kRows + row));
-          s_cur = __half2float(__ushort_as_half((uint16_t)(sz & 0xFFFFu)));
-          // (1024, 1024), (z, z) against chunk 0's (-XP_hi, -XP_lo), (-X_hi, -X_lo),
-          // and for two-chunk groups again against chunk 1's (zeros otherwise:
-          // those slots may hold another expert's sums from an earlier forward)
-          const uint32_t zz = prmt(sz, sz, 0x3232u);
-          const uint32_t cz[4] = {kOne1024, zz, GROUP > 64 ? kOne1024 : 0u, GROUP > 64 ? zz : 0u};
-          tmem_st4_nw(ta + 32, cz);
-        }
-        const uint32_t blk = cs + rb * kBlk;
-        uint32_t w0[4], w1[4];
-        lds_half_words_int<BITS>(blk, row, 0, w0);
-        lds_half_words_int<BITS>(blk, row, 1, w1);
-        uint32_t r0[16], r1[16];
-        int_raw_half<BITS>(w0, r0);
-        int_raw_half<BITS>(w1, r1);
+    const int nsub = min(kSub, n - i0);
+    for (int u = 0; u < nsub; ++u) {
+      const int i = i0 + u;
+      bool first, last;
+      group_pos<FMT, GROUP>(c, i, first, last);
+      const uint32_t ta = tmem + lane_base + kABase + ps.ab.idx * kAStep + u * kACols;
+      uint32_t v[32];
+      if (i < c.nmain) {
+        const uint8_t* cs = sm + ps.st.idx * stage_b + u * sub_b + NTOK * 160;
+        if constexpr (FMT == FMT_INT) {
+          if (first) {
+            const uint32_t sz = lds_u32(smem_u32(cs + cbytes) + 4 * row);
+            // (1024, 1024), (z, z) against chunk 0's (-XP_hi, -XP_lo), (-X_hi, -X_lo),
+            // and for two-chunk groups again against chunk 1's (zeros otherwise:
+            // those slots may hold another expert's sums from an earlier forward)
+            const uint32_t zz = prmt(sz, sz, 0x3232u);
+            const uint32_t cz[4] = {kOne1024, zz, GROUP > 64 ? kOne1024 : 0u, GROUP > 64 ? zz : 0u};
+            tmem_st4_nw(ta + 32, cz);
+          }
+          const uint32_t blk = smem_u32(cs);
+          uint32_t w0[4], w1[4], r0[16], r1[16];
+          lds_half_words_int<BITS>(blk, row, 0, w0);
+          lds_half_words_int<BITS>(blk, row, 1, w1);
+          int_raw_half<BITS>(w0, r0);
+          int_raw_half<BITS>(w1, r1);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          v[j] = r0[j];
-          v[16 + j] = r1[j];
-        }
-      } else if constexpr (FMT == FMT_BITPLANE) {
-        s_cur = 1.f;
-        uint32_t p0[4], p1[4];
-        lds_half_planes<BITS>(cs + rb * 1024, kRB * 1024, row, 0, p0);
-        lds_half_planes<BITS>(cs + rb * 1024, kRB * 1024, row, 1, p1);
-        uint32_t r0[16], r1[16];
-        lut_half<BITS>(p0, lut, r0);
-        lut_half<BITS>(p1, lut, r1);
+          for (int j = 0; j < 16; ++j) {
+            v[j] = r0[j];
+            v[16 + j] = r1[j];
+          }
+        } else if constexpr (FMT == FMT_BITPLANE) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          v[j] = r0[j];
-          v[16 + j] = r1[j];
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pw[4], r16[16];
+            load_half_planes<BITS>(cs, 1024, row, h, pw);
+            lut_half<BITS>(pw, lut, r16);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[16 * h + j] = r16[j];
+          }
+        } else {
+#pragma unroll
+          for (int qd = 0; qd < 8; ++qd) {
+            const uint4 x = reinterpret_cast<const uint4*>(cs + qd * 2048)[row];
+            v[4 * qd] = x.x; v[4 * qd + 1] = x.y; v[4 * qd + 2] = x.z; v[4 * qd + 3] = x.w;
+          }
         }
       } else {
-        s_cur = 1.f;
-        const uint32_t blk = cs + rb * kBlk;
+        // compensator stage: the row's B values (pairs), zero past the rank
 #pragma unroll
-        for (int qd = 0; qd < 8; ++qd) {
-          const uint4 x = lds_v4(blk + qd * 2048 + 16 * row);
-          v[4 * qd] = x.x; v[4 * qd + 1] = x.y; v[4 * qd + 2] = x.z; v[4 * qd + 3] = x.w;
-        }
+        for (int j = 0; j < 32; ++j) v[j] = j < RS2 ? d.brow[(long long)j * a.M + R] : 0u;
       }
-    } else {
-      // compensator stage: the row's B values (pairs), zero past the rank
-      s_cur = 1.f;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = (rvalid && j < RS2) ? d.brow[(long long)j * a.M + R] : 0u;
+      tmem_st32(ta, v);  // includes the wait for the store
     }
-    tmem_st32(ta, v);  // includes the wait for the store
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(afull + 8 * ps.ab.idx);
     ps.st.next(a.nstages);
     ps.ab.next(kA);
     ++ps.steps;
-    if (last) {
-      sh2 = sh1;
-      sh1 = sh0;
-      sh0 = s_cur;
-      ++gdone;
-      if (gdone - gepi > kLag) {
-        // group gdone - 1 - kLag (scale sh2): its MMAs were issued kLag groups ago
-        if (!epilogue_group<NTOK>(a, bars, tmem_acc_row, sh2, y, ps, abort_flag)) return;
-        ++gepi;
-      }
-    }
   }
-  // the last groups of the tile
-  if (gdone - gepi == 2) {
-    if (!epilogue_group<NTOK>(a, bars, tmem_acc_row, sh1, y, ps, abort_flag)) return;
-    if (!epilogue_group<NTOK>(a, bars, tmem_acc_row, sh0, y, ps, abort_flag)) return;
-  } else if (gdone - gepi == 1) {
-    if (!epilogue_group<NTOK>(a, bars, tmem_acc_row, sh0, y, ps, abort_flag)) return;
+}
+
+template <int NTOK, int FMT, int GROUP>
+__device__ void epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, uint32_t bars, uint32_t tmem,
+                         Pos& ps, volatile int* abort_flag) {
+  const uint32_t accfull = bars + 8 * kBarAccFull, accfree = bars + 8 * kBarAccFree;
+  const int lane = threadIdx.x & 31;
+  const int row = threadIdx.x - 32 * kDqWarps;  // 0..127 = TMEM lane
+  const uint32_t lane_base = (uint32_t)(row & ~31) << 16;
+  const int R = c.rb * kRows + row;
+  int nmain_groups = 0;
+  if constexpr (FMT == FMT_INT) nmain_groups = c.nmain / (GROUP / 64);
+  else nmain_groups = c.nmain > 0 ? 1 : 0;
+  const int g0 = (FMT == FMT_INT) ? c.kc0 / (GROUP / 64) : 0;
+  float y[NTOK];
+#pragma unroll
+  for (int t = 0; t < NTOK; ++t) y[t] = 0.f;
+  // the row's group scales, loaded kPre groups ahead of their use (they come
+  // from L2: the producer's copies of the same words went through it)
+  constexpr int kPre = 4;
+  uint32_t pre[kPre];
+#pragma unroll
+  for (int q = 0; q < kPre; ++q)
+    pre[q] = (FMT == FMT_INT && q < nmain_groups) ? d.sz[(long long)(g0 + q) * a.M + R] : 0x3C00u;
+  for (int gi = 0; gi < nmain_groups + c.next; ++gi) {
+    float s = 1.f;
+    if (FMT == FMT_INT && gi < nmain_groups) s = __half2float(__ushort_as_half((uint16_t)(pre[0] & 0xFFFFu)));
+#pragma unroll
+    for (int q = 0; q < kPre - 1; ++q) pre[q] = pre[q + 1];
+    pre[kPre - 1] = (FMT == FMT_INT && gi + kPre < nmain_groups) ? d.sz[(long long)(g0 + gi + kPre) * a.M + R] : 0x3C00u;
+    if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait_fast(accfull + 8 * ps.acc.idx, ps.acc.ph, a.status, a.wait_ns))) {
+      *abort_flag = 1;
+      return;
+    }
+    tc_fence_after();
+    uint32_t v[NTOK];
+    tmem_ld<NTOK>(tmem + lane_base + ps.acc.idx * NTOK, v);
+#pragma unroll
+    for (int t = 0; t < NTOK; ++t) y[t] = fmaf(s, __uint_as_float(v[t]), y[t]);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(accfree + 8 * ps.acc.idx);
+    ps.acc.next(kAcc);
   }
   // ---- outputs: tokens tok0 + t
   const int nt = min(NTOK, c.n_e - c.tok0);
@@ -401,7 +390,7 @@ __device__ void unpack_epilogue(const DecodeArgs& a, const BlockDesc& d, const C
     float up[NTOK];
 #pragma unroll
     for (int t = 0; t < NTOK; ++t) up[t] = __shfl_down_sync(0xffffffffu, y[t], 8);
-    if (rvalid && (R & 15) < 8) {
+    if ((R & 15) < 8) {
       const int col = 8 * (R >> 4) + (R & 7);
 #pragma unroll
       for (int t = 0; t < NTOK; ++t) {
@@ -411,7 +400,7 @@ __device__ void unpack_epilogue(const DecodeArgs& a, const BlockDesc& d, const C
         }
       }
     }
-  } else if (rvalid) {
+  } else {
 #pragma unroll
     for (int t = 0; t < NTOK; ++t)
       if (t < nt) a.out[c.ks * a.out_ks_stride + (long long)(c.prow0 + c.tok0 + t) * a.M + R] = y[t];
@@ -436,7 +425,9 @@ __device__ void decode_tile(const DecodeArgs& a, const BlockDesc& d, const Ctx& 
   }
   const int warp = threadIdx.x >> 5;
   if (warp < kDqWarps) {
-    unpack_epilogue<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, tmem, ps, ab);
+    unpack<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, tmem, ps, ab);
+  } else if (warp < kProdWarp) {
+    epilogue<NTOK, FMT, GROUP>(a, d, c, bars, tmem, ps, ab);
   } else if (warp == kProdWarp) {
     producer<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, ps, ab);
   } else {
@@ -447,11 +438,10 @@ __device__ void decode_tile(const DecodeArgs& a, const BlockDesc& d, const Ctx& 
 }  // namespace dk
 
 template <int NTOK>
-__global__ void __launch_bounds__(dk::kThreads, dk::kCtasPerSm) decode_gemm_kernel(const __grid_constant__ DecodeArgs a,
+__global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __grid_constant__ DecodeArgs a,
                                                                         int stage_b, int cbytes) {
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte aligned base, as an offset into the shared array (the compiler
-  // then keeps the shared address space and emits shared-memory loads)
+  // 1024-byte aligned base, as an offset into the shared array
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ __align__(8) unsigned long long bars[dk::kNumBars];
   __shared__ int s_pre[kMaxExperts + 1];
@@ -467,13 +457,13 @@ __global__ void __launch_bounds__(dk::kThreads, dk::kCtasPerSm) decode_gemm_kern
     }
     for (int i = 0; i < dk::kA; ++i) {
       mbar_init(b0 + 8 * (dk::kBarAFull + i), dk::kDqWarps);      // A buffer written
-      mbar_init(b0 + 8 * (dk::kBarAEmpty + i), dk::kMmaWarps);    // A buffer read (MMA commits)
+      mbar_init(b0 + 8 * (dk::kBarAEmpty + i), 1);                // A buffer read (MMA commit)
     }
     for (int i = 0; i < dk::kAcc; ++i) {
-      mbar_init(b0 + 8 * (dk::kBarAccFull + i), dk::kMmaWarps);   // accumulators complete (MMA commits)
-      mbar_init(b0 + 8 * (dk::kBarAccFree + i), dk::kDqWarps);    // accumulators read
+      mbar_init(b0 + 8 * (dk::kBarAccFull + i), 1);               // accumulator complete (MMA commit)
+      mbar_init(b0 + 8 * (dk::kBarAccFree + i), dk::kEpWarps);    // accumulator read
     }
-    mbar_init(done_bar, dk::kMmaWarps);
+    mbar_init(done_bar, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -482,26 +472,22 @@ __global__ void __launch_bounds__(dk::kThreads, dk::kCtasPerSm) decode_gemm_kern
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  if (warp < dk::kDqWarps) {
-    // correction columns of this warp's A buffers: zeros past the four that
-    // each group's first chunk writes
-    const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t cz[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-    for (int b = 0; b < dk::kA; ++b)
-      tmem_st8_nw(tmem + lb + b * dk::kAStep + (warp >> 2) * dk::kACols + 32, cz);
+  if (warp < 4) {
+    // constant correction columns of the A buffers: (1024, 1024), then zeros
+    const uint32_t lb = (uint32_t)(warp * 32) << 16;
+    const uint32_t cz[8] = {dk::kOne1024, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    for (int b = 0; b < dk::kA * dk::kSub; ++b) tmem_st8_nw(tmem + lb + dk::kABase + b * dk::kACols + 32, cz);
     tmem_wait_st();
   }
   // everything above overlaps the previous kernel's tail
   pdl_wait();
   pdl_trigger();
-  // Work units: per active expert slot, (token pass, K split, row block),
-  // row blocks fastest. Each CTA takes a contiguous, balanced range of units
-  // and walks it two adjacent row blocks at a time (one where a pair would
-  // leave its range, its expert, pass or split, or straddle a 2D-tiled
-  // compensator's row tile). s_pre = exclusive prefix of the token passes
-  // (ceil(n_e / NTOK)) over the slots.
+  // Tiles: per active expert slot, (row block, K split, token pass) with the
+  // passes of one (row block, K split) adjacent, so that they run at about the
+  // same time and share the weight block through L2. s_pre = exclusive prefix
+  // of the token passes (ceil(n_e / NTOK)) over the slots.
   const int RB = a.M / dk::kRows;
-  const long long per = (long long)RB * a.KS;
+  const int per = RB * a.KS;
   const int nact = *a.n_active;
   if (warp == 0) {
     const int lane = threadIdx.x & 31;
@@ -530,30 +516,30 @@ __global__ void __launch_bounds__(dk::kThreads, dk::kCtasPerSm) decode_gemm_kern
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const long long units = (long long)s_pre[nact] * per;
-  const long long u_end = units * (blockIdx.x + 1) / gridDim.x;
+  // each CTA takes a contiguous, balanced range of the tiles (passes of one
+  // row block and K split adjacent: they reuse its weights from L2)
+  const int total = s_pre[nact] * per;
   volatile int* ab = &abort_flag;
   dk::Pos ps;
-  for (long long u = units * blockIdx.x / gridDim.x; u < u_end && !*ab;) {
+  const int tile_end = (int)((long long)total * (blockIdx.x + 1) / gridDim.x);
+  for (int tile = (int)((long long)total * blockIdx.x / gridDim.x); tile < tile_end && !*ab; ++tile) {
     int lo = 0, hi = nact - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (s_pre[mid] * per <= u) lo = mid;
+      if (s_pre[mid] * per <= tile) lo = mid;
       else hi = mid - 1;
     }
     const int slot = lo;
-    const long long local = u - s_pre[slot] * per;
+    const int np = s_pre[slot + 1] - s_pre[slot];
+    const int local = tile - s_pre[slot] * per;
     const int e = a.active[slot];
     dk::Ctx c;
     c.n_e = a.counts[e];
     c.prow0 = a.poffsets[e];
-    c.rb0 = (int)(local % RB);
-    c.ks = (int)((local / RB) % a.KS);
-    c.tok0 = (int)(local / per) * NTOK;
+    c.tok0 = (local % np) * NTOK;
+    c.rb = (local / np) / a.KS;
+    c.ks = (local / np) % a.KS;
     const BlockDesc& d = a.experts[e].blk[a.block];
-    c.nrb = (dk::kRB > 1 && u + 1 < u_end && c.rb0 + 1 < RB &&
-             comp_col_offset(d, c.rb0) == comp_col_offset(d, c.rb0 + 1)) ? 2 : 1;
-    u += c.nrb;
     c.next = (c.ks == 0 && d.rank > 0) ? 1 : 0;
     c.kc0 = c.nmain = 0;
     bool ran = true;
@@ -598,7 +584,7 @@ __global__ void __launch_bounds__(dk::kThreads, dk::kCtasPerSm) decode_gemm_kern
       if (!mbar_wait_fast(b0 + 8 * (dk::kBarFull + p.idx), p.ph, a.status, kDrainLimitNs)) break;
     }
   }
-  if (warp >= dk::kMmaWarp && (threadIdx.x & 31) == 0) {
+  if (warp == dk::kMmaWarp && (threadIdx.x & 31) == 0) {
     // every issued MMA must complete before TMEM is released
     mma_commit(done_bar);
     mbar_wait(done_bar, 0, a.status, kDrainLimitNs);
@@ -644,26 +630,27 @@ static int num_sms() {
 }
 
 int decode_rows_per_cta() { return dk::kRows; }
-int decode_ctas() { return dk::kCtasPerSm * num_sms(); }
+int decode_ctas() { return 2 * num_sms(); }
 int device_sms() { return num_sms(); }
 
 template <int NTOK>
 static cudaError_t launch_ntok(const DecodeArgs& a, int maxbits, int grid_y, cudaStream_t st) {
   const int stage_b = dk::stage_bytes(NTOK, maxbits);
-  // a stage ring as deep as the CTA's share of about 200 KiB of shared
-  // memory per SM holds, so that enough weight bytes are in flight per SM (a
-  // stage is released kA chunks after its own; kA + 2 stages keep the
-  // producer ahead even for the large dense code blocks)
+  // two CTAs per SM (2 x 256 TMEM columns): each takes about 100 KiB of
+  // stages (a stage holds one step of kSub chunks), as deep a ring as fits,
+  // to keep enough weight bytes in flight (a stage is released kA steps
+  // after its own; kA + 2 stages keep the producer ahead, even for the large
+  // dense code blocks, which then leave room for one CTA per SM)
   DecodeArgs b = a;
-  b.nstages = std::max(dk::kA + 2, std::min(dk::kMaxStages, dk::kSmemBudget / stage_b));
+  b.nstages = std::max(dk::kA + 2, std::min(dk::kMaxStages, (100 * 1024 - 1024) / stage_b));
   const size_t smem = (size_t)b.nstages * stage_b + 1024;
   cudaError_t err = cudaFuncSetAttribute(decode_gemm_kernel<NTOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
   if (err != cudaSuccess) return err;
   // at most rows / NTOK + (one ragged pass per expert) token passes
   const long long passes = std::min<long long>(a.rows / NTOK + grid_y, a.rows);
-  const long long units = passes * (a.M / dk::kRows) * a.KS;
-  const int grid = (int)std::min<long long>(units, (long long)dk::kCtasPerSm * num_sms());
+  const long long tiles = passes * (a.M / dk::kRows) * a.KS;
+  const int grid = (int)std::min<long long>(tiles, 2LL * num_sms());
   return launch_kernel(decode_gemm_kernel<NTOK>, dim3(grid), dim3(dk::kThreads), smem, st, true, b, stage_b,
                        dk::code_bytes(maxbits));
 }
