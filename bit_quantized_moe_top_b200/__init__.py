@@ -193,8 +193,10 @@ def moe_layer_last_launch_count(layer: int) -> int:
     return _lib().moe_layer_last_launch_count(layer)
 
 
-def moe_layer_set_profiling(layer: int, enable: bool) -> None:
-    _check(_lib().moe_layer_set_profiling(layer, 1 if enable else 0), "moe_layer_set_profiling")
+def moe_layer_set_profiling(layer: int, enable) -> None:
+    """enable: False/0 off, True/1 every kernel, 2 the gate/up expert GEMM alone."""
+    level = int(enable) if not isinstance(enable, bool) else (1 if enable else 0)
+    _check(_lib().moe_layer_set_profiling(layer, level), "moe_layer_set_profiling")
 
 
 def moe_layer_kernel_times(layer: int, cap: int = 64):

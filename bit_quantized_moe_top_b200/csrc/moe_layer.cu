@@ -111,27 +111,55 @@ struct moe_layer {
   int last_T = 0, last_k = 0, last_launches = 0;
   cudaStream_t last_stream = nullptr;
   cudaEvent_t fwd_done = nullptr;  // recorded at the end of every forward (page release orders after it)
-  // profiling: events around each launch of the last forward
-  bool profiling = false;
+  // profiling: events around each launch of the last forward (1), or around
+  // the gate/up expert GEMM alone (2: the other launches keep their overlap)
+  int profiling = 0;
+  bool prof_open = false;
   std::vector<cudaEvent_t> events;
   std::vector<const char*> prof_names;
   int prof_count = -1;
 };
 
-// records an event before a kernel (profiling only); returns the slot
-static void prof_mark(moe_layer_t* L, cudaStream_t st, const char* name) {
-  if (!L->profiling) return;
-  const size_t i = L->prof_names.size();
-  while (L->events.size() < i + 2) {
+static bool ensure_events(moe_layer_t* L, size_t n) {
+  while (L->events.size() < n) {
     cudaEvent_t ev;
-    if (cudaEventCreate(&ev) != cudaSuccess) return;
+    if (cudaEventCreate(&ev) != cudaSuccess) return false;
     L->events.push_back(ev);
   }
+  return true;
+}
+static bool is_gate_up_gemm(const char* name) { return std::strstr(name, "gemm_w1") != nullptr; }
+// records an event before a kernel (profiling only)
+static void prof_mark(moe_layer_t* L, cudaStream_t st, const char* name) {
+  if (!L->profiling) return;
+  if (L->profiling == 2) {
+    // level 2: one event before the gate/up GEMM and one after it
+    if (L->prof_open) {
+      cudaEventRecord(L->events[1], st);
+      L->prof_open = false;
+    }
+    if (is_gate_up_gemm(name) && ensure_events(L, 2)) {
+      cudaEventRecord(L->events[0], st);
+      L->prof_names.assign(1, name);
+      L->prof_open = true;
+    }
+    return;
+  }
+  const size_t i = L->prof_names.size();
+  if (!ensure_events(L, i + 2)) return;
   cudaEventRecord(L->events[i], st);
   L->prof_names.push_back(name);
 }
 static void prof_end(moe_layer_t* L, cudaStream_t st) {
   if (!L->profiling) return;
+  if (L->profiling == 2) {
+    if (L->prof_open) {
+      cudaEventRecord(L->events[1], st);
+      L->prof_open = false;
+    }
+    L->prof_count = (int)L->prof_names.size();
+    return;
+  }
   const size_t i = L->prof_names.size();
   if (L->events.size() > i) cudaEventRecord(L->events[i], st);
   L->prof_count = (int)i;
@@ -765,8 +793,9 @@ moe_status_t moe_layer_set_path(moe_layer_t* L, int path) {
 int moe_layer_last_launch_count(const moe_layer_t* L) { return L ? L->last_launches : 0; }
 
 moe_status_t moe_layer_set_profiling(moe_layer_t* L, int enable) {
-  if (!L) return MOE_ERR_INVALID_ARG;
-  L->profiling = enable != 0;
+  if (!L || enable < 0 || enable > 2) return MOE_ERR_INVALID_ARG;
+  L->profiling = enable;
+  L->prof_open = false;
   L->prof_count = -1;
   return MOE_OK;
 }

@@ -276,8 +276,10 @@ moe_status_t moe_layer_sync_status(moe_layer_t* layer);
 /* Number of kernels the last moe_layer_forward launched. */
 int moe_layer_last_launch_count(const moe_layer_t* layer);
 
-/* Profiling. When enabled (enable != 0), every forward records a CUDA event on
- * its stream before and after each kernel it launches. */
+/* Profiling. enable = 1: every forward records a CUDA event on its stream
+ * before and after each kernel it launches. enable = 2: only the gate/up
+ * expert GEMM (decode or prefill) is bracketed, so that the other launches keep
+ * their programmatic overlap. enable = 0: off. Other values: MOE_ERR_INVALID_ARG. */
 moe_status_t moe_layer_set_profiling(moe_layer_t* layer, int enable);
 
 /* Durations in ms of the kernels of the last profiled forward, in launch order:
