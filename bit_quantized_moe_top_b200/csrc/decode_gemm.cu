@@ -106,6 +106,13 @@ struct RingPos {
 struct Ctx {
   int n_e, prow0, rb, ks, kc0, nmain, next;
   int tok0;  // first token (within the expert) of this tile's pass of up to NTOK tokens
+  // the part of the tile this CTA runs: chunks [ib, ie) of the tile's nmain
+  // main chunks and its compensator stage (a whole number of steps); a tile
+  // split between two CTAs has a head part (this CTA finishes the tile after
+  // adding the other CTA's partial sums) and a tail part (written as partial
+  // sums for the head's CTA)
+  int ib, ie;
+  int head_wait, tail_write;
 };
 
 // per-role ring positions, kept across tiles
@@ -127,8 +134,8 @@ __device__ __forceinline__ void group_pos(const Ctx& c, int i, bool& first, bool
     first = (i % cpg) == 0;
     last = (i % cpg) == cpg - 1;
   } else {
-    first = i == 0;
-    last = i == c.nmain - 1;
+    first = i == c.ib;
+    last = i == min(c.ie, c.nmain) - 1;
   }
 }
 
@@ -143,9 +150,9 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
   const int row0 = c.prow0 + c.tok0;
   const uint8_t* codes = (FMT == FMT_BITPLANE) ? d.plane[0] : d.codes;
   const int sub_b = stage_b / kSub;
-  const int n = c.nmain + c.next;
+  const int n = c.ie;
   // the whole warp runs the loop (warp-uniform values); one lane issues the copies
-  for (int i0 = 0; i0 < n; i0 += kSub, ps.st.next(a.nstages)) {
+  for (int i0 = c.ib; i0 < n; i0 += kSub, ps.st.next(a.nstages)) {
     if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait_fast(empty + 8 * ps.st.idx, ps.st.ph ^ 1u, a.status, a.wait_ns))) {
       *abort_flag = 1;
       return;
@@ -205,8 +212,8 @@ __device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int s
   const uint32_t idesc = idesc_f16(128, (n_pass + 15) & ~15);
   const uint32_t sm0 = smem_u32(sm);
   const int sub_b = stage_b / kSub;
-  const int n = c.nmain + c.next;
-  for (int i0 = 0; i0 < n; i0 += kSub) {
+  const int n = c.ie;
+  for (int i0 = c.ib; i0 < n; i0 += kSub) {
     const bool ok = !*abort_flag && mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status, a.wait_ns) &&
                     mbar_wait_fast(afull + 8 * ps.ab.idx, ps.ab.ph, a.status, a.wait_ns);
     if (!__all_sync(0xffffffffu, ok)) {
@@ -264,8 +271,8 @@ __device__ void unpack(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, ui
   const int RS2 = d.rank / 2;  // compensator column pairs
   const int R = c.rb * kRows + row;
   const int sub_b = stage_b / kSub;
-  const int n = c.nmain + c.next;
-  for (int i0 = 0; i0 < n; i0 += kSub) {
+  const int n = c.ie;
+  for (int i0 = c.ib; i0 < n; i0 += kSub) {
     // warp-uniform waits: every lane reaches the .sync.aligned TMEM stores
     const bool ok = !*abort_flag && mbar_wait_fast(full + 8 * ps.st.idx, ps.st.ph, a.status, a.wait_ns) &&
                     mbar_wait_fast(aempty + 8 * ps.ab.idx, ps.ab.ph ^ 1u, a.status, a.wait_ns);
@@ -349,21 +356,24 @@ __device__ void epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
   const int row = threadIdx.x - 32 * kDqWarps;  // 0..127 = TMEM lane
   const uint32_t lane_base = (uint32_t)(row & ~31) << 16;
   const int R = c.rb * kRows + row;
+  // the part's groups: main chunks [ib, min(ie, nmain)), then the compensator if ie > nmain
+  const int me = min(c.ie, c.nmain);
   int nmain_groups = 0;
-  if constexpr (FMT == FMT_INT) nmain_groups = c.nmain / (GROUP / 64);
-  else nmain_groups = c.nmain > 0 ? 1 : 0;
-  const int g0 = (FMT == FMT_INT) ? c.kc0 / (GROUP / 64) : 0;
+  if constexpr (FMT == FMT_INT) nmain_groups = max(0, me - c.ib) / (GROUP / 64);
+  else nmain_groups = me > c.ib ? 1 : 0;
+  const int ncomp = c.ie > c.nmain ? 1 : 0;
+  const int g0 = (FMT == FMT_INT) ? (c.kc0 + c.ib) / (GROUP / 64) : 0;
   float y[NTOK];
 #pragma unroll
   for (int t = 0; t < NTOK; ++t) y[t] = 0.f;
   // the row's group scales, loaded kPre groups ahead of their use (they come
   // from L2: the producer's copies of the same words went through it)
-  constexpr int kPre = 4;
+  constexpr int kPre = 3;
   uint32_t pre[kPre];
 #pragma unroll
   for (int q = 0; q < kPre; ++q)
     pre[q] = (FMT == FMT_INT && q < nmain_groups) ? d.sz[(long long)(g0 + q) * a.M + R] : 0x3C00u;
-  for (int gi = 0; gi < nmain_groups + c.next; ++gi) {
+  for (int gi = 0; gi < nmain_groups + ncomp; ++gi) {
     float s = 1.f;
     if (FMT == FMT_INT && gi < nmain_groups) s = __half2float(__ushort_as_half((uint16_t)(pre[0] & 0xFFFFu)));
 #pragma unroll
@@ -382,6 +392,42 @@ __device__ void epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
     __syncwarp();
     if (lane == 0) mbar_arrive(accfree + 8 * ps.acc.idx);
     ps.acc.next(kAcc);
+  }
+  // ---- a tile split between two CTAs: the tail part's sums go to the head's
+  // CTA, which adds them before the outputs (fixed order: head + tail)
+  if (c.tail_write) {
+    float* part = a.sk_part + (long long)blockIdx.x * (kRows * 32) + row * NTOK;
+#pragma unroll
+    for (int t = 0; t < NTOK; t += 4) *reinterpret_cast<float4*>(part + t) = make_float4(y[t], y[t + 1], y[t + 2], y[t + 3]);
+    __threadfence();
+    named_bar_sync(1, 32 * kEpWarps);
+    if (row == 0) st_release_gpu_u32(a.sk_flag + blockIdx.x, a.sk_epoch);
+    return;
+  }
+  if (c.head_wait) {
+    const unsigned* flag = a.sk_flag + blockIdx.x + 1;
+    if (row == 0) {
+      const unsigned long long t0 = clock_cycles();
+      while (ld_acquire_gpu_u32(flag) != a.sk_epoch) {
+        if ((clock_cycles() - t0) / 2 >= a.wait_ns) {
+          atomicOr(a.status, ST_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        __nanosleep(32);
+      }
+    }
+    named_bar_sync(1, 32 * kEpWarps);
+    if (*abort_flag) return;
+    const float* other = a.sk_part + (long long)(blockIdx.x + 1) * (kRows * 32) + row * NTOK;  // the next CTA's slot
+#pragma unroll
+    for (int t = 0; t < NTOK; t += 4) {
+      const float4 o = __ldcg(reinterpret_cast<const float4*>(other + t));
+      y[t] += o.x;
+      y[t + 1] += o.y;
+      y[t + 2] += o.z;
+      y[t + 3] += o.w;
+    }
   }
   // ---- outputs: tokens tok0 + t
   const int nt = min(NTOK, c.n_e - c.tok0);
@@ -408,21 +454,8 @@ __device__ void epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
 }
 
 template <int NTOK, int FMT, int BITS, int GROUP>
-__device__ void decode_tile(const DecodeArgs& a, const BlockDesc& d, const Ctx& c0, uint8_t* sm, int stage_b,
+__device__ void decode_tile(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, uint8_t* sm, int stage_b,
                             int cbytes, uint32_t bars, uint32_t tmem, Pos& ps, volatile int* ab) {
-  // group-aligned K range of this split
-  Ctx c = c0;
-  const int KC = a.K / 64;
-  if constexpr (FMT == FMT_INT) {
-    constexpr int cpg = GROUP / 64;
-    const int NG = KC / cpg;
-    const int g0 = (int)((long long)NG * c.ks / a.KS), g1 = (int)((long long)NG * (c.ks + 1) / a.KS);
-    c.kc0 = g0 * cpg;
-    c.nmain = (g1 - g0) * cpg;
-  } else {
-    c.kc0 = (int)((long long)KC * c.ks / a.KS);
-    c.nmain = (int)((long long)KC * (c.ks + 1) / a.KS) - c.kc0;
-  }
   const int warp = threadIdx.x >> 5;
   if (warp < kDqWarps) {
     unpack<NTOK, FMT, BITS, GROUP>(a, d, c, sm, stage_b, cbytes, bars, tmem, ps, ab);
@@ -516,13 +549,27 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // each CTA takes a contiguous, balanced range of the tiles (passes of one
-  // row block and K split adjacent: they reuse its weights from L2)
+  // Each CTA takes a contiguous range of the tiles (passes of one row block
+  // and K split adjacent: they reuse its weights from L2). With at least one
+  // tile per CTA the ranges are cut at step granularity: CTA b covers
+  // [total b / G, total (b + 1) / G) in tile units, and a fractional edge
+  // splits that tile at step ceil(r n / G) (r = the remainder, n = the tile's
+  // steps), which the two CTAs sharing the tile compute alike. The CTA
+  // holding the tile's tail runs it first and hands its sums over; the CTA
+  // holding the head runs it last and adds them. With fewer tiles than CTAs,
+  // whole tiles only.
   const int total = s_pre[nact] * per;
   volatile int* ab = &abort_flag;
   dk::Pos ps;
-  const int tile_end = (int)((long long)total * (blockIdx.x + 1) / gridDim.x);
-  for (int tile = (int)((long long)total * blockIdx.x / gridDim.x); tile < tile_end && !*ab; ++tile) {
+  const int G = gridDim.x;
+  // (only where whole tiles would leave the busiest CTA over 10% above the mean)
+  const bool split = a.sk_part != nullptr && total >= G && (long long)((total + G - 1) / G) * G * 10 > 11LL * total;
+  const long long P0 = (long long)total * blockIdx.x, P1 = P0 + total;
+  const int t_first = (int)(P0 / G), t_last = (int)(P1 / G);
+  const int r_first = split ? (int)(P0 % G) : 0, r_last = split ? (int)(P1 % G) : 0;
+  const int t_stop = r_last > 0 ? t_last + 1 : t_last;
+  const int KC = a.K / 64;
+  for (int tile = t_first; tile < t_stop && !*ab; ++tile) {
     int lo = 0, hi = nact - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -541,7 +588,25 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
     c.ks = (local / np) % a.KS;
     const BlockDesc& d = a.experts[e].blk[a.block];
     c.next = (c.ks == 0 && d.rank > 0) ? 1 : 0;
-    c.kc0 = c.nmain = 0;
+    // the K range of split ks (group-aligned for integer codes)
+    if (d.fmt == FMT_INT) {
+      const int cpg = max(1, d.group / 64), NG = KC / cpg;
+      const int g0 = (int)((long long)NG * c.ks / a.KS), g1 = (int)((long long)NG * (c.ks + 1) / a.KS);
+      c.kc0 = g0 * cpg;
+      c.nmain = (g1 - g0) * cpg;
+    } else {
+      c.kc0 = (int)((long long)KC * c.ks / a.KS);
+      c.nmain = (int)((long long)KC * (c.ks + 1) / a.KS) - c.kc0;
+    }
+    const int nch = c.nmain + c.next;
+    const int nsteps = (nch + dk::kSub - 1) / dk::kSub;
+    const int sb = (tile == t_first && r_first > 0) ? (int)(((long long)r_first * nsteps + G - 1) / G) : 0;
+    const int se = (tile == t_last && r_last > 0) ? (int)(((long long)r_last * nsteps + G - 1) / G) : nsteps;
+    c.ib = sb * dk::kSub;
+    c.ie = min(se * dk::kSub, nch);
+    c.tail_write = sb > 0 ? 1 : 0;
+    c.head_wait = se < nsteps ? 1 : 0;
+    if (c.ib >= c.ie) continue;  // nothing of this tile falls to this CTA
     bool ran = true;
     if (d.fmt == FMT_INT) {
       switch (d.bits * 1000 + d.group) {

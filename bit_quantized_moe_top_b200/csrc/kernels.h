@@ -82,6 +82,11 @@ struct DecodeArgs {
   int nstages;                // shared-memory stages of the ring (set by the launcher)
   unsigned long long wait_ns; // limit of the hand-off waits between roles
   unsigned* status;
+  // tiles split between two CTAs (null: whole tiles only): per CTA 128 x 32
+  // fp32 partial sums and a flag set to sk_epoch once they are written
+  float* sk_part;
+  unsigned* sk_flag;
+  unsigned sk_epoch;          // nonzero, different for every launch of the layer
 };
 
 // Per-chunk correction columns of the activations for the integer-code

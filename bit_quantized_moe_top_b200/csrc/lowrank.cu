@@ -69,19 +69,32 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
     // rows past the expert's count read the padded slack rows of the buffer
     const long long ra = prow0 + rbase + g, rb = ra + 8;  // rows of a0a1/a4a5 and a2a3/a6a7
     const long long ldw = a.Kpad >> 1;                    // row pitch in u32
-#pragma unroll 4
-    for (int S = s0; S < s1; ++S) {
-      uint32_t av[4];
-      av[0] = act32[ra * ldw + 8 * S + c];
-      av[1] = act32[rb * ldw + 8 * S + c];
-      av[2] = act32[ra * ldw + 8 * S + c + 4];
-      av[3] = act32[rb * ldw + 8 * S + c + 4];
+    // four K steps per round: every load of the round is issued before its
+    // MMAs, so a warp keeps ~1.5 KiB in flight instead of one step's worth
+    constexpr int kB = 4;
+    for (int S0 = s0; S0 < s1; S0 += kB) {
+      uint32_t av[kB][4];
+      uint4 v[kB][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (i < RF) {
-          const uint4 v = afrag[((long long)i * S16 + S) * 32 + lane];
-          mma_16816(acc[2 * i], av, v.x, v.z);
-          mma_16816(acc[2 * i + 1], av, v.y, v.w);
+      for (int q = 0; q < kB; ++q) {
+        const int S = min(S0 + q, s1 - 1);  // (a clamped step is loaded and not used)
+        av[q][0] = act32[ra * ldw + 8 * S + c];
+        av[q][1] = act32[rb * ldw + 8 * S + c];
+        av[q][2] = act32[ra * ldw + 8 * S + c + 4];
+        av[q][3] = act32[rb * ldw + 8 * S + c + 4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (i < RF) v[q][i] = afrag[((long long)i * S16 + S) * 32 + lane];
+      }
+#pragma unroll
+      for (int q = 0; q < kB; ++q) {
+        if (S0 + q >= s1) break;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (i < RF) {
+            mma_16816(acc[2 * i], av[q], v[q][i].x, v[q][i].z);
+            mma_16816(acc[2 * i + 1], av[q], v[q][i].y, v[q][i].w);
+          }
         }
       }
     }
@@ -126,9 +139,16 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
   __threadfence();
   for (int idx = threadIdx.x; idx < nrows * r; idx += blockDim.x) {
     const int n = tile * kLrRows + idx / r, j = idx % r;
+    const float* pp = a.part + (long long)(prow0 + n) * kMaxRank + j;
+    // the partials in split order, eight loads in flight at a time
     float sum = 0.f;
-    for (int k2 = 0; k2 < a.KS; ++k2)
-      sum += __ldcg(a.part + k2 * a.part_ks_stride + (long long)(prow0 + n) * kMaxRank + j);
+    for (int k0 = 0; k0 < a.KS; k0 += 8) {
+      float pv[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) pv[q] = k0 + q < a.KS ? __ldcg(pp + (long long)(k0 + q) * a.part_ks_stride) : 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) sum += pv[q];
+    }
     store_u(n, j, sum);
   }
   if (threadIdx.x == 0) *sem = 0;

@@ -102,6 +102,8 @@ struct moe_layer {
   } tq[2];
   DevBuf block_counts, block_base, pblock_base, sem, status;
   DevBuf xact, zact, obuf, part, corr_x, corr_z;
+  DevBuf sk_part, sk_flag;  // decode GEMM tiles split between two CTAs: partial sums, flags
+  unsigned sk_epoch = 0;
   int ldc_x = 0, ldc_z = 0;  // correction columns per row: 16 per group of 64 (the smallest group)
   DevBuf hx, hl, hy;  // device buffers for forward_host
   CUtensorMap tmap_x, tmap_z;    // activation buffers, 128-row boxes (prefill GEMMs)
@@ -249,7 +251,7 @@ void moe_layer_destroy(moe_layer_t* L) {
   DevBuf* bufs[] = {&L->d_experts, &L->idx, &L->w, &L->counts, &L->offsets, &L->poffsets, &L->active,
                     &L->n_active, &L->ticket, &L->flag, &L->perm, &L->inv_pos, &L->pinv, &L->pslot, &L->ptok, &L->block_counts,
                     &L->block_base, &L->pblock_base, &L->sem, &L->status, &L->xact, &L->zact, &L->obuf,
-                    &L->part, &L->corr_x, &L->corr_z, &L->hx, &L->hl, &L->hy};
+                    &L->part, &L->corr_x, &L->corr_z, &L->hx, &L->hl, &L->hy, &L->sk_part, &L->sk_flag};
   for (DevBuf* b : bufs) dfree(*b);
   for (cudaEvent_t ev : L->events) cudaEventDestroy(ev);
   if (L->fwd_done) cudaEventDestroy(L->fwd_done);
@@ -337,6 +339,8 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   A(L->part, sizeof(float) * (size_t)L->kslr_max * L->rows_pad_max * kMaxRank);
   L->ldc_x = 16 * (K / 64);
   L->ldc_z = 16 * (N / 64);
+  A(L->sk_part, sizeof(float) * (size_t)decode_ctas() * decode_rows_per_cta() * 32);
+  A(L->sk_flag, sizeof(unsigned) * (size_t)decode_ctas());
   A(L->corr_x, sizeof(__half) * (size_t)L->rows_pad_max * L->ldc_x);
   A(L->corr_z, sizeof(__half) * (size_t)L->rows_pad_max * L->ldc_z);
   A(L->hx, sizeof(__nv_bfloat16) * (size_t)max_tokens * K);
@@ -348,7 +352,7 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   }
   cudaError_t ce = cudaSuccess;
   DevBuf* zero[] = {&L->ticket, &L->flag, &L->sem, &L->status, &L->xact, &L->zact, &L->n_active, &L->counts, &L->corr_x,
-                    &L->corr_z};
+                    &L->corr_z, &L->sk_flag};
   for (DevBuf* b : zero)
     if (ce == cudaSuccess) ce = cudaMemset(b->p, 0, b->n);
   if (ce == cudaSuccess)
@@ -832,6 +836,13 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
   const int E = L->E, K = L->K, N = L->N;
   int maxbits[2] = {0, 0}, rmax = 0;
   bool any_int[2] = {false, false};
+  bool uniform[2] = {true, true};
+  for (int e = 1; e < E; ++e)
+    for (int b = 0; b < 2; ++b) {
+      const BlockDesc& x = L->hdesc[e].blk[b];
+      const BlockDesc& y = L->hdesc[0].blk[b];
+      uniform[b] = uniform[b] && x.fmt == y.fmt && x.bits == y.bits && x.group == y.group && x.rank == y.rank;
+    }
   for (int e = 0; e < E; ++e) {
     for (int b = 0; b < 2; ++b) {
       const int bb = L->hdesc[e].blk[b].bits;
@@ -906,7 +917,9 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     ca.status = ra.status;
     return ca;
   };
-  const int corr_rows = (int)std::min<long long>(T, rows);
+  // correction-sum CTAs are sized for twice an expert's mean share of the
+  // routed rows (they loop over their items when an expert holds more)
+  const int corr_rows = (int)std::min<long long>(T, 2 * ((rows + grid_y - 1) / grid_y));
   // correction-sum CTAs per expert slot, at most about 2048 over all slots:
   // sized for one expert taking every token, the count grows with E while
   // most slots hold a few rows (the CTAs loop over their items)
@@ -1051,6 +1064,13 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
       da.rows = rows;
       da.wait_ns = L->wait_ns;
       da.status = ra.status;
+      // tiles split between CTAs only where every expert's block has the same
+      // format, bits, group and rank (steps of one cost); with mixed blocks
+      // the split measured slower than whole tiles
+      da.sk_part = uniform[block] ? static_cast<float*>(L->sk_part.p) : nullptr;
+      da.sk_flag = static_cast<unsigned*>(L->sk_flag.p);
+      if (++L->sk_epoch == 0) L->sk_epoch = 1;
+      da.sk_epoch = L->sk_epoch;
       prof_mark(L, st, block == 0 ? "decode_gemm_w1_swiglu" : "decode_gemm_w2");
       ce = launch_decode_gemm(da, ntok, maxbits[block], grid_y, st, &launches);
     };
@@ -1060,18 +1080,24 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N, corr2);
     tileq(1, corr2);
     // split the down projection's K (fixed-order sum of the partials in the
-    // combine) where that shortens the busiest CTA's share: each CTA takes
-    // ceil(units / CTAs) units of 128 rows x (N / 64 / KS) chunks, plus
-    // about 3 chunks of pipeline fill per unit; splits at least 256 columns
-    // wide, and at least one split (N = 128 gives one)
+    // combine); splits at least 256 columns wide, and at least one split.
+    // With tiles split between CTAs, only until there are at least as many
+    // tiles as CTAs (from there the kernel balances the shares at step
+    // granularity); otherwise where that shortens the busiest CTA's share:
+    // each CTA takes ceil(units / CTAs) units of 128 rows x (N / 64 / KS)
+    // chunks, plus about 3 chunks of pipeline fill per unit
     const long long units1 = (long long)(K / decode_rows_per_cta()) * grid_y;
     const int ctas = decode_ctas(), kmax = std::max(1, std::min(L->ks2_max, N / 256));
-    double best = 0.0;
-    for (int ks = 1; ks <= kmax; ++ks) {
-      const double t = (double)((units1 * ks + ctas - 1) / ctas) * ((double)N / 64.0 / ks + 3.0);
-      if (ks == 1 || t < best * 0.98) {
-        best = t;
-        ks2 = ks;
+    if (uniform[1]) {
+      while (units1 * ks2 < ctas && ks2 < kmax) ++ks2;
+    } else {
+      double best = 0.0;
+      for (int ks = 1; ks <= kmax; ++ks) {
+        const double t = (double)((units1 * ks + ctas - 1) / ctas) * ((double)N / 64.0 / ks + 3.0);
+        if (ks == 1 || t < best * 0.98) {
+          best = t;
+          ks2 = ks;
+        }
       }
     }
     if (rows > 1024) ks2 = 1;

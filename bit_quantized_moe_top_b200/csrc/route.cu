@@ -361,10 +361,11 @@ cudaError_t launch_route_topk(const RouteArgs& a, cudaStream_t st, int* launches
 }
 
 cudaError_t launch_route_fused(const RouteArgs& a, int num_sms, cudaStream_t st, int* launches) {
-  // every CTA must be resident at once: at most one per SM; the first kernel
-  // of a forward, serialized after whatever the stream ran before
+  // every CTA must be resident at once: at most one per SM. Programmatic
+  // launch: the CTAs may be placed while the stream's previous kernel (the
+  // last forward's combine) drains; they write nothing before pdl_wait()
   const int grid = std::max(1, std::min(num_sms, a.nb * a.gs));
-  const cudaError_t err = launch_kernel(route_fused_kernel, dim3(grid), dim3(kRouteThreads), 0, st, false, a);
+  const cudaError_t err = launch_kernel(route_fused_kernel, dim3(grid), dim3(kRouteThreads), 0, st, true, a);
   if (launches) ++*launches;
   return err;
 }
