@@ -17,6 +17,39 @@ constexpr int kLrWarps = 4;    // each warp: 16 routed rows (tokens) x all r col
 constexpr int kLrRows = 16 * kLrWarps;
 constexpr int kCombineThreads = 128;
 
+// K steps [s0, s1) of one warp's 16 rows x 16 RF columns: a few steps per
+// round with every load of the round issued before its MMAs (fewer steps per
+// round at larger ranks, to keep the registers in bounds)
+template <int RF>
+__device__ __forceinline__ void lr_kloop(const uint32_t* act32, const uint4* afrag, long long ra, long long ldw, int S16,
+                                         int s0, int s1, int c, int lane, float (&acc)[8][4]) {
+  constexpr int kB = RF <= 2 ? 4 : 2;
+  const long long rb = ra + 8;
+  for (int S0 = s0; S0 < s1; S0 += kB) {
+    uint32_t av[kB][4];
+    uint4 v[kB][RF];
+#pragma unroll
+    for (int q = 0; q < kB; ++q) {
+      const int S = min(S0 + q, s1 - 1);  // (a clamped step is loaded and not used)
+      av[q][0] = act32[ra * ldw + 8 * S + c];
+      av[q][1] = act32[rb * ldw + 8 * S + c];
+      av[q][2] = act32[ra * ldw + 8 * S + c + 4];
+      av[q][3] = act32[rb * ldw + 8 * S + c + 4];
+#pragma unroll
+      for (int i = 0; i < RF; ++i) v[q][i] = afrag[((long long)i * S16 + S) * 32 + lane];
+    }
+#pragma unroll
+    for (int q = 0; q < kB; ++q) {
+      if (S0 + q >= s1) break;
+#pragma unroll
+      for (int i = 0; i < RF; ++i) {
+        mma_16816(acc[2 * i], av[q], v[q][i].x, v[q][i].z);
+        mma_16816(acc[2 * i + 1], av[q], v[q][i].y, v[q][i].w);
+      }
+    }
+  }
+}
+
 // grid: (KS x token tiles of 64 rows, expert slots). Tokens are the MMA's M:
 // a warp's A fragments are 16 routed rows of the activations, its B
 // fragments come straight from the factor's dense fragments (two n8 tiles per
@@ -26,7 +59,7 @@ constexpr int kCombineThreads = 128;
 // order. With KS == 1 the result is written directly; otherwise each CTA
 // writes an fp32 partial and the last CTA of a (expert, token tile) sums the
 // partials in a fixed order.
-__global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
+__global__ void __launch_bounds__(kLrWarps * 32, 7) lowrank_kernel(LowrankArgs a) {
   __shared__ int is_last;
   __shared__ float red[kLrWarps][16][kMaxRank + 1];
   pdl_wait();
@@ -67,36 +100,12 @@ __global__ void __launch_bounds__(kLrWarps * 32) lowrank_kernel(LowrankArgs a) {
     for (int q = 0; q < 4; ++q) acc[t][q] = 0.f;
   if (rbase < n_e) {
     // rows past the expert's count read the padded slack rows of the buffer
-    const long long ra = prow0 + rbase + g, rb = ra + 8;  // rows of a0a1/a4a5 and a2a3/a6a7
-    const long long ldw = a.Kpad >> 1;                    // row pitch in u32
-    // four K steps per round: every load of the round is issued before its
-    // MMAs, so a warp keeps ~1.5 KiB in flight instead of one step's worth
-    constexpr int kB = 4;
-    for (int S0 = s0; S0 < s1; S0 += kB) {
-      uint32_t av[kB][4];
-      uint4 v[kB][4];
-#pragma unroll
-      for (int q = 0; q < kB; ++q) {
-        const int S = min(S0 + q, s1 - 1);  // (a clamped step is loaded and not used)
-        av[q][0] = act32[ra * ldw + 8 * S + c];
-        av[q][1] = act32[rb * ldw + 8 * S + c];
-        av[q][2] = act32[ra * ldw + 8 * S + c + 4];
-        av[q][3] = act32[rb * ldw + 8 * S + c + 4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (i < RF) v[q][i] = afrag[((long long)i * S16 + S) * 32 + lane];
-      }
-#pragma unroll
-      for (int q = 0; q < kB; ++q) {
-        if (S0 + q >= s1) break;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if (i < RF) {
-            mma_16816(acc[2 * i], av[q], v[q][i].x, v[q][i].z);
-            mma_16816(acc[2 * i + 1], av[q], v[q][i].y, v[q][i].w);
-          }
-        }
-      }
+    const long long ra = prow0 + rbase + g;  // row of a0a1/a4a5 (a2a3/a6a7: 8 rows later)
+    switch (RF) {
+      case 1: lr_kloop<1>(act32, afrag, ra, a.Kpad >> 1, S16, s0, s1, c, lane, acc); break;
+      case 2: lr_kloop<2>(act32, afrag, ra, a.Kpad >> 1, S16, s0, s1, c, lane, acc); break;
+      case 3: lr_kloop<3>(act32, afrag, ra, a.Kpad >> 1, S16, s0, s1, c, lane, acc); break;
+      default: lr_kloop<4>(act32, afrag, ra, a.Kpad >> 1, S16, s0, s1, c, lane, acc); break;
     }
   }
   // acc[t][q]: row g + 8*(q>>1) of the sub-tile, column j = 8t + 2c + (q&1)

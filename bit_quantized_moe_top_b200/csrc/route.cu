@@ -242,49 +242,64 @@ __device__ void permute_item(const RouteArgs& a, int b, int ks, unsigned* mask, 
   const int nch = c1 - c0;
   const int total = rows * nch * 8;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int base = warp * 32; base < total; base += blockDim.x) {
-    const int it = base + lane;
-    const bool valid = it < total;  // 8-lane groups are all valid or all not (total is a multiple of 8)
-    const int q8 = it & 7, pc = it >> 3;
-    const int i = valid ? pc / nch : 0, c = c0 + (valid ? pc % nch : 0);
-    const int t = t0 + i / a.k;
-    const long long prow = prow_s[i];
-    float xs = 0.f, xp = 0.f;
-    if (valid) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(a.X + (long long)t * a.K + 64 * c + 8 * q8);
-      const __nv_bfloat162* bv = reinterpret_cast<const __nv_bfloat162*>(&raw);
-      uint32_t v[4];
+  // four rounds' loads are issued before their stores: a CTA (one per SM)
+  // then keeps 16 KiB of the gather in flight
+  constexpr int kU = 4;
+  for (int base0 = warp * 32; base0 < total; base0 += kU * blockDim.x) {
+    uint4 raw[kU];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) v[q] = pack_half2(__bfloat162float(bv[q].x), __bfloat162float(bv[q].y));
-      *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(a.act) + prow * a.Kpad + 64 * c + 8 * q8) =
-          make_uint4(v[0], v[1], v[2], v[3]);
-      if (a.corr) {
-        const BlockDesc& d = a.experts[exp_s[i]].blk[0];
-        if (d.fmt == FMT_INT) {
+    for (int u = 0; u < kU; ++u) {
+      const int it = base0 + u * blockDim.x + lane;
+      if (it < total) {
+        const int pc = it >> 3;
+        const int i = pc / nch, c = c0 + pc % nch;
+        raw[u] = *reinterpret_cast<const uint4*>(a.X + (long long)(t0 + i / a.k) * a.K + 64 * c + 8 * (it & 7));
+      }
+    }
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const __half2 h = *reinterpret_cast<const __half2*>(&v[q]);
-            const float x0 = __low2float(h), x1 = __high2float(h);
-            xs += x0 + x1;
-            xp = fmaf(int_pfac(d.bits, 8 * q8 + 2 * q), x0, xp);
-            xp = fmaf(int_pfac(d.bits, 8 * q8 + 2 * q + 1), x1, xp);
+    for (int u = 0; u < kU; ++u) {
+      const int it = base0 + u * blockDim.x + lane;
+      const bool valid = it < total;  // 8-lane groups are all valid or all not (total is a multiple of 8)
+      const int q8 = it & 7, pc = it >> 3;
+      const int i = valid ? pc / nch : 0, c = c0 + (valid ? pc % nch : 0);
+      const long long prow = prow_s[i];
+      float xs = 0.f, xp = 0.f;
+      if (valid) {
+        const __nv_bfloat162* bv = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+        uint32_t v[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[q] = pack_half2(__bfloat162float(bv[q].x), __bfloat162float(bv[q].y));
+        *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(a.act) + prow * a.Kpad + 64 * c + 8 * q8) =
+            make_uint4(v[0], v[1], v[2], v[3]);
+        if (a.corr) {
+          const BlockDesc& d = a.experts[exp_s[i]].blk[0];
+          if (d.fmt == FMT_INT) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const __half2 h = *reinterpret_cast<const __half2*>(&v[q]);
+              const float x0 = __low2float(h), x1 = __high2float(h);
+              xs += x0 + x1;
+              xp = fmaf(int_pfac(d.bits, 8 * q8 + 2 * q), x0, xp);
+              xp = fmaf(int_pfac(d.bits, 8 * q8 + 2 * q + 1), x1, xp);
+            }
           }
         }
       }
-    }
-    if (a.corr) {
+      if (a.corr) {
+        // warp-uniform: every lane takes part in the shuffles
 #pragma unroll
-      for (int o = 1; o < 8; o <<= 1) {
-        xs += __shfl_xor_sync(0xffffffffu, xs, o);
-        xp += __shfl_xor_sync(0xffffffffu, xp, o);
-      }
-      if (valid && q8 == 0) {
-        const BlockDesc& d = a.experts[exp_s[i]].blk[0];
-        if (d.fmt == FMT_INT) {
-          const int cpg = d.group / 64;
-          const int g = c / cpg, cc = c % cpg;
-          *reinterpret_cast<uint2*>(a.corr + prow * a.ldc + 16 * g + 4 * cc) =
-              make_uint2(corr_pair(xp, a.status), corr_pair(xs, a.status));
+        for (int o = 1; o < 8; o <<= 1) {
+          xs += __shfl_xor_sync(0xffffffffu, xs, o);
+          xp += __shfl_xor_sync(0xffffffffu, xp, o);
+        }
+        if (valid && q8 == 0) {
+          const BlockDesc& d = a.experts[exp_s[i]].blk[0];
+          if (d.fmt == FMT_INT) {
+            const int cpg = d.group / 64;
+            const int g = c / cpg, cc = c % cpg;
+            *reinterpret_cast<uint2*>(a.corr + prow * a.ldc + 16 * g + 4 * cc) =
+                make_uint2(corr_pair(xp, a.status), corr_pair(xs, a.status));
+          }
         }
       }
     }
