@@ -242,9 +242,9 @@ __device__ void permute_item(const RouteArgs& a, int b, int ks, unsigned* mask, 
   const int nch = c1 - c0;
   const int total = rows * nch * 8;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  // four rounds' loads are issued before their stores: a CTA (one per SM)
-  // then keeps 16 KiB of the gather in flight
-  constexpr int kU = 4;
+  // eight rounds' loads are issued before their stores: a CTA (one per SM)
+  // then keeps 32 KiB of the gather in flight
+  constexpr int kU = 8;
   for (int base0 = warp * 32; base0 < total; base0 += kU * blockDim.x) {
     uint4 raw[kU];
 #pragma unroll
