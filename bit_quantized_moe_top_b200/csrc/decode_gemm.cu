@@ -563,13 +563,18 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
   dk::Pos ps;
   const int G = gridDim.x;
   // (only where whole tiles would leave the busiest CTA over 10% above the mean)
-  const bool split = a.sk_part != nullptr && total >= G && (long long)((total + G - 1) / G) * G * 10 > 11LL * total;
+  const bool split = !a.mixed && a.sk_part != nullptr && total >= G &&
+                     (long long)((total + G - 1) / G) * G * 10 > 11LL * total;
   const long long P0 = (long long)total * blockIdx.x, P1 = P0 + total;
   const int t_first = (int)(P0 / G), t_last = (int)(P1 / G);
   const int r_first = split ? (int)(P0 % G) : 0, r_last = split ? (int)(P1 % G) : 0;
   const int t_stop = r_last > 0 ? t_last + 1 : t_last;
   const int KC = a.K / 64;
-  for (int tile = t_first; tile < t_stop && !*ab; ++tile) {
+  // blocks that differ between experts (bits, format, group, rank) take the
+  // tiles round-robin instead: their costs differ, and contiguous ranges
+  // would pile one expert's dear tiles onto a few CTAs
+  const bool rr = a.mixed != 0;
+  for (int tile = rr ? (int)blockIdx.x : t_first; tile < (rr ? total : t_stop) && !*ab; tile += rr ? G : 1) {
     int lo = 0, hi = nact - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;

@@ -87,6 +87,7 @@ struct DecodeArgs {
   float* sk_part;
   unsigned* sk_flag;
   unsigned sk_epoch;          // nonzero, different for every launch of the layer
+  int mixed;                  // the experts' blocks differ (bits, format, group or rank): tiles dealt round-robin
 };
 
 // Per-chunk correction columns of the activations for the integer-code

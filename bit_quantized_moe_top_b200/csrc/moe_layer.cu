@@ -1068,6 +1068,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
       // format, bits, group and rank (steps of one cost); with mixed blocks
       // the split measured slower than whole tiles
       da.sk_part = uniform[block] ? static_cast<float*>(L->sk_part.p) : nullptr;
+      da.mixed = uniform[block] ? 0 : 1;
       da.sk_flag = static_cast<unsigned*>(L->sk_flag.p);
       if (++L->sk_epoch == 0) L->sk_epoch = 1;
       da.sk_epoch = L->sk_epoch;
