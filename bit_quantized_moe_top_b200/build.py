@@ -15,7 +15,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 
 SOURCES = ["moe_layer.cu", "route.cu", "relayout.cu", "decode_gemm.cu", "lowrank.cu", "noalloc.cu", "prefill_gemm.cu",
            "planner.cpp", "tileq.cu"]
-HEADERS = ["common.cuh", "decode_frag.cuh", "tc.cuh", "corr.cuh", "kernels.h"]
+HEADERS = ["common.cuh", "decode_frag.cuh", "tc.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include")]

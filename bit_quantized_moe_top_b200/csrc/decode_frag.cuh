@@ -8,12 +8,10 @@
 // Integer codes become fp16 through the exponent-bias trick: a b-bit field
 // q OR-ed into the mantissa of a power of two P whose mantissa unit at the
 // field's position is 1 reads as P + q exactly. The "raw" value P_i + q is
-// what the tensor-core path multiplies (the P_i term is removed per group
-// through extra K columns); the dequantising path subtracts P_i exactly and
-// applies one fp16 FMA with the group's scale and -z*s. P_i depends only on
-// the pair index i (both halves of a word use the same bit position), so
-// each format has a fixed table of P_i (int_magic) and of P_i / 1024
-// (int_pfac, used to precompute the correction sums).
+// where dequantising starts: one fp16 subtraction removes P_i exactly and one
+// fp16 FMA applies the group's scale and -z*s. P_i depends only on the pair
+// index i (both halves of a word use the same bit position), so each format
+// has a fixed table of P_i (int_magic).
 //
 // Field positions per format (per 16-bit half of a word; P = 2^(10 - pos)):
 //   INT4: word s (0..3) holds pairs 4s..4s+3: nibbles 0 and 1 of each byte
@@ -40,19 +38,6 @@ __host__ __device__ __forceinline__ uint32_t int_magic(int i) {
   if (i == 15) return 0x48004800u;
   const int f = i % 5;
   return f == 0 ? 0x64006400u : (f & 1) ? 0x58005800u : 0x4C004C00u;
-}
-
-// P / 1024 of the code at position kk (0..63) of a chunk
-__host__ __device__ __forceinline__ float int_pfac(int bits, int kk) {
-  const int i = (kk >> 1) & 15;
-  if (bits == 4) return (i & 1) ? 0.0625f : 1.f;
-  if (bits == 2) {
-    const int j = i & 3;
-    return j == 0 ? 1.f : j == 1 ? 0.25f : j == 2 ? 0.0625f : 0.015625f;
-  }
-  if (i == 15) return 0.0078125f;
-  const int f = i % 5;
-  return f == 0 ? 1.f : (f & 1) ? 0.125f : 0.015625f;
 }
 
 // number of 32-bit code words per half chunk of one row

@@ -7,36 +7,29 @@
 // TMEM lane) and a group-aligned range of 64-wide K chunks; CTAs are
 // persistent and walk the (expert, row block, K split, token pass) tiles.
 //   warp 8     producer: per chunk, the 128 rows' packed codes (one contiguous
-//              block), at a group's first chunk the routed rows' correction
-//              columns and the group's scale/zero pairs, and the expert's
-//              routed activation rows (TMA 2-D boxes of 16 rows, no multicast);
+//              block), at a group's first chunk the group's scale/zero pairs,
+//              and the expert's routed activation rows (TMA 2-D boxes of 16
+//              rows, no multicast);
 //   warps 0-3  unpack: one thread per weight row turns the row's 64 codes into
-//              32 fp16 pairs in registers and stores them into a TMEM buffer
-//              (one tcgen05.st), the MMA's A operand;
+//              32 fp16 pairs of dequantised weights in registers and stores
+//              them into a TMEM buffer, the MMA's A operand;
 //   warp 9     allocates TMEM and issues tcgen05.mma kind::f16 with A from
 //              TMEM (M = 128 weight rows), B = activations from shared memory
 //              (N = tokens, 16 or 32), D in TMEM;
-//   warps 4-7  epilogue: per quantisation group, y += s * acc in fp32
-//              registers; at the end of the tile SwiGLU or fp32 output rows.
+//   warps 4-7  epilogue: the accumulator into fp32 registers; at the end of
+//              the tile SwiGLU or fp32 output rows.
 // Every hand-off is an mbarrier; a warp's work per chunk is kept to a few
 // dozen instructions (ring positions advance incrementally, waits have an
 // inlined fast path), since that instruction stream, not the tensor core,
 // sets the pace.
 //
-// Integer codes are not dequantised per weight. The A operand holds the raw
-// fp16 values P_k + q_k of the exponent-bias unpack (exact small integers
-// offset by a per-position power of two), and each quantisation group g gets
-// its own accumulator:
-//   acc_g = sum_{k in g} (P_k + q_k) x_k + 1024 (-XP_g) + z_g (-X_g)
-//         = sum_{k in g} (q_k - z_g) x_k,
-// the two extra terms being one more K = 16 MMA step per group whose A
-// columns are (1024, 1024, z_g, z_g) once per 64-wide chunk of the group and
-// whose B columns are the routed row's precomputed chunk sums
-// XP_c = sum (P_k/1024) x_k and X_c = sum x_k, each split into fp16 value +
-// fp16 remainder (XP_g, X_g are the sums of the group's chunks). The epilogue of a group is
-// y += s_g * acc_g. Per pair of weights this leaves one or two logic ops and
-// no fp16 arithmetic. Bit-plane (LUT) and dense blocks store their fp16
-// weight values as A and use one accumulator for the whole K range.
+// Integer codes are dequantised in registers: the exponent-bias unpack gives
+// the exact fp16 values P_k + q_k (a small integer offset by a per-position
+// power of two), one fp16 subtraction removes P_k exactly and one fp16 FMA
+// per pair forms (q - z) s with the group's (s, -z s). Every format then
+// stores fp16 weights as A, and one accumulator covers the tile's whole K
+// range (this measured faster than per-group accumulators of raw codes with a
+// correction MMA per group: fewer MMAs, no per-group accumulator hand-off).
 //
 // The rank-r compensator is one more 64-wide stage (its own accumulator,
 // scale 1): the B factor's row values as A against the U = A x columns stored
@@ -53,7 +46,6 @@
 #include "kernels.h"
 #include "decode_frag.cuh"
 #include "tc.cuh"
-#include "corr.cuh"
 
 namespace moeq {
 namespace dk {
@@ -66,13 +58,12 @@ constexpr int kRows = 128;
 constexpr int kMaxStages = 16;  // stage ring depth: as many as about 100 KiB of shared memory hold
 constexpr int kSub = 2;         // 64-wide chunks per barrier round (step)
 constexpr int kA = 2;           // TMEM A buffers, one per step
-constexpr int kAcc = 3;         // TMEM accumulators (one per quantisation group; a step may hold two)
-constexpr int kACols = 40;      // per chunk: 32 code columns + 8 correction columns
+constexpr int kAcc = 3;         // TMEM accumulators (a tile's main K range, its compensator stage)
+constexpr int kACols = 32;      // per chunk: 32 columns of fp16 weight pairs
 constexpr int kAStep = kSub * kACols;
 constexpr int kABase = 96;      // accumulators at [0, kAcc * NTOK), A buffers at [96, 256)
 constexpr int kTmemCols = 256;
 constexpr int kActBox = 16;     // rows per TMA box
-constexpr uint32_t kOne1024 = 0x64006400u;  // fp16 pair (1024, 1024)
 static_assert(kABase + kA * kAStep <= kTmemCols, "TMEM rings exceed the allocation");
 static_assert(kAcc * 32 <= kABase, "accumulators overlap the A buffers");
 
@@ -83,10 +74,10 @@ constexpr int kBarFull = 0, kBarEmpty = kMaxStages, kBarAFull = 2 * kMaxStages, 
 
 // code block bytes of a 128-row x 64-k chunk at the largest bitwidth of the block's experts
 __host__ __device__ inline int code_bytes(int maxbits) { return maxbits >= 16 ? 16384 : 1024 * maxbits; }
-// one chunk's part of a stage: [act NTOK x 128 B][corr NTOK x 32 B][codes][scales 512 B];
+// one chunk's part of a stage: [act NTOK x 128 B][codes][scales 512 B];
 // a stage holds kSub of them (one step)
 __host__ __device__ inline int sub_stage_bytes(int ntok, int maxbits) {
-  const int b = ntok * 160 + code_bytes(maxbits) + 512;
+  const int b = ntok * 128 + code_bytes(maxbits) + 512;
   return (b + 1023) & ~1023;
 }
 __host__ __device__ inline int stage_bytes(int ntok, int maxbits) { return kSub * sub_stage_bytes(ntok, maxbits); }
@@ -129,10 +120,6 @@ template <int FMT, int GROUP>
 __device__ __forceinline__ void group_pos(const Ctx& c, int i, bool& first, bool& last) {
   if (i >= c.nmain) {
     first = last = true;  // compensator stage
-  } else if (FMT == FMT_INT) {
-    constexpr int cpg = GROUP / 64;
-    first = (i % cpg) == 0;
-    last = (i % cpg) == cpg - 1;
   } else {
     first = i == c.ib;
     last = i == min(c.ie, c.nmain) - 1;
@@ -166,7 +153,7 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
       const bool main = i0 + u < c.nmain;
       bytes += nbox * kActBox * 128;
       if (main) bytes += (FMT == FMT_BITPLANE ? BITS * 1024 : kBlk);
-      if (FMT == FMT_INT && main && first) bytes += nbox * kActBox * 32 + 512;
+      if (FMT == FMT_INT && main && ((c.kc0 + i0 + u) * 64) % GROUP == 0) bytes += 512;
     }
     if (elect_one()) {
       mbar_expect_tx(fb, bytes);
@@ -177,9 +164,9 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
         const uint32_t st = smem_u32(sm) + ps.st.idx * stage_b + u * sub_b;
         const bool main = i < c.nmain;
         const int kc = c.kc0 + i;
-        const bool corr = FMT == FMT_INT && main && first;
+        const bool gfirst = FMT == FMT_INT && main && ((c.kc0 + i) * 64) % GROUP == 0;
         const int kx = main ? kc * 64 : a.K + comp_col_offset(d, c.rb);
-        const uint32_t cs = st + NTOK * 160;
+        const uint32_t cs = st + NTOK * 128;
         const long long bidx = (long long)kc * RB + c.rb;
         const int g = kc * 64 / GROUP;
         for (int b = 0; b < nbox; ++b) tma_load_2d(st + b * kActBox * 128, &a.tmap_act, kx, row0 + b * kActBox, fb);
@@ -190,11 +177,7 @@ __device__ void producer(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
           } else {
             bulk_g2s(cs, codes + bidx * kBlk, kBlk, fb);
           }
-          if (corr) {
-            for (int b = 0; b < nbox; ++b)
-              tma_load_2d(st + NTOK * 128 + b * kActBox * 32, &a.tmap_corr, 16 * g, row0 + b * kActBox, fb);
-            bulk_g2s(cs + cbytes, d.sz + (long long)g * a.M + c.rb * kRows, 512, fb);
-          }
+          if (gfirst) bulk_g2s(cs + cbytes, d.sz + (long long)g * a.M + c.rb * kRows, 512, fb);
         }
       }
     }
@@ -237,14 +220,12 @@ __device__ void mma_issuer(const DecodeArgs& a, const Ctx& c, uint8_t* sm, int s
       const uint32_t bt = sm0 + ps.st.idx * stage_b + u * sub_b;
       const uint32_t acc = tmem + ps.acc.idx * NTOK;
       const uint32_t ta = tmem + kABase + ps.ab.idx * kAStep + u * kACols;
-      const bool corr = FMT == FMT_INT && i < c.nmain && first;
-      const uint64_t dact = sw128_desc(bt), dcorr = sw32_desc(bt + NTOK * 128);
+      const uint64_t dact = sw128_desc(bt);
       // the whole warp runs the loop (warp-uniform values); one lane issues
       if (elect_one()) {
-        if (corr) mma_f16_ts(acc, ta + 32, dcorr, idesc, 0);
 #pragma unroll
         for (int k16 = 0; k16 < 4; ++k16)
-          mma_f16_ts(acc, ta + k16 * 8, dact + 2 * k16, idesc, (corr || !first || k16 > 0) ? 1 : 0);
+          mma_f16_ts(acc, ta + k16 * 8, dact + 2 * k16, idesc, (!first || k16 > 0) ? 1 : 0);
         if (last) mma_commit(accfull + 8 * ps.acc.idx);
       }
       __syncwarp();
@@ -271,6 +252,7 @@ __device__ void unpack(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, ui
   const int RS2 = d.rank / 2;  // compensator column pairs
   const int R = c.rb * kRows + row;
   const int sub_b = stage_b / kSub;
+  uint32_t dq_s2 = 0u, dq_n2 = 0u;  // the current group's (s, s) and (-z s, -z s)
   const int n = c.ie;
   for (int i0 = c.ib; i0 < n; i0 += kSub) {
     // warp-uniform waits: every lane reaches the .sync.aligned TMEM stores
@@ -294,16 +276,12 @@ __device__ void unpack(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, ui
       const uint32_t ta = tmem + lane_base + kABase + ps.ab.idx * kAStep + u * kACols;
       uint32_t v[32];
       if (i < c.nmain) {
-        const uint8_t* cs = sm + ps.st.idx * stage_b + u * sub_b + NTOK * 160;
+        const uint8_t* cs = sm + ps.st.idx * stage_b + u * sub_b + NTOK * 128;
         if constexpr (FMT == FMT_INT) {
-          if (first) {
+          if (((c.kc0 + i) * 64) % GROUP == 0) {
             const uint32_t sz = lds_u32(smem_u32(cs + cbytes) + 4 * row);
-            // (1024, 1024), (z, z) against chunk 0's (-XP_hi, -XP_lo), (-X_hi, -X_lo),
-            // and for two-chunk groups again against chunk 1's (zeros otherwise:
-            // those slots may hold another expert's sums from an earlier forward)
-            const uint32_t zz = prmt(sz, sz, 0x3232u);
-            const uint32_t cz[4] = {kOne1024, zz, GROUP > 64 ? kOne1024 : 0u, GROUP > 64 ? zz : 0u};
-            tmem_st4_nw(ta + 32, cz);
+            dq_s2 = prmt(sz, sz, 0x1010u);
+            dq_n2 = hmul2u(hneg2u(prmt(sz, sz, 0x3232u)), dq_s2);
           }
           const uint32_t blk = smem_u32(cs);
           uint32_t w0[4], w1[4], r0[16], r1[16];
@@ -311,10 +289,13 @@ __device__ void unpack(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, ui
           lds_half_words_int<BITS>(blk, row, 1, w1);
           int_raw_half<BITS>(w0, r0);
           int_raw_half<BITS>(w1, r1);
+          uint32_t d0[16], d1[16];
+          int_dequant_half<BITS>(r0, dq_s2, dq_n2, d0);
+          int_dequant_half<BITS>(r1, dq_s2, dq_n2, d1);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            v[j] = r0[j];
-            v[16 + j] = r1[j];
+            v[j] = d0[j];
+            v[16 + j] = d1[j];
           }
         } else if constexpr (FMT == FMT_BITPLANE) {
 #pragma unroll
@@ -356,29 +337,13 @@ __device__ void epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
   const int row = threadIdx.x - 32 * kDqWarps;  // 0..127 = TMEM lane
   const uint32_t lane_base = (uint32_t)(row & ~31) << 16;
   const int R = c.rb * kRows + row;
-  // the part's groups: main chunks [ib, min(ie, nmain)), then the compensator if ie > nmain
-  const int me = min(c.ie, c.nmain);
-  int nmain_groups = 0;
-  if constexpr (FMT == FMT_INT) nmain_groups = max(0, me - c.ib) / (GROUP / 64);
-  else nmain_groups = me > c.ib ? 1 : 0;
-  const int ncomp = c.ie > c.nmain ? 1 : 0;
-  const int g0 = (FMT == FMT_INT) ? (c.kc0 + c.ib) / (GROUP / 64) : 0;
+  // the part's accumulators: one over its main chunks [ib, min(ie, nmain)),
+  // then the compensator's if ie > nmain (both added with weight 1)
+  const int nacc = (min(c.ie, c.nmain) > c.ib ? 1 : 0) + (c.ie > c.nmain ? 1 : 0);
   float y[NTOK];
 #pragma unroll
   for (int t = 0; t < NTOK; ++t) y[t] = 0.f;
-  // the row's group scales, loaded kPre groups ahead of their use (they come
-  // from L2: the producer's copies of the same words went through it)
-  constexpr int kPre = 3;
-  uint32_t pre[kPre];
-#pragma unroll
-  for (int q = 0; q < kPre; ++q)
-    pre[q] = (FMT == FMT_INT && q < nmain_groups) ? d.sz[(long long)(g0 + q) * a.M + R] : 0x3C00u;
-  for (int gi = 0; gi < nmain_groups + ncomp; ++gi) {
-    float s = 1.f;
-    if (FMT == FMT_INT && gi < nmain_groups) s = __half2float(__ushort_as_half((uint16_t)(pre[0] & 0xFFFFu)));
-#pragma unroll
-    for (int q = 0; q < kPre - 1; ++q) pre[q] = pre[q + 1];
-    pre[kPre - 1] = (FMT == FMT_INT && gi + kPre < nmain_groups) ? d.sz[(long long)(g0 + gi + kPre) * a.M + R] : 0x3C00u;
+  for (int gi = 0; gi < nacc; ++gi) {
     if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait_fast(accfull + 8 * ps.acc.idx, ps.acc.ph, a.status, a.wait_ns))) {
       *abort_flag = 1;
       return;
@@ -387,7 +352,7 @@ __device__ void epilogue(const DecodeArgs& a, const BlockDesc& d, const Ctx& c, 
     uint32_t v[NTOK];
     tmem_ld<NTOK>(tmem + lane_base + ps.acc.idx * NTOK, v);
 #pragma unroll
-    for (int t = 0; t < NTOK; ++t) y[t] = fmaf(s, __uint_as_float(v[t]), y[t]);
+    for (int t = 0; t < NTOK; ++t) y[t] += __uint_as_float(v[t]);
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(accfree + 8 * ps.acc.idx);
@@ -505,13 +470,6 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  if (warp < 4) {
-    // constant correction columns of the A buffers: (1024, 1024), then zeros
-    const uint32_t lb = (uint32_t)(warp * 32) << 16;
-    const uint32_t cz[8] = {dk::kOne1024, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-    for (int b = 0; b < dk::kA * dk::kSub; ++b) tmem_st8_nw(tmem + lb + dk::kABase + b * dk::kACols + 32, cz);
-    tmem_wait_st();
-  }
   // everything above overlaps the previous kernel's tail
   pdl_wait();
   pdl_trigger();
@@ -665,27 +623,6 @@ __global__ void __launch_bounds__(dk::kThreads, 2) decode_gemm_kernel(const __gr
     tc_fence_after();
     tmem_dealloc(tmem, dk::kTmemCols);
   }
-}
-
-// ---------------------------------------------------------------------------
-// per-group correction sums (one warp per routed row x group)
-
-__global__ void __launch_bounds__(256) act_corr_kernel(const CorrArgs a) {
-  pdl_wait();
-  pdl_trigger();
-  act_corr_rows(a, blockIdx.y, blockIdx.x, gridDim.x);
-}
-
-int act_corr_ctas(int rows_per_expert, int K) {
-  const long long items = (long long)rows_per_expert * (K / 64);
-  return (int)std::max<long long>(1, std::min<long long>((items + 7) / 8, 256));
-}
-
-cudaError_t launch_act_corr(const CorrArgs& a, int rows_per_expert, int grid_y, cudaStream_t st, int* launches) {
-  const cudaError_t err =
-      launch_kernel(act_corr_kernel, dim3(act_corr_ctas(rows_per_expert, a.K), grid_y), dim3(256), 0, st, true, a);
-  if (launches) ++*launches;
-  return err;
 }
 
 static int num_sms() {

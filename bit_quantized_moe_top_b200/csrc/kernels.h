@@ -55,15 +55,11 @@ struct RouteArgs {
   int* flag;                  // [1] set to epoch once the scan is done
   unsigned epoch;             // nonzero, different for every forward of the layer
   int nb, gs;                 // token blocks of 16, K slices of the gather
-  const ExpertDesc* experts;  // W1 descriptors (bits, group, format) for the correction sums
-  __half* corr;               // per-chunk correction sums of the gathered rows, or null
-  long long ldc;
   unsigned long long wait_ns; // limit of the wait for the scan
 };
 
 struct DecodeArgs {
   CUtensorMap tmap_act;       // activations [rows, Kpad] fp16 row-major; box 64 x 16, 128-byte swizzle
-  CUtensorMap tmap_corr;      // per-group correction columns [rows, 16 * groups] fp16; box 16 x 16, 32-byte swizzle
   const ExpertDesc* experts;
   int block;                  // 0 = W1, 1 = W2
   const int* active;
@@ -90,29 +86,7 @@ struct DecodeArgs {
   int mixed;                  // the experts' blocks differ (bits, format, group or rank): tiles dealt round-robin
 };
 
-// Per-chunk correction columns of the activations for the integer-code
-// decode GEMM: for routed row p and 64-column chunk c of group g (cpg chunks
-// per group), corr[p][16g + 4(c % cpg) .. +3] = (-XP_hi, -XP_lo, -X_hi, -X_lo)
-// in fp16, with XP = sum_k (P_k / 1024) x_pk and X = sum_k x_pk over the
-// chunk, each split into an fp16 value and its fp16 remainder.
-struct CorrArgs {
-  const ExpertDesc* experts;
-  int block;
-  const int* active;
-  const int* n_active;
-  const int* counts;
-  const int* poffsets;
-  const __half* act;          // activations [rows, lda] fp16
-  long long lda;
-  int K;                      // input features of the block
-  __half* corr;               // [rows, ldc] fp16
-  long long ldc;
-  unsigned* status;
-};
-
 struct LowrankArgs {
-  CorrArgs corr;              // corr.act != nullptr: CTAs past the low-rank grid compute correction sums
-  int corr_ctas;
   const ExpertDesc* experts;
   int block;
   const int* active;
@@ -157,8 +131,6 @@ struct TileqArgs {
   const __half* c16;          // cores [E][P][Q][r (output i)][r (input j)], fp16
   float* z;                   // [sources][Q][r]
   int comp_top_n;             // > 0: routed rows in slots >= comp_top_n get u = 0
-  CorrArgs corr;              // corr.act != nullptr: CTAs past the z grid compute the correction sums
-  int corr_ctas;
 };
 
 struct PrefillArgs {
@@ -211,8 +183,6 @@ int route_num_blocks(int T);
 int route_gather_slices(int T, int K);
 int device_sms();
 
-cudaError_t launch_act_corr(const CorrArgs& a, int rows_per_expert, int grid_y, cudaStream_t st, int* launches);
-int act_corr_ctas(int rows_per_expert, int K);
 int decode_rows_per_cta();
 int decode_ctas();
 cudaError_t launch_decode_gemm(const DecodeArgs& a, int ntok, int maxbits, int grid_y, cudaStream_t st,

@@ -9,7 +9,7 @@
 // combine_kernel: y_t = sum_j w[t, j] * o_(t, j), slots in a fixed order, the
 // K-split partials of o summed first; bf16 out.
 #include "kernels.h"
-#include "corr.cuh"
+#include "common.cuh"
 
 namespace moeq {
 
@@ -65,12 +65,6 @@ __global__ void __launch_bounds__(kLrWarps * 32, 7) lowrank_kernel(LowrankArgs a
   pdl_wait();
   pdl_trigger();
   const int slot = blockIdx.y;
-  const int lr_ctas = a.KS * a.tiles;
-  if ((int)blockIdx.x >= lr_ctas) {
-    // the same launch also computes the decode GEMM's correction sums
-    act_corr_rows(a.corr, slot, blockIdx.x - lr_ctas, a.corr_ctas);
-    return;
-  }
   if (slot >= *a.n_active) return;
   const int e = a.active[slot];
   const int n_e = a.counts[e];
@@ -195,7 +189,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 }
 
 cudaError_t launch_lowrank(const LowrankArgs& a, int grid_y, cudaStream_t st, int* launches) {
-  dim3 grid(a.KS * a.tiles + (a.corr.act ? a.corr_ctas : 0), grid_y);
+  dim3 grid(a.KS * a.tiles, grid_y);
   const cudaError_t err = launch_kernel(lowrank_kernel, grid, dim3(kLrWarps * 32), 0, st, true, a);
   if (launches) ++*launches;
   return err;

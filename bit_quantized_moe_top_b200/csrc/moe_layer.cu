@@ -101,14 +101,12 @@ struct moe_layer {
     DevBuf brow, v, ct, z;  // v: V [r][Kin] in the z MMA's operand type (W1 bf16, W2 fp16); ct: cores, fp16
   } tq[2];
   DevBuf block_counts, block_base, pblock_base, sem, status;
-  DevBuf xact, zact, obuf, part, corr_x, corr_z;
+  DevBuf xact, zact, obuf, part;
   DevBuf sk_part, sk_flag;  // decode GEMM tiles split between two CTAs: partial sums, flags
   unsigned sk_epoch = 0;
-  int ldc_x = 0, ldc_z = 0;  // correction columns per row: 16 per group of 64 (the smallest group)
   DevBuf hx, hl, hy;  // device buffers for forward_host
   CUtensorMap tmap_x, tmap_z;    // activation buffers, 128-row boxes (prefill GEMMs)
   CUtensorMap tmap_xd, tmap_zd;  // activation buffers, 16-row boxes (decode GEMMs)
-  CUtensorMap tmap_cx, tmap_cz;  // correction columns, 16 x 16 boxes (decode GEMMs)
   bool have_tmaps = false;
   int last_T = 0, last_k = 0, last_launches = 0;
   cudaStream_t last_stream = nullptr;
@@ -251,7 +249,7 @@ void moe_layer_destroy(moe_layer_t* L) {
   DevBuf* bufs[] = {&L->d_experts, &L->idx, &L->w, &L->counts, &L->offsets, &L->poffsets, &L->active,
                     &L->n_active, &L->ticket, &L->flag, &L->perm, &L->inv_pos, &L->pinv, &L->pslot, &L->ptok, &L->block_counts,
                     &L->block_base, &L->pblock_base, &L->sem, &L->status, &L->xact, &L->zact, &L->obuf,
-                    &L->part, &L->corr_x, &L->corr_z, &L->hx, &L->hl, &L->hy, &L->sk_part, &L->sk_flag};
+                    &L->part, &L->hx, &L->hl, &L->hy, &L->sk_part, &L->sk_flag};
   for (DevBuf* b : bufs) dfree(*b);
   for (cudaEvent_t ev : L->events) cudaEventDestroy(ev);
   if (L->fwd_done) cudaEventDestroy(L->fwd_done);
@@ -337,12 +335,8 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   A(L->zact, sizeof(__half) * (size_t)L->rows_pad_max * L->Kpad_z);
   A(L->obuf, sizeof(float) * (size_t)o_elems * K);
   A(L->part, sizeof(float) * (size_t)L->kslr_max * L->rows_pad_max * kMaxRank);
-  L->ldc_x = 16 * (K / 64);
-  L->ldc_z = 16 * (N / 64);
   A(L->sk_part, sizeof(float) * (size_t)decode_ctas() * decode_rows_per_cta() * 32);
   A(L->sk_flag, sizeof(unsigned) * (size_t)decode_ctas());
-  A(L->corr_x, sizeof(__half) * (size_t)L->rows_pad_max * L->ldc_x);
-  A(L->corr_z, sizeof(__half) * (size_t)L->rows_pad_max * L->ldc_z);
   A(L->hx, sizeof(__nv_bfloat16) * (size_t)max_tokens * K);
   A(L->hl, sizeof(float) * (size_t)max_tokens * E);
   A(L->hy, sizeof(__nv_bfloat16) * (size_t)max_tokens * K);
@@ -351,8 +345,8 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
     return st;
   }
   cudaError_t ce = cudaSuccess;
-  DevBuf* zero[] = {&L->ticket, &L->flag, &L->sem, &L->status, &L->xact, &L->zact, &L->n_active, &L->counts, &L->corr_x,
-                    &L->corr_z, &L->sk_flag};
+  DevBuf* zero[] = {&L->ticket, &L->flag, &L->sem, &L->status, &L->xact, &L->zact, &L->n_active, &L->counts,
+                    &L->sk_flag};
   for (DevBuf* b : zero)
     if (ce == cudaSuccess) ce = cudaMemset(b->p, 0, b->n);
   if (ce == cudaSuccess)
@@ -366,9 +360,7 @@ moe_status_t moe_layer_create(int E, int K, int N, int max_tokens, int max_top_k
   L->have_tmaps = encode_act_map(&L->tmap_x, L->xact.p, L->Kpad_x, L->rows_pad_max, 128) &&
                   encode_act_map(&L->tmap_z, L->zact.p, L->Kpad_z, L->rows_pad_max, 128) &&
                   encode_act_map(&L->tmap_xd, L->xact.p, L->Kpad_x, L->rows_pad_max, 16) &&
-                  encode_act_map(&L->tmap_zd, L->zact.p, L->Kpad_z, L->rows_pad_max, 16) &&
-                  encode_map(&L->tmap_cx, L->corr_x.p, L->ldc_x, L->rows_pad_max, 16, 16, CU_TENSOR_MAP_SWIZZLE_32B) &&
-                  encode_map(&L->tmap_cz, L->corr_z.p, L->ldc_z, L->rows_pad_max, 16, 16, CU_TENSOR_MAP_SWIZZLE_32B);
+                  encode_act_map(&L->tmap_zd, L->zact.p, L->Kpad_z, L->rows_pad_max, 16);
   if (!L->have_tmaps) {
     moe_layer_destroy(L);
     return MOE_ERR_CUDA;
@@ -835,7 +827,6 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int E = L->E, K = L->K, N = L->N;
   int maxbits[2] = {0, 0}, rmax = 0;
-  bool any_int[2] = {false, false};
   bool uniform[2] = {true, true};
   for (int e = 1; e < E; ++e)
     for (int b = 0; b < 2; ++b) {
@@ -847,7 +838,6 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     for (int b = 0; b < 2; ++b) {
       const int bb = L->hdesc[e].blk[b].bits;
       maxbits[b] = bb > maxbits[b] ? bb : maxbits[b];
-      any_int[b] = any_int[b] || L->hdesc[e].blk[b].fmt == FMT_INT;
     }
     rmax = L->hdesc[e].blk[0].rank > rmax ? L->hdesc[e].blk[0].rank : rmax;
   }
@@ -889,55 +879,16 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
   ra.epoch = L->route_epoch;
   ra.nb = route_num_blocks(T);
   ra.gs = route_gather_slices(T, K);
-  ra.experts = dexp;
-  // the decode GEMM's correction sums of the gathered rows (integer-code W1 blocks)
-  ra.corr = (!prefill && any_int[0]) ? static_cast<__half*>(L->corr_x.p) : nullptr;
-  ra.ldc = L->ldc_x;
   ra.wait_ns = L->wait_ns;
   L->prof_names.clear();
   prof_mark(L, st, "route");
   ce = launch_route_fused(ra, device_sms(), st, &launches);
 
   const long long prows = (rows + 7LL * E + 7) / 8 * 8;
-  // per-group correction sums of a block's input rows (decode path, integer-code blocks)
-  auto make_corr = [&](int block, const __half* act, long long lda, int Kin, __half* corr, long long ldc) {
-    CorrArgs ca{};
-    if (prefill || !any_int[block]) return ca;  // ca.act == nullptr: nothing to compute
-    ca.experts = dexp;
-    ca.block = block;
-    ca.active = ra.active;
-    ca.n_active = ra.n_active;
-    ca.counts = ra.counts;
-    ca.poffsets = ra.poffsets;
-    ca.act = act;
-    ca.lda = lda;
-    ca.K = Kin;
-    ca.corr = corr;
-    ca.ldc = ldc;
-    ca.status = ra.status;
-    return ca;
-  };
-  // correction-sum CTAs are sized for twice an expert's mean share of the
-  // routed rows (they loop over their items when an expert holds more)
-  const int corr_rows = (int)std::min<long long>(T, 2 * ((rows + grid_y - 1) / grid_y));
-  // correction-sum CTAs per expert slot, at most about 2048 over all slots:
-  // sized for one expert taking every token, the count grows with E while
-  // most slots hold a few rows (the CTAs loop over their items)
-  const int corr_cap = std::max(8, std::min(256, 2048 / std::max(1, grid_y)));
-  // the low-rank down-projection, with the correction sums in the same launch
-  auto lowrank = [&](int block, __half* act, int Kpad, int Kin, const CorrArgs& corr) {
-    if (ce != cudaSuccess) return;
-    if (rmax == 0) {
-      // a block type with tiled shared compensators computes the sums in its z launch
-      if (corr.act && !L->tq[block].on) {
-        prof_mark(L, st, block == 0 ? "act_corr_w1" : "act_corr_w2");
-        ce = launch_act_corr(corr, corr_rows, grid_y, st, &launches);
-      }
-      return;
-    }
+  // the low-rank down-projection U = V A^T of a block's routed rows
+  auto lowrank = [&](int block, __half* act, int Kpad, int Kin) {
+    if (ce != cudaSuccess || rmax == 0) return;
     LowrankArgs la{};
-    la.corr = corr;
-    la.corr_ctas = corr.act ? std::min(act_corr_ctas(corr_rows, Kin), corr_cap) : 0;
     la.experts = dexp;
     la.block = block;
     la.active = ra.active;
@@ -965,16 +916,10 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     ce = launch_lowrank(la, grid_y, st, &launches);
   };
   // a block type's shared 2D-tiled compensator: z = V x, u = C z
-  auto tileq = [&](int block, const CorrArgs& corr) {
+  auto tileq = [&](int block) {
     const auto& t = L->tq[block];
     if (ce != cudaSuccess || !t.on) return;
     TileqArgs ta{};
-    if (rmax == 0 && corr.act) {
-      // no low-rank launch carries the correction sums: the z launch does
-      ta.corr = corr;
-      // twice the standalone kernel's CTAs: these CTAs have half its threads
-      ta.corr_ctas = 2 * std::min(act_corr_ctas(corr_rows, block == 0 ? K : N), corr_cap);
-    }
     ta.mode = block;
     ta.x = static_cast<const __nv_bfloat16*>(X);
     ta.act = static_cast<__half*>(block == 0 ? L->xact.p : L->zact.p);
@@ -1000,9 +945,9 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     prof_mark(L, st, block == 0 ? "tileq_w1" : "tileq_w2");
     ce = launch_tileq(ta, grid_y, st, &launches);
   };
-  // W1 side compensator U1 = X A1^T (the routing kernel computed X's correction sums)
-  lowrank(0, static_cast<__half*>(L->xact.p), L->Kpad_x, K, CorrArgs{});
-  tileq(0, CorrArgs{});
+  // W1 side compensator U1 = X A1^T
+  lowrank(0, static_cast<__half*>(L->xact.p), L->Kpad_x, K);
+  tileq(0);
   int ks2 = 1;
   if (prefill) {
     // tcgen05 path: one launch per block, CTAs over (row tile, 256-token pair, expert)
@@ -1030,8 +975,8 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
       ce = launch_prefill_gemm(pa, pairs, grid_y, st, &launches);
     };
     prefill_gemm(0, L->tmap_x, K, 2 * N, MODE_SWIGLU);
-    lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N, CorrArgs{});
-    tileq(1, CorrArgs{});
+    lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N);
+    tileq(1);
     prefill_gemm(1, L->tmap_z, N, K, MODE_OUT);
   } else {
     // tokens per pass: cover the expected per-expert batch (mean + 3 sd);
@@ -1040,13 +985,11 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
     const int want = (int)std::ceil(avg + 3.0 * std::sqrt(avg) + 1.0);
     // (larger batches take more passes, run as separate tiles that share the weights through L2)
     const int ntok = std::min(T, want) <= 16 ? 16 : 32;
-    auto decode_gemm = [&](int block, const CUtensorMap& map, const CUtensorMap& cmap, int Kin, int M, int mode,
-                           int KS) {
+    auto decode_gemm = [&](int block, const CUtensorMap& map, int Kin, int M, int mode, int KS) {
       if (ce != cudaSuccess) return;
       DecodeArgs da;
       std::memset(&da, 0, sizeof(da));
       da.tmap_act = map;
-      da.tmap_corr = cmap;
       da.experts = dexp;
       da.block = block;
       da.active = ra.active;
@@ -1075,11 +1018,9 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
       prof_mark(L, st, block == 0 ? "decode_gemm_w1_swiglu" : "decode_gemm_w2");
       ce = launch_decode_gemm(da, ntok, maxbits[block], grid_y, st, &launches);
     };
-    decode_gemm(0, L->tmap_xd, L->tmap_cx, K, 2 * N, MODE_SWIGLU, 1);
-    const CorrArgs corr2 =
-        make_corr(1, static_cast<const __half*>(L->zact.p), L->Kpad_z, N, static_cast<__half*>(L->corr_z.p), L->ldc_z);
-    lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N, corr2);
-    tileq(1, corr2);
+    decode_gemm(0, L->tmap_xd, K, 2 * N, MODE_SWIGLU, 1);
+    lowrank(1, static_cast<__half*>(L->zact.p), L->Kpad_z, N);
+    tileq(1);
     // split the down projection's K (fixed-order sum of the partials in the
     // combine); splits at least 256 columns wide, and at least one split.
     // With tiles split between CTAs, only until there are at least as many
@@ -1102,7 +1043,7 @@ moe_status_t moe_layer_forward(moe_layer_t* L, const void* X, const float* logit
       }
     }
     if (rows > 1024) ks2 = 1;
-    decode_gemm(1, L->tmap_zd, L->tmap_cz, N, K, MODE_OUT, ks2);
+    decode_gemm(1, L->tmap_zd, N, K, MODE_OUT, ks2);
   }
   if (ce == cudaSuccess) {
     CombineArgs ca{};

@@ -1,8 +1,6 @@
 // Routing: top-k softmax per token, per-expert histogram, exclusive scan and a
 // stable token permutation (expert-major, token-ascending), plus the gather of
-// routed token rows into the activation layout of the expert GEMMs and, for
-// the decode GEMM's integer-code blocks, the per-chunk correction sums of the
-// gathered rows.
+// routed token rows into the activation layout of the expert GEMMs.
 //
 // Top-k per token follows the routing of the Bandwidth-Efficient Adaptive
 // Mixture-of-Experts via Low-Rank Compensation page (abstract: each token has
@@ -20,7 +18,7 @@
 #include <algorithm>
 
 #include "kernels.h"
-#include "corr.cuh"
+#include "common.cuh"
 
 namespace moeq {
 
@@ -203,9 +201,8 @@ __device__ __forceinline__ void st_release_gpu(int* p, int v) {
 
 // Phase B item: ranks of block b's routed pairs from per-expert token
 // bitmasks, the permutation (slice 0 only), and the gather of chunks
-// [c0, c1) of the block's routed rows (bf16 -> fp16) with, where asked, the
-// per-chunk correction sums of the integer-code W1 blocks.
-__device__ void permute_item(const RouteArgs& a, int b, int ks, unsigned* mask, int* prow_s, int* exp_s) {
+// [c0, c1) of the block's routed rows (bf16 -> fp16).
+__device__ void permute_item(const RouteArgs& a, int b, int ks, unsigned* mask, int* prow_s) {
   const int t0 = b * kRouteTokensPerCta;
   const int nt = min(kRouteTokensPerCta, a.T - t0);
   const int rows = nt * a.k;
@@ -225,7 +222,6 @@ __device__ void permute_item(const RouteArgs& a, int b, int ks, unsigned* mask, 
     const long long bi = (long long)b * a.E + e;
     const int ppos = __ldcg(a.pblock_base + bi) + rank;
     prow_s[i] = ppos;
-    exp_s[i] = e;
     if (ks == 0) {
       a.pslot[ppos] = j;
       a.ptok[ppos] = t;
@@ -263,7 +259,6 @@ __device__ void permute_item(const RouteArgs& a, int b, int ks, unsigned* mask, 
       const int q8 = it & 7, pc = it >> 3;
       const int i = valid ? pc / nch : 0, c = c0 + (valid ? pc % nch : 0);
       const long long prow = prow_s[i];
-      float xs = 0.f, xp = 0.f;
       if (valid) {
         const __nv_bfloat162* bv = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
         uint32_t v[4];
@@ -271,36 +266,6 @@ __device__ void permute_item(const RouteArgs& a, int b, int ks, unsigned* mask, 
         for (int q = 0; q < 4; ++q) v[q] = pack_half2(__bfloat162float(bv[q].x), __bfloat162float(bv[q].y));
         *reinterpret_cast<uint4*>(reinterpret_cast<__half*>(a.act) + prow * a.Kpad + 64 * c + 8 * q8) =
             make_uint4(v[0], v[1], v[2], v[3]);
-        if (a.corr) {
-          const BlockDesc& d = a.experts[exp_s[i]].blk[0];
-          if (d.fmt == FMT_INT) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const __half2 h = *reinterpret_cast<const __half2*>(&v[q]);
-              const float x0 = __low2float(h), x1 = __high2float(h);
-              xs += x0 + x1;
-              xp = fmaf(int_pfac(d.bits, 8 * q8 + 2 * q), x0, xp);
-              xp = fmaf(int_pfac(d.bits, 8 * q8 + 2 * q + 1), x1, xp);
-            }
-          }
-        }
-      }
-      if (a.corr) {
-        // warp-uniform: every lane takes part in the shuffles
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
-          xs += __shfl_xor_sync(0xffffffffu, xs, o);
-          xp += __shfl_xor_sync(0xffffffffu, xp, o);
-        }
-        if (valid && q8 == 0) {
-          const BlockDesc& d = a.experts[exp_s[i]].blk[0];
-          if (d.fmt == FMT_INT) {
-            const int cpg = d.group / 64;
-            const int g = c / cpg, cc = c % cpg;
-            *reinterpret_cast<uint2*>(a.corr + prow * a.ldc + 16 * g + 4 * cc) =
-                make_uint2(corr_pair(xp, a.status), corr_pair(xs, a.status));
-          }
-        }
       }
     }
   }
@@ -313,7 +278,6 @@ __global__ void __launch_bounds__(kRouteThreads) route_fused_kernel(RouteArgs a)
   __shared__ int seg[kMaxExperts > kRouteThreads ? kMaxExperts : kRouteThreads];
   __shared__ unsigned mask[kMaxExperts];
   __shared__ int prow_s[kRouteTokensPerCta * kMaxTopK];
-  __shared__ int exp_s[kRouteTokensPerCta * kMaxTopK];
   __shared__ int is_last, go;
   pdl_wait();
   pdl_trigger();
@@ -353,9 +317,9 @@ __global__ void __launch_bounds__(kRouteThreads) route_fused_kernel(RouteArgs a)
   }
   __syncthreads();
   if (!go) return;
-  // ---- phase B: permutation, gather, correction sums
+  // ---- phase B: permutation, gather
   for (int item = blockIdx.x; item < a.nb * a.gs; item += gridDim.x)
-    permute_item(a, item / a.gs, item % a.gs, mask, prow_s, exp_s);
+    permute_item(a, item / a.gs, item % a.gs, mask, prow_s);
 }
 
 int route_num_blocks(int T) { return (T + kRouteTokensPerCta - 1) / kRouteTokensPerCta; }

@@ -17,7 +17,6 @@
 // [Kin, r] per column tile (the tile's K range split over four warps, partial
 // sums added in a fixed order). u: per (row tile, expert) [rows, Q r] x
 // [Q r, r], with z rounded to fp16 as the A operand and the fp16 cores as B.
-#include "corr.cuh"
 #include "kernels.h"
 
 namespace moeq {
@@ -34,19 +33,14 @@ __device__ __forceinline__ void mma_16816_bf16(float (&d)[4], const uint32_t (&a
 }
 }  // namespace
 
-// grid (Q + corr CTAs, max(ceil(sources / (16 MT)), corr slots)), kZWarps
-// warps: warp w covers the w-th quarter of column tile q's K range for the
-// CTA's 16 MT source rows (MT m-tiles share each load of V). CTAs past Q
-// compute the decode GEMM's correction sums in the same launch.
+// grid (Q, ceil(sources / (16 MT))), kZWarps warps: warp w covers the w-th
+// quarter of column tile q's K range for the CTA's 16 MT source rows (MT
+// m-tiles share each load of V).
 template <int MODE, int MT>
 __global__ void __launch_bounds__(kZWarps * 32) tileq_z_kernel(const TileqArgs a) {
   __shared__ float red[kZWarps][16 * MT][33];
   pdl_wait();
   pdl_trigger();
-  if ((int)blockIdx.x >= a.Q) {
-    act_corr_rows(a.corr, blockIdx.y, blockIdx.x - a.Q, a.corr_ctas);
-    return;
-  }
   const int q = blockIdx.x;
   const int nsrc = MODE == 0 ? a.T : a.T * a.k;
   const int s0 = blockIdx.y * 16 * MT;
@@ -245,8 +239,8 @@ cudaError_t launch_tileq(const TileqArgs& a, int grid_y, cudaStream_t st, int* l
   const int nsrc = a.mode == 0 ? a.T : a.T * a.k;
   const bool big = nsrc >= 512;
   const int mt = big ? 4 : 1;
-  const int zy = std::max((nsrc + 16 * mt - 1) / (16 * mt), a.corr.act ? grid_y : 0);
-  const dim3 zg(a.Q + (a.corr.act ? a.corr_ctas : 0), zy);
+  const int zy = (nsrc + 16 * mt - 1) / (16 * mt);
+  const dim3 zg(a.Q, zy);
   const dim3 zb(kZWarps * 32);
   cudaError_t err;
   if (a.mode == 0)
