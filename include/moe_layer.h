@@ -62,12 +62,9 @@
  *   - One layer is used from one stream at a time.
  *   - Arithmetic: fp16 tensor-core operands (X, the SwiGLU output and the
  *     compensator terms are rounded to fp16, the tiled compensators' inner
- *     projections and cores too; dequantised weights too on the
- *     prefill path, while the decode path multiplies the exact integer codes
- *     and applies scale and zero per group in fp32), fp32 accumulation, bf16
- *     output. |X| and |z| must stay below 65504, and on the decode path of an
- *     INT_ASYM block so must the sum of |x| over each quantisation group
- *     (otherwise moe_layer_sync_status reports MOE_ERR_DEVICE_CHECK).
+ *     projections and cores too, and the dequantised weights (q - z) * s on
+ *     both paths), fp32 accumulation, bf16 output. |X|, |z| and |z * s| must
+ *     stay below 65504.
  */
 #ifndef MOE_LAYER_H
 #define MOE_LAYER_H
