@@ -32,7 +32,7 @@ constexpr int kMaxExperts = 256;
 enum : int { FMT_INT = 0, FMT_BITPLANE = 1, FMT_DENSE = 2 };
 
 // device status word bits
-enum : unsigned { ST_BOUNDS = 1u, ST_TIMEOUT = 2u, ST_ROUTE = 4u };
+enum : unsigned { ST_BOUNDS = 1u, ST_TIMEOUT = 2u, ST_ROUTE = 4u, ST_RANGE = 8u };
 
 // One expert linear block as the kernels see it.
 struct BlockDesc {
